@@ -1,0 +1,183 @@
+"""Float64 CPU oracle for decode context parallelism (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU
+baseline and reference arm) may import this package.  It shares no code with
+the CUDA library; its only common dependency is the seeded input generator in
+``synth``, which draws numbers and holds none of the method's arithmetic.
+
+The C source ``oracle.c`` holds every computation; this module compiles it
+with gcc on first use (or through ``build()``) and marshals numpy arrays.
+Function-level citations are in ``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+_lock = threading.Lock()
+
+GQA, MLA = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (plain gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", tmp,
+                               _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = C.CDLL(build())
+            p = C.c_void_p
+            lib.oracle_token_shard.restype = C.c_int
+            lib.oracle_token_shard.argtypes = [C.c_int64, C.c_int, C.c_int]
+            lib.oracle_token_local_block.restype = C.c_int64
+            lib.oracle_token_local_block.argtypes = [C.c_int64, C.c_int, C.c_int]
+            lib.oracle_block_tables.restype = C.c_int
+            lib.oracle_block_tables.argtypes = [p, C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_int, p, p, p]
+            lib.oracle_place_request.restype = None
+            lib.oracle_place_request.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                 C.c_int, p, C.c_int64, p, p]
+            lib.oracle_attend.restype = None
+            lib.oracle_attend.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, C.c_int64, p,
+                                          C.c_double, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, p]
+            lib.oracle_merge.restype = None
+            lib.oracle_merge.argtypes = [p, p, C.c_int, C.c_int64, C.c_int, p, p]
+            lib.oracle_merge_ml.restype = None
+            lib.oracle_merge_ml.argtypes = [p, p, p, C.c_int, C.c_int64, C.c_int, p]
+            lib.oracle_kv_bytes_per_token.restype = C.c_int64
+            lib.oracle_kv_bytes_per_token.argtypes = [C.c_int, C.c_int, C.c_int]
+            lib.oracle_validate_config.restype = C.c_int
+            lib.oracle_validate_config.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int]
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(C.c_void_p)
+
+
+# ---------------------------------------------------------------------------
+# sharding
+# ---------------------------------------------------------------------------
+def token_shard(t: int, block_size: int, D: int) -> int:
+    return _load().oracle_token_shard(t, block_size, D)
+
+
+def token_local_block(t: int, block_size: int, D: int) -> int:
+    return _load().oracle_token_local_block(t, block_size, D)
+
+
+def block_tables(seq_lens: Sequence[int], block_size: int, D: int, perm_seed: int = 0,
+                 max_local_blocks: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Returns ``(tables[D][B][max_local_blocks], local_len[D][B], num_pages[D])`` (int32)."""
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B = sl.shape[0]
+    if max_local_blocks is None:
+        nblk = (int(sl.max()) + block_size - 1) // block_size if B else 0
+        max_local_blocks = (nblk + D - 1) // D
+    tables = np.empty((D, B, max_local_blocks), dtype=np.int32)
+    local_len = np.empty((D, B), dtype=np.int32)
+    num_pages = np.empty((D,), dtype=np.int32)
+    rc = _load().oracle_block_tables(_ptr(sl), B, block_size, D, perm_seed, max_local_blocks, _ptr(tables),
+                                     _ptr(local_len), _ptr(num_pages))
+    if rc != 0:
+        raise ValueError(f"oracle_block_tables failed ({rc})")
+    return tables, local_len, num_pages
+
+
+def place(layout: int, Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray,
+          sources: List[np.ndarray], num_pages: np.ndarray, fill: int = 0xFFFF) -> List[np.ndarray]:
+    """Reference cache placement: returns D pools (uint16 bf16 bits), unused slots set to ``fill``."""
+    B = len(sources)
+    mlb = tables.shape[2]
+    page_elems = (2 * Hkv * block_size * d) if layout == GQA else (block_size * d)
+    pools = [np.full(int(num_pages[s]) * page_elems, fill, dtype=np.uint16) for s in range(D)]
+    arr = (C.c_void_p * D)(*[p.ctypes.data for p in pools])
+    t = np.ascontiguousarray(tables, dtype=np.int32)
+    for b, src in enumerate(sources):
+        src = np.ascontiguousarray(src, dtype=np.uint16)
+        _load().oracle_place_request(layout, Hkv, d, block_size, D, B, b, mlb, _ptr(t), src.shape[0], _ptr(src),
+                                     C.cast(arr, C.c_void_p))
+    return pools
+
+
+# ---------------------------------------------------------------------------
+# attention and merge
+# ---------------------------------------------------------------------------
+def attend(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
+           block_size: int = 1, D: int = 1, shard: int = -1, heads: Optional[Tuple[int, int]] = None
+           ) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention of one request (q bf16 bits [Hq][d_qk], src unsharded rows) -> (O[Hq][d_v], LSE[Hq]) f64.
+
+    ``shard < 0``: all tokens; otherwise only the tokens whose logical block
+    ``t // block_size`` is congruent to ``shard`` modulo ``D``.  Heads outside
+    ``heads = (begin, end)`` are left as NaN.
+    """
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    src = np.ascontiguousarray(src, dtype=np.uint16)
+    hb, he = heads if heads is not None else (0, Hq)
+    O = np.full((Hq, d_v), np.nan)
+    LSE = np.full((Hq,), np.nan)
+    _load().oracle_attend(layout, Hq, Hkv, d_qk, d_v, _ptr(q), src.shape[0], _ptr(src), scale, block_size, D,
+                          shard, hb, he, _ptr(O), _ptr(LSE))
+    return O, LSE
+
+
+def merge(O_parts: np.ndarray, LSE_parts: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """LSE-weighted merge. ``O_parts[D][rows][d_v]``, ``LSE_parts[D][rows]`` -> (O[rows][d_v], LSE[rows])."""
+    Op = np.ascontiguousarray(O_parts, dtype=np.float64)
+    Lp = np.ascontiguousarray(LSE_parts, dtype=np.float64)
+    D, rows, d_v = Op.shape
+    O = np.empty((rows, d_v))
+    LSE = np.empty((rows,))
+    _load().oracle_merge(_ptr(Op), _ptr(Lp), D, rows, d_v, _ptr(O), _ptr(LSE))
+    return O, LSE
+
+
+def merge_ml(U_parts: np.ndarray, m_parts: np.ndarray, l_parts: np.ndarray) -> np.ndarray:
+    """Merge in the local-max / local-sum form (unnormalised partial outputs)."""
+    U = np.ascontiguousarray(U_parts, dtype=np.float64)
+    m = np.ascontiguousarray(m_parts, dtype=np.float64)
+    l = np.ascontiguousarray(l_parts, dtype=np.float64)
+    D, rows, d_v = U.shape
+    O = np.empty((rows, d_v))
+    _load().oracle_merge_ml(_ptr(U), _ptr(m), _ptr(l), D, rows, d_v, _ptr(O))
+    return O
+
+
+def sharded(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
+            block_size: int, D: int, heads: Optional[Tuple[int, int]] = None):
+    """Per-shard partials followed by the merge: returns (O, LSE, O_parts[D], LSE_parts[D])."""
+    parts = [attend(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s, heads) for s in range(D)]
+    Op = np.stack([p[0] for p in parts])
+    Lp = np.stack([p[1] for p in parts])
+    hb, he = heads if heads is not None else (0, Hq)
+    O, LSE = merge(Op[:, hb:he], Lp[:, hb:he])
+    Of = np.full((Hq, d_v), np.nan)
+    Lf = np.full((Hq,), np.nan)
+    Of[hb:he], Lf[hb:he] = O, LSE
+    return Of, Lf, Op, Lp
+
+
+def kv_bytes_per_token(num_kv_heads: int, head_dim: int, elem_bytes: int) -> int:
+    return _load().oracle_kv_bytes_per_token(num_kv_heads, head_dim, elem_bytes)
+
+
+def validate_config(tp: int, dcp: int, num_kv_heads: int, layout: int) -> int:
+    return _load().oracle_validate_config(tp, dcp, num_kv_heads, layout)

@@ -1,0 +1,317 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+Every check here is independent of the oracle's own code: page-printed worked
+examples (tests/golden), closed forms, a library routine (torch's float64
+scaled_dot_product_attention, torch.logsumexp), brute force in extended
+precision without the max shift, and algebraic invariants of the merge.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import golden, golden_kv
+
+GQA, MLA = oracle.GQA, oracle.MLA
+
+
+# ---------------------------------------------------------------------------
+# sharding rule and tables
+# ---------------------------------------------------------------------------
+def test_interleave_example_from_page():
+    g = golden_kv("interleave_example.txt")
+    D = int(g["D"][0])
+    bs = 16
+    for blk in map(int, g["rank0_blocks"]):
+        assert oracle.token_shard(blk * bs, bs, D) == 0
+        assert oracle.token_shard(blk * bs + bs - 1, bs, D) == 0
+    for blk in map(int, g["rank1_blocks"]):
+        assert oracle.token_shard(blk * bs, bs, D) == 1
+    t = int(g["remap_global"][0]) * bs
+    assert oracle.token_shard(t, bs, D) == int(g["remap_rank"][0])
+    assert oracle.token_local_block(t, bs, D) == int(g["remap_local"][0])
+    total = int(g["even_split_total_blocks"][0])
+    _, _, num_pages = oracle.block_tables([total * bs], bs, D)
+    assert list(num_pages) == [int(g["even_split_per_rank"][0])] * D
+
+
+def test_tiny_tables_worked_by_hand():
+    tables, local_len, num_pages = oracle.block_tables([100, 257], 16, 2)
+    for row in golden("tiny_tables.txt"):
+        bar = row.index("|")
+        s, b, ntok = int(row[0]), int(row[1]), int(row[2])
+        gblocks = list(map(int, row[3:bar]))
+        pages = list(map(int, row[bar + 1:]))
+        assert local_len[s, b] == ntok
+        assert list(tables[s, b, :len(pages)]) == pages
+        assert all(x == -1 for x in tables[s, b, len(pages):])
+        for j, gb in enumerate(gblocks):  # local block j holds global block j*D + s
+            assert gb == j * 2 + s
+    assert list(num_pages) == [13, 11]
+
+
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("bs", [1, 16, 64])
+@pytest.mark.parametrize("perm", [0, 77])
+def test_tables_are_a_bijection(D, bs, perm):
+    rng = np.random.default_rng(D * 100 + bs + perm)
+    seq_lens = list(rng.integers(0, 700, size=7)) + [1, bs, bs + 1]
+    tables, local_len, num_pages = oracle.block_tables(seq_lens, bs, D, perm_seed=perm)
+    seen = [set() for _ in range(D)]
+    for b, n in enumerate(seq_lens):
+        assert int(local_len[:, b].sum()) == n
+        for t in range(n):
+            s = (t // bs) % D
+            page = tables[s, b, (t // bs) // D]
+            assert 0 <= page < num_pages[s]
+            key = (int(page), t % bs)
+            assert key not in seen[s]  # no slot holds two tokens
+            seen[s].add(key)
+    for s in range(D):  # every page of a shard is used, ids are 0..n-1
+        used = {p for p, _ in seen[s]}
+        assert used == set(range(int(num_pages[s])))
+
+
+def test_tables_capacity_error():
+    with pytest.raises(ValueError):
+        oracle.block_tables([100], 16, 2, max_local_blocks=3)
+
+
+def test_permutation_relabels_only():
+    seq_lens = [300, 5, 1000]
+    t0, l0, n0 = oracle.block_tables(seq_lens, 16, 4)
+    t1, l1, n1 = oracle.block_tables(seq_lens, 16, 4, perm_seed=12345)
+    assert (l0 == l1).all() and (n0 == n1).all()
+    assert ((t0 < 0) == (t1 < 0)).all()
+    assert not (t0 == t1).all()
+    for s in range(4):
+        a, b = t0[s][t0[s] >= 0], t1[s][t1[s] >= 0]
+        assert sorted(a) == sorted(b)
+
+
+def test_placement_roundtrip():
+    w = synth.custom(GQA, [37, 16, 1], 4, 2, 64, 64, 16, seed=9)
+    D = 3
+    tables, _, num_pages = oracle.block_tables(w.seq_lens, 16, D, perm_seed=5)
+    srcs = [w.kv_source(b) for b in range(w.batch)]
+    pools = oracle.place(GQA, 2, 64, 16, D, tables, srcs, num_pages, fill=0xFFFF)
+    used = [np.zeros(p.shape, bool) for p in pools]
+    for b, src in enumerate(srcs):
+        for t in range(src.shape[0]):
+            s = (t // 16) % D
+            page = tables[s, b, (t // 16) // D]
+            view = pools[s].reshape(-1, 2, 2, 16, 64)
+            assert (view[page, :, :, t % 16, :] == src[t]).all()
+            used[s].reshape(-1, 2, 2, 16, 64)[page, :, :, t % 16, :] = True
+    for s in range(D):
+        assert (pools[s][~used[s]] == 0xFFFF).all()
+
+
+# ---------------------------------------------------------------------------
+# arithmetic and configuration rules printed on the pages
+# ---------------------------------------------------------------------------
+def test_kv_size_13b_example():
+    g = golden_kv("kv_size_13b.txt")
+    per = oracle.kv_bytes_per_token(int(g["num_kv_heads"][0]), int(g["head_dim"][0]), int(g["elem_bytes"][0]))
+    assert per == int(g["bytes_per_token_per_layer"][0])
+    assert per * int(g["layers"][0]) == int(g["bytes_per_token"][0])
+    assert oracle.kv_bytes_per_token(8, 128, 2) == 4096  # the 70B-class GQA layer
+
+
+def test_validate_config_examples():
+    for row in golden("validate_config.txt"):
+        layout, tp, dcp, kvh, want = map(int, row)
+        assert oracle.validate_config(tp, dcp, kvh, layout) == want, row
+
+
+# ---------------------------------------------------------------------------
+# direct attention
+# ---------------------------------------------------------------------------
+def _f64(bits):
+    return synth.bf16_bits_to_f64(bits)
+
+
+def _torch_reference(layout, Hq, Hkv, d_qk, d_v, q, src, scale):
+    """torch float64 SDPA + logsumexp as an independent library reference."""
+    qd = torch.from_numpy(_f64(q))  # [Hq, d_qk]
+    if layout == GQA:
+        kv = torch.from_numpy(_f64(src))  # [n, 2, Hkv, d]
+        K = kv[:, 0].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)  # [Hq, n, d]
+        V = kv[:, 1].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    else:
+        c = torch.from_numpy(_f64(src))  # [n, d_qk]
+        K = c.unsqueeze(0).expand(Hq, -1, -1)
+        V = c[:, :d_v].unsqueeze(0).expand(Hq, -1, -1)
+    O = torch.nn.functional.scaled_dot_product_attention(qd.unsqueeze(1), K, V, scale=scale).squeeze(1)
+    S = torch.einsum("hd,hnd->hn", qd, K) * scale
+    return O.numpy(), torch.logsumexp(S, dim=1).numpy()
+
+
+@pytest.mark.parametrize("case", [
+    (GQA, 8, 2, 64, 64, 100), (GQA, 8, 8, 128, 128, 33), (GQA, 16, 2, 64, 64, 5), (GQA, 6, 3, 64, 64, 70),
+    (MLA, 4, 1, 576, 512, 90), (MLA, 64, 1, 576, 512, 17)])
+def test_attend_matches_torch_sdpa(case):
+    layout, Hq, Hkv, d_qk, d_v, n = case
+    w = synth.custom(layout, [n], Hq, Hkv, d_qk, d_v, 16, seed=n + Hq)
+    q, src = w.query(0), w.kv_source(0)
+    O, LSE = oracle.attend(layout, Hq, Hkv, d_qk, d_v, q, src, w.softmax_scale)
+    Ot, Lt = _torch_reference(layout, Hq, Hkv, d_qk, d_v, q, src, w.softmax_scale)
+    np.testing.assert_allclose(O, Ot, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE, Lt, rtol=1e-13, atol=1e-12)
+
+
+def test_attend_bruteforce_extended_precision():
+    # Naive softmax without the max shift, in x87 extended precision, on small scores.
+    w = synth.custom(GQA, [23], 4, 2, 64, 64, 16, seed=3, q_amp=0.25, kv_amp=0.25)
+    q, src = w.query(0), w.kv_source(0)
+    O, LSE = oracle.attend(GQA, 4, 2, 64, 64, q, src, 0.125)
+    qd = _f64(q).astype(np.longdouble)
+    kv = _f64(src).astype(np.longdouble)
+    for h in range(4):
+        kvh = h // 2
+        e = np.array([np.exp(np.longdouble(0.125) * np.dot(qd[h], kv[t, 0, kvh])) for t in range(23)])
+        o = (e[:, None] * kv[:, 1, kvh]).sum(0) / e.sum()
+        np.testing.assert_allclose(O[h], o.astype(np.float64), rtol=0, atol=1e-13)
+        assert abs(LSE[h] - float(np.log(e.sum()))) < 1e-13
+
+
+def test_closed_forms():
+    # seq_len 1: O = v_0, LSE = s_0.
+    w = synth.custom(GQA, [1], 4, 1, 64, 64, 16, seed=11)
+    q, src = w.query(0), w.kv_source(0)
+    O, LSE = oracle.attend(GQA, 4, 1, 64, 64, q, src, 0.5)
+    for h in range(4):
+        np.testing.assert_array_equal(O[h], _f64(src[0, 1, 0]))
+        assert LSE[h] == pytest.approx(0.5 * float(_f64(q[h]) @ _f64(src[0, 0, 0])), abs=1e-12)
+    # q = 0: uniform weights, O = mean of V, LSE = ln n.
+    w = synth.custom(MLA, [37], 2, 1, 576, 512, 64, seed=12)
+    src = w.kv_source(0)
+    O, LSE = oracle.attend(MLA, 2, 1, 576, 512, np.zeros((2, 576), np.uint16), src, 0.1)
+    np.testing.assert_allclose(O[0], _f64(src)[:, :512].mean(0), atol=1e-13)
+    assert LSE[1] == pytest.approx(math.log(37), abs=1e-14)
+    # all keys equal, values distinct: uniform weights again, O = mean(V), LSE = s + ln n.
+    w = synth.custom(GQA, [37], 2, 1, 64, 64, 16, seed=15)
+    q, src = w.query(0), w.kv_source(0).copy()
+    src[:, 0] = src[0, 0]
+    O, LSE = oracle.attend(GQA, 2, 1, 64, 64, q, src, 0.1)
+    s0 = 0.1 * float(_f64(q[1]) @ _f64(src[0, 0, 0]))
+    np.testing.assert_allclose(O[1], _f64(src[:, 1, 0]).mean(0), atol=1e-13)
+    assert LSE[1] == pytest.approx(s0 + math.log(37), abs=1e-12)
+    # one dominant score: O ~= v_j.
+    w = synth.custom(GQA, [50], 2, 1, 64, 64, 16, seed=13)
+    q, src = w.query(0), w.kv_source(0).copy()
+    j = 31
+    src[j, 0, 0] = q[0]  # key j = q, so s_j = scale*|q|^2 dominates by a huge margin
+    O, _ = oracle.attend(GQA, 2, 1, 64, 64, q, src, 10.0)
+    np.testing.assert_allclose(O[0], _f64(src[j, 1, 0]), atol=1e-12)
+
+
+def test_empty_token_set():
+    w = synth.custom(GQA, [16], 2, 1, 64, 64, 16, seed=14)
+    O, LSE = oracle.attend(GQA, 2, 1, 64, 64, w.query(0), w.kv_source(0), 0.1, block_size=16, D=2, shard=1)
+    assert (O == 0).all() and (LSE == -np.inf).all()
+
+
+# ---------------------------------------------------------------------------
+# sharded partials + merge == direct attention
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("bs", [1, 16, 64])
+def test_sharded_merge_equals_direct(D, bs):
+    for layout, Hq, Hkv, dqk, dv in [(GQA, 8, 2, 64, 64), (MLA, 4, 1, 576, 512)]:
+        w = synth.custom(layout, [257], Hq, Hkv, dqk, dv, bs, seed=D * 7 + bs)
+        q, src = w.query(0), w.kv_source(0)
+        O, LSE = oracle.attend(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale)
+        Om, Lm, Op, Lp = oracle.sharded(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, bs, D)
+        np.testing.assert_allclose(Om, O, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(Lm, LSE, rtol=0, atol=1e-12)
+        if D == 1:
+            np.testing.assert_array_equal(Op[0], O)
+
+
+def test_merge_worked_example():
+    g = golden_kv("merge_worked.txt")
+    Op = np.array([[list(map(float, g["O1"]))], [list(map(float, g["O2"]))]])
+    Lp = np.array([[float(g["LSE1"][0])], [math.log(float(g["LSE2_log_of"][0]))]])
+    O, LSE = oracle.merge(Op, Lp)
+    np.testing.assert_allclose(O[0], list(map(float, g["O"])), atol=1e-15)
+    assert LSE[0] == pytest.approx(math.log(float(g["LSE_log_of"][0])), abs=1e-15)
+    # the same instance through the local-max / local-sum form
+    U = np.array([[[1.0, 0.0]], [[0.0, 1.0]]])
+    m = np.array([[0.0], [math.log(3.0)]])
+    l = np.array([[1.0], [1.0]])
+    np.testing.assert_allclose(oracle.merge_ml(U, m, l)[0], [0.25, 0.75], atol=1e-15)
+
+
+def test_merge_invariants():
+    rng = np.random.default_rng(5)
+    Op = rng.standard_normal((4, 6, 16))
+    Lp = rng.standard_normal((4, 6)) * 5
+    O, LSE = oracle.merge(Op, Lp)
+    # D = 1 is the identity
+    O1, L1 = oracle.merge(Op[:1], Lp[:1])
+    np.testing.assert_array_equal(O1, Op[0])
+    np.testing.assert_array_equal(L1, Lp[0])
+    # adding a constant to every LSE_i leaves O unchanged and shifts LSE
+    O2, L2 = oracle.merge(Op, Lp + 1234.5)
+    np.testing.assert_allclose(O2, O, atol=1e-12)
+    np.testing.assert_allclose(L2, LSE + 1234.5, atol=1e-9)
+    # a -inf part is ignored
+    Lq = Lp.copy()
+    Lq[2] = -np.inf
+    O3, L3 = oracle.merge(Op, Lq)
+    O4, L4 = oracle.merge(Op[[0, 1, 3]], Lp[[0, 1, 3]])
+    np.testing.assert_allclose(O3, O4, atol=1e-14)
+    np.testing.assert_allclose(L3, L4, atol=1e-14)
+    # all parts empty -> zeros and -inf
+    O5, L5 = oracle.merge(Op, np.full_like(Lp, -np.inf))
+    assert (O5 == 0).all() and (L5 == -np.inf).all()
+    # weights are a convex combination: merged O lies in the hull of the parts per element
+    assert (O <= Op.max(0) + 1e-12).all() and (O >= Op.min(0) - 1e-12).all()
+    # the local-max / local-sum form agrees for any choice of local maxima
+    m = Lp - rng.uniform(0, 3, size=Lp.shape)
+    l = np.exp(Lp - m)
+    U = Op * l[..., None]
+    np.testing.assert_allclose(oracle.merge_ml(U, m, l), O, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# the seeded generator (shared input module)
+# ---------------------------------------------------------------------------
+def test_generator_rounding_matches_torch_bf16():
+    v = np.random.default_rng(0).standard_normal(100000).astype(np.float32) * 3
+    mine = synth.f32_to_bf16_bits(v)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(mine, ref)
+
+
+def test_generator_statistics_and_determinism():
+    a = synth.values_bf16(7, synth.T_K, 3, 0, 200000, 0.5)
+    b = synth.values_bf16(7, synth.T_K, 3, 100000, 100000, 0.5)
+    np.testing.assert_array_equal(a[100000:], b)
+    x = synth.bf16_bits_to_f64(a)
+    assert abs(x.mean()) < 0.01 and abs(x.std() - 0.5) < 0.01
+    assert np.abs(x).max() <= 0.5 * 3.47
+    c = synth.values_bf16(7, synth.T_V, 3, 0, 1000, 0.5)
+    assert not (c == a[:1000]).all()
+
+
+def test_workload_recipes():
+    mix = synth.workload("mla_mix").seq_lens
+    s = np.array(mix)
+    assert len(s) == 256 and s.max() <= 327680
+    assert 60000 < np.median(s) < 75000
+    assert abs((s > 65536).mean() - 0.53) < 0.01
+    assert abs((s > 131072).mean() - 0.08) < 0.01
+    assert 0.03 <= (s > 262144).mean() <= 0.04
+    assert abs((s < 8192).mean() - 0.18) < 0.01
+    g = synth.workload("gqa_70b").seq_lens
+    assert len(g) == 64 and min(g) >= 8192 and max(g) <= 32768
+    m = synth.workload("mla_b32").seq_lens
+    assert len(m) == 32 and 40000 < np.median(m) < 100000
+    lg = synth.workload("mla_long").seq_lens
+    assert len(lg) == 4 and min(lg) >= 204800 and max(lg) <= 262144
+    assert synth.workload("gqa_tiny").seq_lens == [100, 257]

@@ -1,0 +1,242 @@
+/*
+ * dcp.h -- C ABI of the decode-context-parallel (DCP) attention library.
+ *
+ * The operation (sources, cited by page title and section):
+ *   [P1] "Efficient Decode Context Parallelism with vLLM for Long Context
+ *        Workloads" (papercache.org summary of the vLLM blog), "A2 方法细节":
+ *        the KV cache of every request is split along the sequence into D
+ *        shards; each shard attends the full single-token query against its
+ *        local KV slice and emits a partial output O_i with its log-sum-exp
+ *        LSE_i; the partials are combined as
+ *            O = sum_i exp(LSE_i) / sum_j exp(LSE_j) * O_i.
+ *   [P3] "vLLM长序列推理优化：DCP切分KV Cache原理与实战", §2.2: logical block
+ *        b of a request belongs to shard b % D (interleaved sharding);
+ *        §3.2: each shard stores its blocks in its own physical pool and
+ *        addresses them through a global -> local remap (global block 4 of
+ *        shard 0 with D = 4 is local block 1).
+ *
+ * All D shards live on ONE GPU here: D separate paged pools in the same HBM,
+ * and the pages' AllGather / ReduceScatter exchange becomes an on-device
+ * merge kernel (dcp_lse_merge).
+ *
+ * Conventions for every call:
+ *   - The caller owns all memory.  The library never allocates device or
+ *     host memory on the compute path and keeps no global state (it caches
+ *     one driver entry point, looked up once).  Calls are thread-safe.
+ *   - "device" pointers are CUDA device addresses (e.g. a torch tensor's
+ *     data_ptr()); "host" pointers are ordinary CPU memory.
+ *   - GPU calls are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = legacy default stream).  They never synchronise, except
+ *     dcp_read_device_error which is documented as synchronous.
+ *   - Return value: DCP_OK, or an error code.  Argument errors are detected
+ *     on the host before anything is launched (nothing is written then).
+ *     DCP_ERR_CUDA means a CUDA runtime call or a launch failed.
+ *   - Data types: queries and KV are bf16 (raw 16-bit patterns), outputs
+ *     and LSE are fp32, LSE in natural-log units of the SCALED scores,
+ *     tables and lengths are int32.
+ *   - Supported shapes (anything else is DCP_ERR_UNSUPPORTED):
+ *       GQA: head_dim_qk == head_dim_v in {64, 128}; Hq % Hkv == 0 and
+ *            Hq / Hkv <= 16; block_size a multiple of 16, at most 256.
+ *       MLA: Hq == 64, Hkv == 1, head_dim_qk == 576, head_dim_v == 512,
+ *            block_size == 64.
+ *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.
+ */
+#ifndef DCP_H
+#define DCP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DCP_API __attribute__((visibility("default")))
+#else
+#define DCP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dcp_status {
+    DCP_OK = 0,
+    DCP_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent arguments */
+    DCP_ERR_UNSUPPORTED = 2, /* shape outside the supported set listed above */
+    DCP_ERR_CAPACITY = 3,    /* a caller buffer (table row, workspace) is too small */
+    DCP_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    DCP_ERR_DEVICE = 5       /* the device recorded an invalid page id (see dcp_read_device_error) */
+} dcp_status;
+
+typedef enum dcp_layout {
+    DCP_LAYOUT_GQA = 0, /* grouped-query attention: Hkv KV heads, q head h reads KV head h / (Hq/Hkv) */
+    DCP_LAYOUT_MLA = 1  /* multi-head latent attention, absorbed form: one shared latent row per token */
+} dcp_layout;
+
+/*
+ * Problem description shared by the decode calls.
+ *   layout           dcp_layout.
+ *   batch            B, number of requests (one decode token each).
+ *   num_q_heads      Hq.
+ *   num_kv_heads     Hkv (GQA); must be 1 for MLA.
+ *   head_dim_qk      query/key width (GQA head_dim; MLA 576 = 512 latent + 64 rope).
+ *   head_dim_v       value width (GQA head_dim; MLA 512 = the first 512 entries of the latent row).
+ *   block_size       tokens per KV page.
+ *   max_local_blocks row length of each shard's block table (>= the largest local block count).
+ *   softmax_scale    multiplier of q.k (e.g. 1/sqrt(head_dim); MLA 1/sqrt(192)).
+ */
+typedef struct dcp_attn_desc {
+    int32_t layout;
+    int32_t batch;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim_qk;
+    int32_t head_dim_v;
+    int32_t block_size;
+    int32_t max_local_blocks;
+    float softmax_scale;
+} dcp_attn_desc;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+DCP_API int32_t dcp_version(void);
+
+/* Static string naming a status code. */
+DCP_API const char *dcp_status_string(dcp_status status);
+
+/*
+ * Table extent (host only).  [P3 §2.2, §3.2]
+ *   seq_lens          host int32[batch], tokens already in the cache per request (>= 0).
+ *   max_local_blocks  out: largest number of blocks any request has in any shard.
+ *   num_pages         out, host int32[D]: pages shard s needs (sum over requests).
+ * Errors: DCP_ERR_INVALID_ARG for null pointers, batch < 0, block_size <= 0,
+ * D < 1 or D > 16, or a negative length.
+ */
+DCP_API dcp_status dcp_block_table_extent(const int32_t *seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                  int32_t *max_local_blocks, int32_t *num_pages);
+
+/*
+ * Per-shard block tables (host only).  [P3 §2.2 interleaved rule, §3.2 remap]
+ * Token t of request b lies in logical block g = t / block_size, owned by
+ * shard s = g % D as local block j = g / D.  For every shard s:
+ *   tables[s][b][j]  = physical page of shard s's pool holding global block
+ *                      j*D + s of request b; -1 past the request's local blocks;
+ *   local_len[s][b]  = tokens of request b stored by shard s.
+ * Pages of each shard are numbered 0.. in (request, local block) order.  If
+ * perm_seed != 0, the ids of shard s are relabelled by the permutation of
+ * [0, num_pages[s]) that a Fisher-Yates shuffle produces from the SplitMix64
+ * stream whose state starts at perm_seed + (s+1) * 0xD1B54A32D192ED03
+ * (i from n-1 down to 1: state += 0x9E3779B97F4A7C15, j = mix(state) % (i+1),
+ * swap entries i and j) -- non-contiguous page ids for testing allocators.
+ *   tables     out, host int32[D][batch][max_local_blocks].
+ *   local_len  out, host int32[D][batch]; may be NULL.
+ * Errors: as dcp_block_table_extent; DCP_ERR_CAPACITY if max_local_blocks is
+ * smaller than a request's local block count (tables then undefined).
+ */
+DCP_API dcp_status dcp_build_block_table(const int32_t *seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                 uint64_t perm_seed, int32_t max_local_blocks, int32_t *tables,
+                                 int32_t *local_len);
+
+/* Bytes of one KV page for `desc` (GQA: 2*Hkv*block_size*head_dim*2; MLA: block_size*576*2); 0 if invalid. */
+DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
+
+/*
+ * Cache placement: scatter every request's unsharded KV rows into the D
+ * shard pools (the cache write that precedes decoding).  [P3 §3.2]
+ *   kv_src      device bf16, requests concatenated in order:
+ *               GQA rows [token][2 (K,V)][Hkv][head_dim]; MLA rows [token][576].
+ *   cu_seqlens  device int64[batch+1], prefix sums of seq_lens (row offsets in kv_src).
+ *   seq_lens    device int32[batch].
+ *   tables      host array of D device pointers, each int32[batch][max_local_blocks]
+ *               (as built by dcp_build_block_table).
+ *   kv_pools    host array of D device pointers; pool s holds pool_pages[s] pages:
+ *               GQA page [2 (K,V)][Hkv][block_size][head_dim] bf16;
+ *               MLA page [block_size][576] bf16.
+ *   pool_pages  host int32[D].
+ *   device_error optional device int32 (may be NULL): set to 1 if a table entry
+ *               lies outside its pool; such rows are skipped, never written.
+ * Slots past a request's last token keep whatever they held.
+ */
+DCP_API dcp_status dcp_place_kv(const dcp_attn_desc *desc, int32_t D, const void *kv_src, const int64_t *cu_seqlens,
+                        const int32_t *seq_lens, const int32_t *const *tables, void *const *kv_pools,
+                        const int32_t *pool_pages, int32_t *device_error, void *stream);
+
+/*
+ * Workspace bytes the decode calls need for `desc` and D shards on the
+ * current device (split partials, arrival counters, a status word).  The
+ * workspace must be zeroed once by dcp_workspace_init before its first use;
+ * every decode call leaves its counters at zero again.  One workspace may
+ * not be used by two decode calls that overlap in time.  0 if invalid.
+ */
+DCP_API size_t dcp_decode_workspace_bytes(const dcp_attn_desc *desc, int32_t D);
+
+/* Zero a workspace (asynchronous, on `stream`). */
+DCP_API dcp_status dcp_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Partial attention of ONE shard.  [P1 "A2 方法细节", Compute step]
+ * For every request b and query head h, over the tokens of b that shard
+ * `shard` stores (logical blocks g with g % D == shard):
+ *   s_t = softmax_scale * q[b][h] . k_t,  m = max s_t,  l = sum exp(s_t - m),
+ *   O_i[b][h] = sum exp(s_t - m) v_t / l,  LSE_i[b][h] = m + ln l.
+ * GQA: k_t, v_t are KV head h / (Hq/Hkv) of token t.  MLA: k_t is the whole
+ * 576-wide latent row, v_t its first 512 entries.  A request with no token
+ * in this shard gets O_i = 0 and LSE_i = -inf.
+ *   q           device bf16 [batch][Hq][head_dim_qk] (the full query: every shard reads it).
+ *   kv_pool     device, this shard's pool (layout as in dcp_place_kv), pool_pages pages.
+ *   table       device int32 [batch][max_local_blocks], this shard's block table.
+ *   seq_lens    device int32 [batch], GLOBAL lengths; the local token count is
+ *               derived from (seq_len, block_size, shard, D).
+ *   O_i         device fp32 [batch][Hq][head_dim_v];  LSE_i  device fp32 [batch][Hq].
+ *   workspace   device, >= dcp_decode_workspace_bytes(desc, D) bytes, initialised.
+ * Page ids outside [0, pool_pages) are not read (their tokens count as zero
+ * keys and values) and set the workspace status (see dcp_read_device_error).
+ */
+DCP_API dcp_status dcp_decode_partial(const dcp_attn_desc *desc, const void *q, const void *kv_pool, int32_t pool_pages,
+                              const int32_t *table, const int32_t *seq_lens, int32_t shard, int32_t D, float *O_i,
+                              float *LSE_i, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * All D partials in one launch (the same results as D calls of
+ * dcp_decode_partial, bit for bit).  Host arrays of D device pointers:
+ * kv_pools[s], tables[s], O_parts[s], LSE_parts[s]; pool_pages host int32[D].
+ */
+DCP_API dcp_status dcp_decode_partial_all(const dcp_attn_desc *desc, const void *q, const void *const *kv_pools,
+                                  const int32_t *pool_pages, const int32_t *const *tables, const int32_t *seq_lens,
+                                  int32_t D, float *const *O_parts, float *const *LSE_parts, void *workspace,
+                                  size_t workspace_bytes, void *stream);
+
+/*
+ * LSE merge of D partials.  [P1 "A2 方法细节", merge equation;
+ * P3 §2.3 equivalent local-max/local-sum form]
+ *   O[r] = sum_i w_i O_i[r] / sum_i w_i,  w_i = exp(LSE_i[r] - max_j LSE_j[r]),
+ *   LSE_out[r] = max_j LSE_j[r] + ln sum_i w_i.
+ * Parts with LSE = -inf weigh 0; if all are -inf then O = 0, LSE_out = -inf.
+ *   O_parts, LSE_parts  host arrays of D device pointers: fp32 [rows][d_v] and fp32 [rows].
+ *   rows                number of (request, head) rows (batch * Hq).
+ *   O                   device fp32 [rows][d_v]; LSE_out device fp32 [rows] or NULL.
+ * d_v must be a multiple of 4 and all pointers 16-byte aligned.
+ */
+DCP_API dcp_status dcp_lse_merge(const float *const *O_parts, const float *const *LSE_parts, int32_t D, int32_t rows,
+                         int32_t d_v, float *O, float *LSE_out, void *stream);
+
+/*
+ * Read (synchronously: waits for `stream`) and clear the status word of a
+ * workspace.  *error_out is a bit set, 0 if nothing was recorded since the
+ * last read: bit 0 (1) = a block-table entry lay outside its pool; bit 1
+ * (2) = an internal pipeline wait exceeded its time limit (the results of
+ * that call are invalid; never expected in correct operation).
+ */
+DCP_API dcp_status dcp_read_device_error(void *workspace, int32_t *error_out, void *stream);
+
+/*
+ * Parallel-configuration rule of [P1 "A2 方法细节"] (MLA and GQA backend paragraphs):
+ *   MLA: tp >= dcp and tp % dcp == 0;
+ *   GQA: (tp / num_kv_heads) >= dcp and (tp / num_kv_heads) % dcp == 0.
+ * dcp == 1 is always accepted.  DCP_OK if allowed, DCP_ERR_UNSUPPORTED if
+ * not, DCP_ERR_INVALID_ARG for non-positive arguments.
+ */
+DCP_API dcp_status dcp_validate_config(int32_t tp, int32_t dcp, int32_t num_kv_heads, int32_t layout);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCP_H */

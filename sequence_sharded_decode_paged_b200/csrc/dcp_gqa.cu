@@ -1,0 +1,497 @@
+// dcp_gqa.cu -- GQA partial decode attention over D interleaved paged shards.
+//
+// What it computes ("Efficient Decode Context Parallelism with vLLM for Long
+// Context Workloads", A2 方法细节, Compute step; "vLLM长序列推理优化：DCP切分KV
+// Cache原理与实战" §2.2/§3.2 for the shard layout): for every shard s, request
+// b and query head h, softmax attention of q[b][h] over the tokens of b that
+// shard s stores, giving the normalised partial O_s[b][h] and LSE_s[b][h].
+//
+// Design (memory bound: 8 flop per KV byte at 8 query heads per KV head):
+//  * Persistent CTAs.  The local page lists of all (shard, request) segments
+//    are concatenated and cut into equal contiguous ranges, one per CTA, so
+//    long and short requests balance exactly (flash-decoding split with no
+//    fixed split size).  A segment cut by a range boundary is finished by the
+//    last CTA to arrive on its counter (no spinning, no extra launch).
+//  * One producer thread streams whole pages of the CTA's KV-head group into
+//    a ring of shared-memory stages with 2-D TMA tiles (128-byte swizzle, no
+//    multicast); K and V of all heads of one page arrive on one mbarrier.
+//  * Eight consumer warps; each owns one KV head and all G <= 16 query heads
+//    sharing it (16-row mma tile).  Per 16-token chunk: S = Q K^T with
+//    mma.m16n8k16 (K fragments by ldmatrix), online softmax in fp32 with quad
+//    shuffles, P rounded to bf16 in registers and O += P V (V by
+//    ldmatrix.trans).  Tokens past the sequence end are masked in both S and
+//    the V fragments, so stale cache contents (even NaN) never leak in.
+#include <float.h>
+
+#include "dcp_device.cuh"
+#include "dcp_internal.h"
+
+namespace dcp {
+
+constexpr int kGqaConsumerWarps = 8;
+constexpr int kGqaThreads = (kGqaConsumerWarps + 1) * 32;
+constexpr int kScratchInts = 64;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+struct GqaParams {
+  CUtensorMap tmap[kMaxShards];
+  const int32_t* table[kMaxShards];
+  float* O[kMaxShards];
+  float* LSE[kMaxShards];
+  int pool_pages[kMaxShards];
+  int shard_of_si[kMaxShards];
+  const __nv_bfloat16* q;
+  const int32_t* seq_lens;
+  int* status;
+  int* counters;
+  float* slots;
+  float scale_log2;
+  int n_si, B, Hq, Hkv, G, bs, D, mlb;
+  int hpc, n_hg, stages, wph;
+  uint32_t stage_bytes;
+  int slot_floats;
+};
+
+template <int HEAD_DIM>
+struct GqaGeom {
+  static constexpr int kBoxes = HEAD_DIM / 64;  // 64-element (128-byte) swizzled boxes per row
+  static constexpr int kNTiles = HEAD_DIM / 8;  // n-tiles of O
+  static constexpr int kKTiles = HEAD_DIM / 16; // k-tiles of Q K^T
+  static constexpr int kCombineFloats = kNTiles * 4 + 4;  // per lane per warp
+};
+
+template <int HEAD_DIM>
+__global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid_constant__ GqaParams p) {
+  using Geo = GqaGeom<HEAD_DIM>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* stage_mem = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * p.stage_bytes);
+  uint64_t* empty = full + p.stages;
+  int* stage_ok = reinterpret_cast<int*>(empty + p.stages);
+  int* scratch = stage_ok + 8;
+  int* bcast = scratch + kScratchInts;
+  float* combine = reinterpret_cast<float*>(bcast + 8);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hg = blockIdx.y, cta = blockIdx.x, nctas = gridDim.x;
+  const int B = p.B, bs = p.bs, D = p.D;
+  const uint32_t box_bytes = (uint32_t)p.hpc * bs * 128u;
+
+  if ((smem_u32(smem) & 1023u) != 0u) {  // swizzled TMA tiles need 1024-byte aligned stages
+    if (tid == 0) atomicOr(p.status, kDevTimeout);
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kGqaConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == kGqaConsumerWarps && lane == 0)
+    for (int si = 0; si < p.n_si; ++si)
+      if (p.pool_pages[si] > 0) prefetch_tmap(&p.tmap[si]);
+  __syncthreads();
+
+  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, bs, D, cta, nctas, scratch);
+  const int T = plan.T, P = plan.P;
+  const int lo = cta * P, hi = min(lo + P, T);
+  const int S = p.n_si * B;
+
+  // ------------------------------------------------------------------ producer
+  if (warp == kGqaConsumerWarps) {
+    if (lane != 0) return;
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool aborted = false;
+    int pre = plan.pre0;
+    for (int sid = plan.sid0; sid < S && !aborted; ++sid) {
+      const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+      const int n = local_pages(p.seq_lens[b], bs, D, shard);
+      if (seg_first_cta(pre, n, T, P) > cta) break;
+      const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+      const int32_t* trow = p.table[si] + (size_t)b * p.mlb;
+      for (int j = a; j < e; ++j) {
+        const int page = trow[j];
+        const bool ok = page >= 0 && page < p.pool_pages[si];
+        if (!ok) atomicOr(p.status, kDevBadPage);
+        if (!mbar_wait(&empty[stage], phase ^ 1u)) {
+          atomicOr(p.status, kDevTimeout);
+          aborted = true;
+          break;
+        }
+        stage_ok[stage] = ok ? 1 : 0;
+        if (ok) {
+          mbar_arrive_expect_tx(&full[stage], p.stage_bytes);
+          uint8_t* dst = stage_mem + (size_t)stage * p.stage_bytes;
+          const int row_k = ((page * 2 + 0) * p.Hkv + hg * p.hpc) * bs;
+          const int row_v = ((page * 2 + 1) * p.Hkv + hg * p.hpc) * bs;
+#pragma unroll
+          for (int bx = 0; bx < Geo::kBoxes; ++bx) {
+            tma_load_2d(dst + bx * box_bytes, &p.tmap[si], bx * 64, row_k, &full[stage]);
+            tma_load_2d(dst + (Geo::kBoxes + bx) * box_bytes, &p.tmap[si], bx * 64, row_v, &full[stage]);
+          }
+        } else {
+          mbar_arrive(&full[stage]);
+        }
+        ++issued;
+        if (++stage == p.stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      pre += n;
+    }
+    // Never leave the CTA while a copy into its shared memory is in flight.
+    const long first = issued > p.stages ? issued - p.stages : 0;
+    for (long i = first; i < issued; ++i) {
+      const int s = (int)(i % p.stages);
+      const uint32_t par = (uint32_t)((i / p.stages) & 1);
+      if (!mbar_wait(&full[s], par)) atomicOr(p.status, kDevTimeout);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int hpc = p.hpc, G = p.G, wph = p.wph;
+  const bool active = warp < hpc * wph;
+  const int hh = warp % hpc, sub = warp / hpc;
+  const int g4 = lane >> 2, c4 = lane & 3;
+  const int rows_hg = hpc * G;
+  const int qrow0 = hg * rows_hg;  // first query head of this head group
+  int stage = 0;
+  uint32_t phase = 0;
+  int pre = plan.pre0;
+  bool dead = false;
+
+  for (int sid = plan.sid0; sid < S; ++sid) {
+    const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+    const int seq_len = p.seq_lens[b];
+    const int n = local_pages(seq_len, bs, D, shard);
+    const int c0 = seg_first_cta(pre, n, T, P);
+    if (c0 > cta) break;
+    const int c1 = seg_last_cta(pre, n, T, P);
+    float* Oout = p.O[si] + ((size_t)b * p.Hq + qrow0) * HEAD_DIM;
+    float* Lout = p.LSE[si] + (size_t)b * p.Hq + qrow0;
+    if (n == 0) {  // no token of this request in this shard
+      for (int i = tid; i < rows_hg * HEAD_DIM; i += kGqaConsumerWarps * 32) Oout[i] = 0.f;
+      for (int i = tid; i < rows_hg; i += kGqaConsumerWarps * 32) Lout[i] = -INFINITY;
+      pre += n;
+      continue;
+    }
+    const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+
+    // query fragments (16-row A tile; rows >= G are zero)
+    uint32_t qa[Geo::kKTiles][4];
+    const int kvh = hg * hpc + hh;
+    {
+      const uint32_t* qb = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * HEAD_DIM);
+#pragma unroll
+      for (int kt = 0; kt < Geo::kKTiles; ++kt) {
+        const int col = kt * 16 + c4 * 2;
+        qa[kt][0] = (active && g4 < G) ? __ldg(qb + (g4 * HEAD_DIM + col) / 2) : 0u;
+        qa[kt][1] = (active && g4 + 8 < G) ? __ldg(qb + ((g4 + 8) * HEAD_DIM + col) / 2) : 0u;
+        qa[kt][2] = (active && g4 < G) ? __ldg(qb + (g4 * HEAD_DIM + col + 8) / 2) : 0u;
+        qa[kt][3] = (active && g4 + 8 < G) ? __ldg(qb + ((g4 + 8) * HEAD_DIM + col + 8) / 2) : 0u;
+      }
+    }
+    float o[Geo::kNTiles][4];
+#pragma unroll
+    for (int i = 0; i < Geo::kNTiles; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+    for (int j = a; j < e; ++j) {
+      // a wait that times out marks this warp dead: it stops waiting and computing
+      // but keeps the block-wide barrier sequence, so nothing else can hang on it
+      if (!dead && !mbar_wait(&full[stage], phase)) {
+        atomicOr(p.status, kDevTimeout);
+        dead = true;
+      }
+      if (!dead && active && ((j - a) % wph) == sub && stage_ok[stage]) {
+        const int gblk = j * D + shard;
+        const int valid = min(bs, seq_len - gblk * bs);
+        const uint32_t kbase = smem_u32(stage_mem + (size_t)stage * p.stage_bytes);
+        const uint32_t vbase = kbase + Geo::kBoxes * box_bytes;
+        for (int t0 = 0; t0 < valid; t0 += 16) {
+          // ---- S = Q K^T for 16 tokens (two 8-token n-tiles)
+          float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          const uint32_t krow = (uint32_t)(hh * bs + t0 + (lane & 7) + ((lane >> 4) << 3));
+#pragma unroll
+          for (int kt = 0; kt < Geo::kKTiles; ++kt) {
+            const uint32_t chunk = (uint32_t)((kt & 3) * 2 + ((lane >> 3) & 1));
+            uint32_t b00, b01, b10, b11;
+            ldsm_x4(kbase + (kt >> 2) * box_bytes + sw128(krow, chunk), b00, b01, b10, b11);
+            mma_bf16_16816(s[0], qa[kt], b00, b01);
+            mma_bf16_16816(s[1], qa[kt], b10, b11);
+          }
+          // ---- online softmax (log2 domain), rows g4 and g4 + 8
+          const int vrem = valid - t0;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int tok = nt * 8 + c4 * 2 + (i & 1);
+              s[nt][i] = tok < vrem ? s[nt][i] * p.scale_log2 : -INFINITY;
+            }
+          float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+          float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+          m0 = mn0;
+          m1 = mn1;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            s[nt][0] = exp2f(s[nt][0] - mn0);
+            s[nt][1] = exp2f(s[nt][1] - mn0);
+            s[nt][2] = exp2f(s[nt][2] - mn1);
+            s[nt][3] = exp2f(s[nt][3] - mn1);
+          }
+          l0 = l0 * al0 + (s[0][0] + s[0][1] + s[1][0] + s[1][1]);
+          l1 = l1 * al1 + (s[0][2] + s[0][3] + s[1][2] + s[1][3]);
+#pragma unroll
+          for (int i = 0; i < Geo::kNTiles; ++i) {
+            o[i][0] *= al0;
+            o[i][1] *= al0;
+            o[i][2] *= al1;
+            o[i][3] *= al1;
+          }
+          uint32_t pa[4];
+          pa[0] = pack_bf16x2(s[0][0], s[0][1]);
+          pa[1] = pack_bf16x2(s[0][2], s[0][3]);
+          pa[2] = pack_bf16x2(s[1][0], s[1][1]);
+          pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+          // ---- O += P V; V fragments of tokens past the end are zeroed
+          const uint32_t vrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
+          const bool tail = vrem < 16;
+          const uint32_t keep0 = (c4 * 2 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 1 < vrem ? 0xFFFF0000u : 0u);
+          const uint32_t keep1 = (c4 * 2 + 8 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 9 < vrem ? 0xFFFF0000u : 0u);
+#pragma unroll
+          for (int np = 0; np < Geo::kNTiles / 2; ++np) {
+            const uint32_t chunk = (uint32_t)((np & 3) * 2 + (lane >> 4));
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(vbase + (np >> 2) * box_bytes + sw128(vrow, chunk), v0, v1, v2, v3);
+            if (tail) {
+              v0 &= keep0;
+              v1 &= keep1;
+              v2 &= keep0;
+              v3 &= keep1;
+            }
+            mma_bf16_16816(o[2 * np], pa, v0, v1);
+            mma_bf16_16816(o[2 * np + 1], pa, v2, v3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == p.stages) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+
+    // ---- finish the (warp-local) softmax state
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (wph > 1) {  // several warps shared this head: combine their states
+      float* mine = combine + (size_t)warp * Geo::kCombineFloats * 32;
+#pragma unroll
+      for (int i = 0; i < Geo::kNTiles; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mine[(i * 4 + k) * 32 + lane] = o[i][k];
+      mine[(Geo::kNTiles * 4 + 0) * 32 + lane] = m0;
+      mine[(Geo::kNTiles * 4 + 1) * 32 + lane] = m1;
+      mine[(Geo::kNTiles * 4 + 2) * 32 + lane] = l0;
+      mine[(Geo::kNTiles * 4 + 3) * 32 + lane] = l1;
+      named_bar_sync(1, kGqaConsumerWarps * 32);
+      if (active && sub == 0) {
+        for (int w2 = 1; w2 < wph; ++w2) {
+          const float* other = combine + (size_t)(w2 * hpc + hh) * Geo::kCombineFloats * 32;
+          const float om0 = other[(Geo::kNTiles * 4 + 0) * 32 + lane];
+          const float om1 = other[(Geo::kNTiles * 4 + 1) * 32 + lane];
+          const float ol0 = other[(Geo::kNTiles * 4 + 2) * 32 + lane];
+          const float ol1 = other[(Geo::kNTiles * 4 + 3) * 32 + lane];
+          const float nm0 = fmaxf(m0, om0), nm1 = fmaxf(m1, om1);
+          const float sa0 = nm0 == -INFINITY ? 0.f : exp2f(m0 - nm0);
+          const float sb0 = nm0 == -INFINITY ? 0.f : exp2f(om0 - nm0);
+          const float sa1 = nm1 == -INFINITY ? 0.f : exp2f(m1 - nm1);
+          const float sb1 = nm1 == -INFINITY ? 0.f : exp2f(om1 - nm1);
+#pragma unroll
+          for (int i = 0; i < Geo::kNTiles; ++i) {
+            o[i][0] = o[i][0] * sa0 + other[(i * 4 + 0) * 32 + lane] * sb0;
+            o[i][1] = o[i][1] * sa0 + other[(i * 4 + 1) * 32 + lane] * sb0;
+            o[i][2] = o[i][2] * sa1 + other[(i * 4 + 2) * 32 + lane] * sb1;
+            o[i][3] = o[i][3] * sa1 + other[(i * 4 + 3) * 32 + lane] * sb1;
+          }
+          l0 = l0 * sa0 + ol0 * sb0;
+          l1 = l1 * sa1 + ol1 * sb1;
+          m0 = nm0;
+          m1 = nm1;
+        }
+      }
+      named_bar_sync(1, kGqaConsumerWarps * 32);
+    }
+
+    const bool complete = (c0 == c1);
+    int slot = 0;
+    if (!complete) slot = 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
+    if (active && sub == 0) {
+      // base-2 log-sum-exp of each row; empty state (all pages skipped) -> -inf
+      const float lse0 = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
+      const float lse1 = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
+      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      float* dstO;
+      float* dstL;
+      size_t stride;
+      if (complete) {
+        dstO = Oout + (size_t)hh * G * HEAD_DIM;
+        dstL = Lout + hh * G;
+        stride = HEAD_DIM;
+      } else {
+        float* sl = p.slots + ((size_t)slot * p.n_hg + hg) * p.slot_floats;
+        dstO = sl + (size_t)hh * G * HEAD_DIM;
+        dstL = sl + (size_t)rows_hg * HEAD_DIM + hh * G;
+        stride = HEAD_DIM;
+      }
+      if (g4 < G) {
+#pragma unroll
+        for (int i = 0; i < Geo::kNTiles; ++i)
+          *reinterpret_cast<float2*>(dstO + g4 * stride + i * 8 + c4 * 2) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
+        if (c4 == 0) dstL[g4] = complete ? lse0 * kLn2 : lse0;
+      }
+      if (g4 + 8 < G) {
+#pragma unroll
+        for (int i = 0; i < Geo::kNTiles; ++i)
+          *reinterpret_cast<float2*>(dstO + (g4 + 8) * stride + i * 8 + c4 * 2) =
+              make_float2(o[i][2] * inv1, o[i][3] * inv1);
+        if (c4 == 0) dstL[g4 + 8] = complete ? lse1 * kLn2 : lse1;
+      }
+    }
+    if (!complete) {
+      // publish this CTA's piece; the last CTA to arrive merges all pieces
+      __threadfence();
+      named_bar_sync(1, kGqaConsumerWarps * 32);
+      int* ctr = p.counters + (size_t)sid * p.n_hg + hg;
+      if (tid == 0) bcast[0] = (atomicAdd(ctr, 1) == c1 - c0) ? 1 : 0;
+      named_bar_sync(1, kGqaConsumerWarps * 32);
+      if (bcast[0]) {
+        __threadfence();
+        constexpr int kPer = HEAD_DIM / 32;
+        for (int r = warp; r < rows_hg; r += kGqaConsumerWarps) {
+          float mx = -INFINITY;
+          for (int c = c0; c <= c1; ++c) {
+            const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+            const float* sl = p.slots + ((size_t)k * p.n_hg + hg) * p.slot_floats;
+            mx = fmaxf(mx, __ldcg(sl + (size_t)rows_hg * HEAD_DIM + r));
+          }
+          float acc[kPer];
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+          float wsum = 0.f;
+          if (mx != -INFINITY) {
+            for (int c = c0; c <= c1; ++c) {
+              const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+              const float* sl = p.slots + ((size_t)k * p.n_hg + hg) * p.slot_floats;
+              const float lk = __ldcg(sl + (size_t)rows_hg * HEAD_DIM + r);
+              const float w = lk == -INFINITY ? 0.f : exp2f(lk - mx);
+              wsum += w;
+#pragma unroll
+              for (int i = 0; i < kPer; ++i) acc[i] += w * __ldcg(sl + (size_t)r * HEAD_DIM + lane * kPer + i);
+            }
+          }
+          const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) Oout[(size_t)r * HEAD_DIM + lane * kPer + i] = acc[i] * inv;
+          if (lane == 0) Lout[r] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+        }
+        if (tid == 0) *ctr = 0;  // leave the counter ready for the next call
+      }
+    }
+    pre += n;
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
+int gqa_heads_per_cta(int Hkv, int bs) {
+  const int cap = min(kGqaConsumerWarps, 256 / bs);
+  int best = 1;
+  for (int h = 1; h <= cap; ++h)
+    if (Hkv % h == 0) best = h;
+  return best;
+}
+
+static int gqa_stage_count(uint32_t stage_bytes, size_t fixed_bytes) {
+  const size_t budget = 225 * 1024 - fixed_bytes;
+  int st = (int)(budget / stage_bytes);
+  return st > 8 ? 8 : st;
+}
+
+template <int HEAD_DIM>
+static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
+                                  const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
+  WorkspaceLayout L;
+  if (!workspace_layout(d, D, &L)) return DCP_ERR_UNSUPPORTED;
+  if (ws_bytes < L.total) return DCP_ERR_CAPACITY;
+  GqaParams p;
+  memset(&p, 0, sizeof(p));
+  p.n_si = set.n;
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.G = d.num_q_heads / d.num_kv_heads;
+  p.bs = d.block_size;
+  p.D = D;
+  p.mlb = d.max_local_blocks;
+  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs);
+  p.n_hg = p.Hkv / p.hpc;
+  p.wph = kGqaConsumerWarps / p.hpc;
+  p.stage_bytes = (uint32_t)(2 * p.hpc * p.bs * HEAD_DIM * 2);
+  const size_t combine_bytes =
+      p.wph > 1 ? (size_t)kGqaConsumerWarps * GqaGeom<HEAD_DIM>::kCombineFloats * 32 * sizeof(float) : 0;
+  const size_t fixed = 16 * 8 + 8 * 4 + kScratchInts * 4 + 8 * 4 + combine_bytes;
+  p.stages = gqa_stage_count(p.stage_bytes, fixed);
+  if (p.stages < 2) return DCP_ERR_UNSUPPORTED;
+  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.seq_lens = seq_lens;
+  p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
+  p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);
+  p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slots_off);
+  p.slot_floats = L.slot_floats;
+  for (int si = 0; si < set.n; ++si) {
+    p.table[si] = set.table[si];
+    p.O[si] = set.O[si];
+    p.LSE[si] = set.LSE[si];
+    p.pool_pages[si] = set.pool_pages[si];
+    p.shard_of_si[si] = set.shard[si];
+    if (set.pool_pages[si] > 0) {
+      const uint64_t rows = (uint64_t)set.pool_pages[si] * 2 * p.Hkv * p.bs;
+      if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+      if (encode_tiled_2d(&p.tmap[si], set.pool[si], HEAD_DIM, rows, HEAD_DIM * 2, 64, (uint32_t)(p.hpc * p.bs)) !=
+          CUDA_SUCCESS)
+        return DCP_ERR_CUDA;
+    }
+  }
+  const size_t smem = (size_t)p.stages * p.stage_bytes + fixed;
+  auto kern = gqa_decode_kernel<HEAD_DIM>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return DCP_ERR_CUDA;
+  dim3 grid(L.nctas, p.n_hg);
+  kern<<<grid, kGqaThreads, smem, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
+}
+
+dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
+                             const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (d.head_dim_qk == 128) return launch_gqa_impl<128>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+  if (d.head_dim_qk == 64) return launch_gqa_impl<64>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+  return DCP_ERR_UNSUPPORTED;
+}
+
+}  // namespace dcp

@@ -1,0 +1,106 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The shard tables built by the library are compared bit for bit with the
+oracle's independent construction; the library must export every symbol that
+include/dcp.h declares; argument errors must come back as status codes.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from helpers import ROOT, golden
+from sequence_sharded_decode_paged_b200 import dcp
+
+HEADER = os.path.join(ROOT, "include", "dcp.h")
+
+
+def declared_symbols():
+    text = open(HEADER, encoding="utf-8").read()
+    return sorted(set(re.findall(r"DCP_API\s+[\w\s\*]*?\b(dcp_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_symbols() == sorted(dcp.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(dcp.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert dcp.dcp_version() >= 100
+
+
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8, 16])
+@pytest.mark.parametrize("bs", [16, 64])
+@pytest.mark.parametrize("perm", [0, 99])
+def test_tables_bit_exact_vs_oracle(D, bs, perm):
+    rng = np.random.default_rng(D * 1000 + bs + perm)
+    seq_lens = list(rng.integers(0, 3000, size=9)) + [0, 1, bs, bs + 1, D * bs, D * bs + 1]
+    t_lib, l_lib = dcp.dcp_build_block_table(seq_lens, bs, D, perm)
+    mlb, pages = dcp.dcp_block_table_extent(seq_lens, bs, D)
+    t_or, l_or, p_or = oracle.block_tables(seq_lens, bs, D, perm_seed=perm, max_local_blocks=t_lib.shape[2])
+    np.testing.assert_array_equal(t_lib, t_or)
+    np.testing.assert_array_equal(l_lib, l_or)
+    np.testing.assert_array_equal(pages, p_or)
+    assert mlb == int((t_or >= 0).sum(axis=2).max())
+
+
+@pytest.mark.parametrize("name", ["gqa_tiny", "gqa_70b", "mla_b32", "mla_long", "mla_mix"])
+def test_tables_bit_exact_on_workloads(name):
+    import synth
+    w = synth.workload(name)
+    for D in w.shards:
+        t_lib, l_lib = dcp.dcp_build_block_table(w.seq_lens, w.block_size, D)
+        t_or, l_or, _ = oracle.block_tables(w.seq_lens, w.block_size, D, max_local_blocks=t_lib.shape[2])
+        np.testing.assert_array_equal(t_lib, t_or)
+        np.testing.assert_array_equal(l_lib, l_or)
+
+
+def test_table_capacity_and_argument_errors():
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_build_block_table([100], 16, 2, 0, max_local_blocks=3)
+    assert e.value.status == dcp.DCP_ERR_CAPACITY
+    for args in [([5], 0, 2), ([5], 16, 0), ([5], 16, 17), ([-1], 16, 2)]:
+        with pytest.raises(dcp.DcpError) as e:
+            dcp.dcp_build_block_table(*args)
+        assert e.value.status == dcp.DCP_ERR_INVALID_ARG
+
+
+def test_validate_config_matches_page_examples():
+    for row in golden("validate_config.txt"):
+        layout, tp, dcp_, kvh, want = map(int, row)
+        got = dcp.dcp_validate_config(tp, dcp_, kvh, layout)
+        assert got == (dcp.DCP_OK if want else dcp.DCP_ERR_UNSUPPORTED), row
+    assert dcp.dcp_validate_config(0, 1, 1, 0) == dcp.DCP_ERR_INVALID_ARG
+
+
+def test_page_bytes_and_supported_shapes():
+    d = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 64, 64, 8, 128, 128, 16, 10, 0.1)
+    assert dcp.dcp_kv_page_bytes(d) == 16 * oracle.kv_bytes_per_token(8, 128, 2)
+    m = dcp.make_desc(dcp.DCP_LAYOUT_MLA, 4, 64, 1, 576, 512, 64, 10, 0.07)
+    assert dcp.dcp_kv_page_bytes(m) == 64 * 576 * 2
+    for bad in [dcp.make_desc(0, 1, 8, 2, 96, 96, 16, 1, 0.1),    # head_dim 96
+                dcp.make_desc(0, 1, 8, 3, 64, 64, 16, 1, 0.1),    # Hq % Hkv != 0
+                dcp.make_desc(0, 1, 64, 2, 64, 64, 16, 1, 0.1),   # G = 32 > 16
+                dcp.make_desc(0, 1, 8, 2, 64, 64, 24, 1, 0.1),    # block 24
+                dcp.make_desc(1, 1, 32, 1, 576, 512, 64, 1, 0.1)]:  # MLA with 32 heads
+        assert dcp.dcp_kv_page_bytes(bad) == 0
+        assert dcp.dcp_decode_workspace_bytes(bad, 2) == 0
+    assert dcp.dcp_decode_workspace_bytes(d, 0) == 0
+    assert dcp.dcp_decode_workspace_bytes(d, 4) > 0
+
+
+def test_device_calls_reject_bad_arguments_before_launch():
+    d = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 2, 8, 2, 64, 64, 16, 9, 0.125)
+    lib = ctypes.CDLL(dcp.LIB_PATH)
+    lib.dcp_decode_partial.restype = ctypes.c_int
+    null = ctypes.c_void_p(0)
+    st = lib.dcp_decode_partial(ctypes.byref(d), null, null, 0, null, null, 0, 2, null, null, null,
+                                ctypes.c_size_t(0), null)
+    assert st == dcp.DCP_ERR_INVALID_ARG
+    lib.dcp_lse_merge.restype = ctypes.c_int
+    assert lib.dcp_lse_merge(null, null, 2, 4, 64, null, null, null) == dcp.DCP_ERR_INVALID_ARG

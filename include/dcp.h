@@ -36,7 +36,9 @@
  *     tables and lengths are int32.
  *   - Supported shapes (anything else is DCP_ERR_UNSUPPORTED):
  *       GQA: head_dim_qk == head_dim_v in {64, 128}; Hq % Hkv == 0 and
- *            Hq / Hkv <= 16; block_size a multiple of 16, at most 256.
+ *            Hq / Hkv <= 16; block_size a multiple of 16 with
+ *            block_size * head_dim <= 16384 (up to 256 tokens at head_dim
+ *            64, 128 tokens at head_dim 128).
  *       MLA: Hq == 64, Hkv == 1, head_dim_qk == 576, head_dim_v == 512,
  *            block_size == 64.
  *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.

@@ -75,7 +75,7 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
   if (d.layout == DCP_LAYOUT_GQA) {
     if (d.head_dim_qk != d.head_dim_v || (d.head_dim_qk != 64 && d.head_dim_qk != 128)) return false;
     if (d.num_q_heads % d.num_kv_heads != 0 || d.num_q_heads / d.num_kv_heads > 16) return false;
-    if (d.block_size % 16 != 0 || d.block_size > 256) return false;
+    if (d.block_size % 16 != 0 || d.block_size > 256 || d.block_size * d.head_dim_qk > 16384) return false;
     return true;
   }
   if (d.layout == DCP_LAYOUT_MLA) {
@@ -93,7 +93,7 @@ bool workspace_layout(const dcp_attn_desc& d, int D, WorkspaceLayout* L) {
   if (!desc_supported(d, D, &why)) return false;
   const int sms = device_sm_count();
   if (d.layout == DCP_LAYOUT_GQA) {
-    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size);
+    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size, d.head_dim_qk);
     L->n_hg = d.num_kv_heads / hpc;
     L->rows_per_hg = hpc * (d.num_q_heads / d.num_kv_heads);
     L->nctas = sms / L->n_hg > 0 ? sms / L->n_hg : 1;

@@ -418,8 +418,12 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
 }
 
 // ---------------------------------------------------------------------------- host side
-int gqa_heads_per_cta(int Hkv, int bs) {
-  const int cap = min(kGqaConsumerWarps, 256 / bs);
+// KV heads one CTA streams per page: a divisor of Hkv, at most 8 (one consumer
+// warp each), a TMA box of at most 256 rows, and a stage (K and V of those
+// heads for one page) of at most 64 KB so that three or more stages fit.
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim) {
+  int cap = min(kGqaConsumerWarps, 256 / bs);
+  cap = min(cap, 65536 / (bs * head_dim * 4));
   int best = 1;
   for (int h = 1; h <= cap; ++h)
     if (Hkv % h == 0) best = h;
@@ -448,7 +452,7 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.bs = d.block_size;
   p.D = D;
   p.mlb = d.max_local_blocks;
-  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs);
+  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs, HEAD_DIM);
   p.n_hg = p.Hkv / p.hpc;
   p.wph = kGqaConsumerWarps / p.hpc;
   p.stage_bytes = (uint32_t)(2 * p.hpc * p.bs * HEAD_DIM * 2);

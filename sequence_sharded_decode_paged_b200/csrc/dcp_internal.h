@@ -56,6 +56,6 @@ dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, co
                            const int32_t* pool_pages, int32_t* device_error, cudaStream_t st);
 
 // GQA geometry helpers (shared by the workspace sizing and the launcher).
-int gqa_heads_per_cta(int Hkv, int bs);
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim);
 
 }  // namespace dcp

@@ -120,6 +120,18 @@ def values_bf16(seed: int, tensor: int, request: int, e0: int, n: int, amp: floa
     return f32_to_bf16_bits(v)
 
 
+def values_bf16_at(seed: int, tensor: int, request: int, e: np.ndarray, amp: float) -> np.ndarray:
+    """bf16 bit patterns of the stream elements with indices ``e`` (any shape)."""
+    with np.errstate(over="ignore"):
+        key = np.uint64(stream_key(seed, tensor, request))
+        ee = np.asarray(e, dtype=np.uint64)
+        x = _mix64_np(key + np.uint64(GAMMA) * (ee + np.uint64(1)))
+        s = ((x & np.uint64(0xFFFF)) + ((x >> np.uint64(16)) & np.uint64(0xFFFF))
+             + ((x >> np.uint64(32)) & np.uint64(0xFFFF)) + (x >> np.uint64(48)))
+    z = (s.astype(np.int64) - CENTRE).astype(np.float64) * INV_SD
+    return f32_to_bf16_bits((z * amp).astype(np.float32))
+
+
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
@@ -160,12 +172,23 @@ class Workload:
         n = self.num_q_heads * self.head_dim_qk
         return values_bf16(self.seed, T_Q, b, 0, n, self.q_amp).reshape(self.num_q_heads, self.head_dim_qk)
 
-    def kv_source(self, b: int) -> np.ndarray:
-        """Unsharded KV rows of request ``b`` (bf16 bits).
+    def kv_source_head(self, b: int, h: int, n_tok: Optional[int] = None) -> np.ndarray:
+        """GQA: request ``b``'s rows of KV head ``h`` only, as a one-head source ``[n][2][1][d]``
+        (the first ``n_tok`` tokens if given)."""
+        n_tok = self.seq_lens[b] if n_tok is None else min(n_tok, self.seq_lens[b])
+        d, H = self.head_dim_qk, self.num_kv_heads
+        e = (np.arange(n_tok, dtype=np.uint64)[:, None] * np.uint64(H) + np.uint64(h)) * np.uint64(d) \
+            + np.arange(d, dtype=np.uint64)[None, :]
+        k = values_bf16_at(self.seed, T_K, b, e, self.kv_amp)
+        v = values_bf16_at(self.seed, T_V, b, e, self.kv_amp)
+        return np.stack([k, v], axis=1).reshape(n_tok, 2, 1, d)
+
+    def kv_source(self, b: int, n_tok: Optional[int] = None) -> np.ndarray:
+        """Unsharded KV rows of request ``b`` (bf16 bits), the first ``n_tok`` tokens if given.
 
         GQA: ``[seq_len][2][Hkv][d]``; MLA: ``[seq_len][d_qk]``.
         """
-        n_tok = self.seq_lens[b]
+        n_tok = self.seq_lens[b] if n_tok is None else min(n_tok, self.seq_lens[b])
         if self.layout == GQA:
             per = self.num_kv_heads * self.head_dim_qk
             k = values_bf16(self.seed, T_K, b, 0, n_tok * per, self.kv_amp).reshape(n_tok, 1, per)

@@ -87,6 +87,7 @@ def test_page_bytes_and_supported_shapes():
                 dcp.make_desc(0, 1, 8, 3, 64, 64, 16, 1, 0.1),    # Hq % Hkv != 0
                 dcp.make_desc(0, 1, 64, 2, 64, 64, 16, 1, 0.1),   # G = 32 > 16
                 dcp.make_desc(0, 1, 8, 2, 64, 64, 24, 1, 0.1),    # block 24
+                dcp.make_desc(0, 1, 8, 2, 128, 128, 256, 1, 0.1),  # block 256 at head_dim 128
                 dcp.make_desc(1, 1, 32, 1, 576, 512, 64, 1, 0.1)]:  # MLA with 32 heads
         assert dcp.dcp_kv_page_bytes(bad) == 0
         assert dcp.dcp_decode_workspace_bytes(bad, 2) == 0

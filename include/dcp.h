@@ -206,6 +206,37 @@ DCP_API dcp_status dcp_decode_partial_all(const dcp_attn_desc *desc, const void 
                                   size_t workspace_bytes, void *stream);
 
 /*
+ * dcp_decode_partial_all for callers that cannot allocate device memory
+ * (GQA layout only).  The pages have no counterpart of this call.
+ *
+ * Some callers cannot call cudaMalloc where they run a decode step: code
+ * that is handed only its input and output buffers (an inference-engine
+ * plugin, an embedded runtime without a device allocator), serving loops
+ * that forbid allocation after start-up so that memory never fragments and
+ * no step waits on the allocator, and code that must not touch the
+ * allocator while other work is being captured.  This call takes no
+ * workspace: it uses a 16 MiB scratch array that lives in the library and
+ * that every GPU which loads the library holds until the process exits.
+ * Inputs, outputs and results are those of dcp_decode_partial_all.
+ *   - The first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - Each call clears the scratch's status word and arrival counters on
+ *     `stream`, then launches the decode kernel.  It allocates nothing.
+ *   - All calls share the scratch, which keeps the last call's contents:
+ *     calls that overlap on the GPU (e.g. on two streams) race; serialise them.
+ *   - Out-of-range page ids are skipped as in dcp_decode_partial_all but not
+ *     reported (there is no caller-visible status word).
+ * Errors: as dcp_decode_partial_all; DCP_ERR_UNSUPPORTED for MLA;
+ * DCP_ERR_CAPACITY if the problem needs more than the 16 MiB scratch
+ * (dcp_decode_workspace_bytes(desc, D) > 16 MiB, e.g. very wide head groups).
+ */
+DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc *desc, const void *q,
+                                                  const void *const *kv_pools, const int32_t *pool_pages,
+                                                  const int32_t *const *tables, const int32_t *seq_lens, int32_t D,
+                                                  float *const *O_parts, float *const *LSE_parts, void *stream);
+
+/*
  * LSE merge of D partials.  [P1 "A2 方法细节", merge equation;
  * P3 §2.3 equivalent local-max/local-sum form]
  *   O[r] = sum_i w_i O_i[r] / sum_i w_i,  w_i = exp(LSE_i[r] - max_j LSE_j[r]),

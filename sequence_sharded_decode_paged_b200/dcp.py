@@ -25,7 +25,7 @@ DCP_LAYOUT_GQA, DCP_LAYOUT_MLA = 0, 1
 EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_build_block_table",
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
-            "dcp_validate_config"]
+            "dcp_validate_config", "dcp_decode_partial_all_noalloc"]
 
 
 class DcpError(RuntimeError):
@@ -60,6 +60,7 @@ def _load() -> C.CDLL:
         "dcp_lse_merge": (C.c_int, [p, p, i32, i32, i32, p, p, p]),
         "dcp_read_device_error": (C.c_int, [p, p, p]),
         "dcp_validate_config": (C.c_int, [i32, i32, i32, i32]),
+        "dcp_decode_partial_all_noalloc": (C.c_int, [p, p, p, p, p, p, i32, p, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -179,6 +180,15 @@ def dcp_decode_partial_all(desc: dcp_attn_desc, q, kv_pools, pool_pages, tables,
     _check("dcp_decode_partial_all", _lib.dcp_decode_partial_all(
         C.byref(desc), _addr(q), _ptr_array(kv_pools), pp.ctypes.data, _ptr_array(tables), _addr(seq_lens), D,
         _ptr_array(O_parts), _ptr_array(LSE_parts), _addr(workspace), n, _stream(stream)))
+
+
+def dcp_decode_partial_all_noalloc(desc: dcp_attn_desc, q, kv_pools, pool_pages, tables, seq_lens, D: int,
+                                   O_parts, LSE_parts, stream=None) -> None:
+    """GQA all-shard partials without a workspace (the library's own fixed scratch; see include/dcp.h)."""
+    pp = _i32(pool_pages)
+    _check("dcp_decode_partial_all_noalloc", _lib.dcp_decode_partial_all_noalloc(
+        C.byref(desc), _addr(q), _ptr_array(kv_pools), pp.ctypes.data, _ptr_array(tables), _addr(seq_lens), D,
+        _ptr_array(O_parts), _ptr_array(LSE_parts), _stream(stream)))
 
 
 def dcp_lse_merge(O_parts, LSE_parts, D: int, rows: int, d_v: int, O, LSE_out=None, stream=None) -> None:

@@ -1,0 +1,78 @@
+"""The allocation-free GQA entry point against the workspace entry point.
+
+dcp_decode_partial_all_noalloc serves callers that cannot allocate device
+memory (plugins handed only their buffers, serving loops that forbid
+allocation after start-up): it runs the same decode kernel on a fixed
+scratch array inside the library.  Its outputs must match
+dcp_decode_partial_all on the same inputs, on two calls in a row (the second
+call reuses the scratch the first one left behind).  This file is collected
+last so that a run stopping at the first failure has run everything else.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_cases import LSE_TOL, O_TOL, build_cache
+from sequence_sharded_decode_paged_b200 import dcp
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_noalloc(cache, q):
+    O = torch.full_like(cache.O_parts, float("nan"))
+    L = torch.full_like(cache.LSE_parts, float("nan"))
+    dcp.dcp_decode_partial_all_noalloc(cache.desc, q, cache.pools, cache.pool_pages, cache.tables,
+                                       cache.seq_lens_dev, cache.D, list(O), list(L))
+    torch.cuda.synchronize()
+    return O, L
+
+
+def _close(a_O, a_L, b_O, b_L):
+    assert torch.isfinite(a_O).all()
+    assert (a_O - b_O).abs().max().item() <= O_TOL
+    inf = torch.isinf(b_L)
+    assert torch.equal(torch.isinf(a_L), inf)
+    if (~inf).any():
+        assert (a_L[~inf] - b_L[~inf]).abs().max().item() <= LSE_TOL
+
+
+@pytest.mark.parametrize("case", [
+    ("gqa_tiny", None, 2),
+    ("mixed", ([5000, 33, 12000, 0, 700], 64, 8, 128, 16), 4),  # splits across CTAs, an empty request
+])
+def test_noalloc_matches_workspace_entry_point_twice(case):
+    name, shape, D = case
+    if shape is None:
+        w = synth.workload(name)
+    else:
+        seq_lens, Hq, Hkv, d, bs = shape
+        w = synth.custom(synth.GQA, seq_lens, Hq, Hkv, d, d, bs, seed=41)
+    cache, q = build_cache(w, D)
+    cache.partials(q)
+    torch.cuda.synchronize()
+    ref_O, ref_L = cache.O_parts.clone(), cache.LSE_parts.clone()
+    for _ in range(2):
+        O, L = _run_noalloc(cache, q)
+        _close(O, L, ref_O, ref_L)
+
+
+def test_noalloc_rejects_problems_larger_than_its_scratch():
+    # 16 query heads per KV head and 8 KV heads per CTA: the split partials need more than 16 MiB.
+    w = synth.custom(synth.GQA, [64], 128, 8, 128, 128, 16, seed=3)
+    cache, q = build_cache(w, 1)
+    assert cache.ws_bytes > 16 << 20
+    with pytest.raises(dcp.DcpError) as e:
+        _run_noalloc(cache, q)
+    assert e.value.status == dcp.DCP_ERR_CAPACITY
+
+
+def test_noalloc_rejects_mla():
+    d = dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07)
+    x = torch.zeros(64 * 576, dtype=torch.int16, device="cuda")
+    o = torch.zeros(64 * 512, dtype=torch.float32, device="cuda")
+    l = torch.zeros(64, dtype=torch.float32, device="cuda")
+    t = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_decode_partial_all_noalloc(d, x, [x], [1], [t], t, 1, [o], [l])
+    assert e.value.status == dcp.DCP_ERR_UNSUPPORTED

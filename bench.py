@@ -173,6 +173,21 @@ def load_workload(args):
     return w
 
 
+def tensor_figures(w, decode_ms: float, peaks: dict, peaks_kind: str):
+    """Tensor-pipe side of the roofline: the method's flops per launch vs the dense bf16 peak.
+
+    Per context token and query head: 2*d_qk (q.k) + 2*d_v (p*v) flops."""
+    flops = w.total_tokens * w.num_q_heads * 2 * (w.head_dim_qk + w.head_dim_v)
+    tf = flops / decode_ms / 1e9
+    peak = peaks["bf16_tflops"]
+    bytes_time = w.total_tokens * w.kv_bytes_per_token / (peaks["hbm_gbs"] * 1e9)
+    flop_time = flops / (peak * 1e12)
+    return {"flops_per_launch": flops, "achieved_tflops": round(tf, 1), "peak_tflops": peak,
+            "frac": round(tf / peak, 4), "peak_kind": f"{peaks_kind} dense bf16 (burst)",
+            "roofline_bound": "hbm" if bytes_time >= flop_time else "tensor",
+            "roofline_us": round(max(bytes_time, flop_time) * 1e6, 2)}
+
+
 def algorithmic_bytes(w, D: int):
     """(KV bytes, decode-kernel bytes, merge bytes) the method must move per step."""
     rows = w.batch * w.num_q_heads
@@ -365,6 +380,7 @@ def run_ours(args, rank, world, local):
         "merge_gbs": round(mrg_b / merge_ms_max / 1e6, 1),
         "context_tokens_per_s": round(world * w.total_tokens / step_ms_max * 1e3, 1),
         "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
+        "tensor": tensor_figures(w, part_ms_max, peaks, peaks_kind),
         "median_step_ms": round(step_med, 4),
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,

@@ -196,9 +196,13 @@ DCP_API dcp_status dcp_decode_partial(const dcp_attn_desc *desc, const void *q, 
                               float *LSE_i, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * All D partials in one launch (the same results as D calls of
- * dcp_decode_partial, bit for bit).  Host arrays of D device pointers:
+ * All D partials in one launch.  Host arrays of D device pointers:
  * kv_pools[s], tables[s], O_parts[s], LSE_parts[s]; pool_pages host int32[D].
+ * Each launch splits the concatenated page lists of its shards into equal
+ * ranges, one per CTA, so the rounding of a result depends on which shards
+ * share the launch: this call and D calls of dcp_decode_partial agree to
+ * rounding (not bit for bit).  Repeating the same call on the same inputs
+ * gives bit-identical results.
  */
 DCP_API dcp_status dcp_decode_partial_all(const dcp_attn_desc *desc, const void *q, const void *const *kv_pools,
                                   const int32_t *pool_pages, const int32_t *const *tables, const int32_t *seq_lens,

@@ -123,6 +123,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// 2^k for an integer-valued k <= 0 (or -inf), exactly: the running maxima of the
+// online softmax are kept integral (in log2 units), so every rescale factor is
+// an exact power of two and P values computed against different maxima differ
+// only by powers of two -- which bf16 rounding preserves, so results do not
+// depend on how a sequence was split (across shards or across CTAs).
+__device__ __forceinline__ float exp2_int(float k) {
+  if (!(k >= -126.f)) return 0.f;  // -inf and tiny factors
+  return __int_as_float(((int)k + 127) << 23);
+}
+
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
 // Byte offset of 16-byte chunk `chunk` of row `row` inside a 128-byte-swizzled
 // tile (TMA CU_TENSOR_MAP_SWIZZLE_128B: rows of 128 B, chunk index XOR row % 8;
 // the tile base must be 1024-byte aligned).

@@ -199,6 +199,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     float o[Geo::kNTiles][4];
 #pragma unroll
     for (int i = 0; i < Geo::kNTiles; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    // One sum of the fp32 weights serves both the normalisation of O and the LSE, so
+    // pieces of a split sequence merge back to exactly the unsplit result (up to
+    // fp32 order); the PV product uses the same weights rounded to bf16.
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
     for (int j = a; j < e; ++j) {
@@ -240,8 +243,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
           mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-          const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-          const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+          // integral running maximum (exact power-of-two rescales, split-independent P)
+          const float mn0 = mx0 > m0 ? ceilf(mx0) : m0, mn1 = mx1 > m1 ? ceilf(mx1) : m1;
+          const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
           m0 = mn0;
           m1 = mn1;
 #pragma unroll
@@ -318,10 +322,8 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           const float ol0 = other[(Geo::kNTiles * 4 + 2) * 32 + lane];
           const float ol1 = other[(Geo::kNTiles * 4 + 3) * 32 + lane];
           const float nm0 = fmaxf(m0, om0), nm1 = fmaxf(m1, om1);
-          const float sa0 = nm0 == -INFINITY ? 0.f : exp2f(m0 - nm0);
-          const float sb0 = nm0 == -INFINITY ? 0.f : exp2f(om0 - nm0);
-          const float sa1 = nm1 == -INFINITY ? 0.f : exp2f(m1 - nm1);
-          const float sb1 = nm1 == -INFINITY ? 0.f : exp2f(om1 - nm1);
+          const float sa0 = exp2_int(m0 - nm0), sb0 = exp2_int(om0 - nm0);
+          const float sa1 = exp2_int(m1 - nm1), sb1 = exp2_int(om1 - nm1);
 #pragma unroll
           for (int i = 0; i < Geo::kNTiles; ++i) {
             o[i][0] = o[i][0] * sa0 + other[(i * 4 + 0) * 32 + lane] * sb0;

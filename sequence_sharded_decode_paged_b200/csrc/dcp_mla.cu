@@ -1,14 +1,564 @@
-// dcp_mla.cu -- MLA (absorbed, shared 576-wide latent) partial decode attention.
+// dcp_mla.cu -- MLA partial decode attention (absorbed form) over D interleaved paged shards.
+//
+// What it computes ("Efficient Decode Context Parallelism with vLLM for Long
+// Context Workloads", A2 方法细节: MLA keeps one latent vector per token shared
+// by every query head, and DCP splits that latent cache along the sequence;
+// "vLLM长序列推理优化：DCP切分KV Cache原理与实战" §2.2/§3.2 for the shard layout):
+// for every shard s, request b and query head h (64 heads),
+//   s_t = scale * q[b][h] . C_t          (C_t: the 576-wide latent row of token t)
+//   O_s[b][h] = sum_t softmax(s)_t * C_t[0:512],  LSE_s[b][h] = log-sum-exp of s,
+// over the tokens of b that shard s stores.
+//
+// Design (121 flop per KV byte, about half the B200 bf16 ridge, so both the
+// HBM stream and the tensor pipe matter):
+//  * Persistent CTAs (one per SM), each owning an equal contiguous range of the
+//    concatenated local page lists of all (shard, request) segments; pieces of
+//    a segment cut by a range boundary are merged by the last CTA to arrive.
+//  * Warp 0 (one thread): TMA producer.  Per segment the query tile (64 x 576
+//    bf16, 72 KB) and per page the latent tile (64 tokens x 576, 72 KB), both
+//    as nine 64 x 64 boxes with 128-byte swizzle, into a 2-stage ring.
+//  * Warp 1: TMEM allocator and the single MMA-issuing thread.
+//      S  = Q K^T   : tcgen05.mma M=64 (heads) N=64 (tokens) K=576, into one of
+//                     two 64-column TMEM buffers (head h in lane h%16 + 32*(h/16)).
+//      O^T += V^T P^T: M=128 (value dims, four tiles) N=64 (heads) K=64 tokens;
+//                     V^T is read straight from the latent tile as an MN-major
+//                     operand, P^T from a 64 x 64 bf16 tile the softmax writes.
+//    S of page i+1 is issued before O of page i, so the tensor pipe works while
+//    the softmax runs.
+//  * Warps 2-5: softmax (one thread per head row of S), fp32, base-2; the
+//    reference maximum is an integer and is only raised (O^T rescaled in TMEM
+//    by an exact power of two) when a page's maximum exceeds it by more than 8
+//    (a factor of 256); the result is unchanged because the final
+//    normalisation uses the same reference.  Tokens
+//    past the sequence end are masked in S and their value rows zeroed in
+//    shared memory before the PV product, so stale cache contents never leak in.
+//    Epilogue: O^T rows (value dims) are read from TMEM, normalised per head
+//    and stored with coalesced 128-byte writes.
+#include <float.h>
+
 #include "dcp_device.cuh"
 #include "dcp_internal.h"
+#include "dcp_tcgen05.cuh"
 
 namespace dcp {
 
+namespace {
+
+constexpr int kMlaThreads = 192;
+constexpr int kMlaHeads = 64;
+constexpr int kMlaDqk = 576;
+constexpr int kMlaDv = 512;
+constexpr int kMlaBs = 64;
+constexpr uint32_t kBlockBytes = 8192;                // 64 rows x 64 bf16, 128-byte swizzled
+constexpr uint32_t kTileBytes = 9 * kBlockBytes;      // 64 rows x 576 bf16
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = kTileBytes;               // two stages
+constexpr uint32_t kOffP = 3 * kTileBytes;            // P^T tile: 64 heads x 64 tokens bf16
+constexpr uint32_t kOffMisc = kOffP + kBlockBytes;
+constexpr uint32_t kMlaSmem = kOffMisc + 2048;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 0;                         // O^T: 4 tiles x 64 columns
+constexpr uint32_t kColS = 256;                       // S: 2 buffers x 64 columns
+constexpr float kRescaleThreshold = 8.0f;             // log2 units
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kSoftmaxThreads = 128;
+
+struct MlaMisc {
+  uint64_t q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, o_free, mma_done;
+  uint32_t tmem_base;
+  int bcast;
+  float alpha[kMlaHeads];
+  float inv_l[kMlaHeads];
+  float lse2[kMlaHeads];
+  int scratch[32];
+};
+static_assert(sizeof(MlaMisc) <= 2048, "misc block");
+
+}  // namespace
+
+struct MlaParams {
+  CUtensorMap kvmap[kMaxShards];
+  CUtensorMap qmap;
+  const int32_t* table[kMaxShards];
+  float* O[kMaxShards];
+  float* LSE[kMaxShards];
+  int pool_pages[kMaxShards];
+  int shard_of_si[kMaxShards];
+  const int32_t* seq_lens;
+  int* status;
+  int* counters;
+  float* slots;
+  float scale_log2;
+  int n_si, B, D, mlb, slot_floats;
+};
+
+namespace {
+
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// Wait unless the caller has already given up; a failed wait marks it dead.
+__device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
+  if (dead) return;
+  if (!mbar_wait(bar, parity)) {
+    atomicOr(status, kDevTimeout);
+    dead = true;
+  }
+}
+
+// Warp-wide variant: the verdict is made uniform across the warp, because the
+// tcgen05.ld / st that follow are warp-collective.
+__device__ __forceinline__ void wait_or_die_warp(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
+  wait_or_die(bar, parity, dead, status);
+  dead = __any_sync(0xffffffffu, dead);
+}
+
+__device__ __forceinline__ bool page_ok(const MlaParams& p, int si, int b, int j, int* page_out) {
+  const int page = p.table[si][(size_t)b * p.mlb + j];
+  *page_out = page;
+  return page >= 0 && page < p.pool_pages[si];
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid_constant__ MlaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x, nctas = gridDim.x;
+  const int B = p.B, D = p.D;
+
+  if ((smem_u32(smem) & 1023u) != 0u) {  // swizzled tiles need 1024-byte alignment
+    if (tid == 0) atomicOr(p.status, kDevTimeout);
+    return;
+  }
+  if (tid == 0) {
+    mbar_init(&misc->q_full, 1);
+    mbar_init(&misc->q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&misc->kv_full[i], 1);
+      mbar_init(&misc->kv_empty[i], 1);
+      mbar_init(&misc->s_full[i], 1);
+      mbar_init(&misc->s_empty[i], 4);
+    }
+    mbar_init(&misc->p_full, 4);
+    mbar_init(&misc->o_done, 1);
+    mbar_init(&misc->o_free, 4);
+    mbar_init(&misc->mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.qmap);
+    for (int si = 0; si < p.n_si; ++si)
+      if (p.pool_pages[si] > 0) prefetch_tmap(&p.kvmap[si]);
+  }
+  if (warp == 1) {
+    tmem_alloc(&misc->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = misc->tmem_base;
+
+  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, kMlaBs, D, cta, nctas, misc->scratch);
+  const int T = plan.T, P = plan.P;
+  const int lo = cta * P, hi = min(lo + P, T);
+  const int S = p.n_si * B;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t st = 0, kv_ph = 0, q_ph = 0;
+      long issued = 0;
+      bool dead = false, q_issued = false;
+      int pre = plan.pre0;
+      for (int sid = plan.sid0; sid < S; ++sid) {
+        const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard);
+        if (seg_first_cta(pre, n, T, P) > cta) break;
+        const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+        pre += n;
+        if (n == 0) continue;
+        wait_or_die(&misc->q_empty, q_ph ^ 1u, dead, p.status);
+        q_ph ^= 1u;
+        if (dead) break;
+        mbar_arrive_expect_tx(&misc->q_full, kTileBytes);
+        for (int cb = 0; cb < 9; ++cb)
+          tma_load_2d(smem + kOffQ + cb * kBlockBytes, &p.qmap, cb * 64, b * kMlaHeads, &misc->q_full);
+        q_issued = true;
+        for (int j = a; j < e; ++j) {
+          int page;
+          const bool ok = page_ok(p, si, b, j, &page);
+          if (!ok) atomicOr(p.status, kDevBadPage);
+          wait_or_die(&misc->kv_empty[st], kv_ph ^ 1u, dead, p.status);
+          if (dead) break;
+          if (ok) {
+            mbar_arrive_expect_tx(&misc->kv_full[st], kTileBytes);
+            uint8_t* dst = smem + kOffKV + st * kTileBytes;
+            for (int cb = 0; cb < 9; ++cb)
+              tma_load_2d(dst + cb * kBlockBytes, &p.kvmap[si], cb * 64, page * kMlaBs, &misc->kv_full[st]);
+          } else {
+            mbar_arrive(&misc->kv_full[st]);
+          }
+          ++issued;
+          if (++st == 2) {
+            st = 0;
+            kv_ph ^= 1u;
+          }
+        }
+        if (dead) break;
+      }
+      // never leave with a copy into shared memory in flight
+      const long first = issued > 2 ? issued - 2 : 0;
+      for (long i = first; i < issued; ++i) {
+        bool d2 = false;
+        wait_or_die(&misc->kv_full[i & 1], (uint32_t)((i >> 1) & 1), d2, p.status);
+      }
+      if (q_issued) {
+        bool d2 = false;
+        wait_or_die(&misc->q_full, q_ph ^ 1u, d2, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16_f32(64, 64, false, false);
+      const uint32_t idO = idesc_bf16_f32(128, 64, true, false);
+      const uint32_t qa = smem_u32(smem + kOffQ), pa = smem_u32(smem + kOffP);
+      uint32_t st = 0, kv_ph = 0, q_ph = 0, p_ph = 0, of_ph = 0;
+      uint32_t gpage = 0;
+      bool dead = false;
+      int pre = plan.pre0;
+      for (int sid = plan.sid0; sid < S && !dead; ++sid) {
+        const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard);
+        if (seg_first_cta(pre, n, T, P) > cta) break;
+        const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+        pre += n;
+        if (n == 0) continue;
+        wait_or_die(&misc->q_full, q_ph, dead, p.status);
+        q_ph ^= 1u;
+        tc_fence_after();
+        bool o_init = false, first_o = true;
+        int prev_st = -1;
+        bool prev_ok = false;
+        auto issue_o = [&](int ost, bool ook) {
+          wait_or_die(&misc->p_full, p_ph, dead, p.status);
+          p_ph ^= 1u;
+          if (first_o) {  // the previous segment's epilogue must have read O^T
+            wait_or_die(&misc->o_free, of_ph ^ 1u, dead, p.status);
+            of_ph ^= 1u;
+            first_o = false;
+          }
+          tc_fence_after();
+          if (ook && !dead) {
+            const uint32_t kva = smem_u32(smem + kOffKV + ost * kTileBytes);
+            for (int mt = 0; mt < 4; ++mt)
+              for (int ks = 0; ks < 4; ++ks)
+                umma_bf16(tbase + kColO + mt * 64, sw128_desc(kva + 2 * mt * kBlockBytes + ks * 2048, kBlockBytes, 1024),
+                          sw128_desc(pa + ks * 32, 16, 1024), idO, (o_init || ks > 0) ? 1u : 0u);
+            o_init = true;
+          }
+          umma_commit(&misc->o_done);
+          umma_commit(&misc->kv_empty[ost]);
+        };
+        for (int j = a; j < e; ++j) {
+          int page;
+          const bool ok = page_ok(p, si, b, j, &page);
+          const uint32_t sb = gpage & 1u;
+          wait_or_die(&misc->kv_full[st], kv_ph, dead, p.status);
+          wait_or_die(&misc->s_empty[sb], ((gpage >> 1) & 1u) ^ 1u, dead, p.status);
+          tc_fence_after();
+          if (ok && !dead) {
+            const uint32_t kva = smem_u32(smem + kOffKV + st * kTileBytes);
+            for (int ks = 0; ks < 36; ++ks) {
+              const uint32_t off = (ks >> 2) * kBlockBytes + (ks & 3) * 32;
+              umma_bf16(tbase + kColS + sb * 64, sw128_desc(qa + off, 16, 1024), sw128_desc(kva + off, 16, 1024), idS,
+                        ks > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(&misc->s_full[sb]);
+          if (prev_st >= 0) issue_o(prev_st, prev_ok);
+          prev_st = (int)st;
+          prev_ok = ok;
+          ++gpage;
+          if (++st == 2) {
+            st = 0;
+            kv_ph ^= 1u;
+          }
+        }
+        umma_commit(&misc->q_empty);  // Q is free once the S products above are done
+        if (prev_st >= 0) issue_o(prev_st, prev_ok);
+      }
+      umma_commit(&misc->mma_done);  // everything issued has completed before TMEM is released
+      bool d2 = false;
+      wait_or_die(&misc->mma_done, 0, d2, p.status);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue (warps 2-5)
+    const int q4 = warp & 3;
+    const int ts = tid - 64;                       // 0..127
+    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    const bool head_thread = lane < 16;
+    const int h = 16 * q4 + (lane & 15);           // head row of S held by this thread
+    uint32_t gpage = 0, od_ph = 0, st = 0;
+    bool dead = false;
+    int pre = plan.pre0;
+    for (int sid = plan.sid0; sid < S; ++sid) {
+      const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+      const int seq_len = p.seq_lens[b];
+      const int n = local_pages(seq_len, kMlaBs, D, shard);
+      const int c0 = seg_first_cta(pre, n, T, P);
+      if (c0 > cta) break;
+      const int c1 = seg_last_cta(pre, n, T, P);
+      float* Oout = p.O[si] + (size_t)b * kMlaHeads * kMlaDv;
+      float* Lout = p.LSE[si] + (size_t)b * kMlaHeads;
+      if (n == 0) {
+        for (int i = ts; i < kMlaHeads * kMlaDv / 4; i += kSoftmaxThreads)
+          reinterpret_cast<float4*>(Oout)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (ts < kMlaHeads) Lout[ts] = -INFINITY;
+        pre += n;
+        continue;
+      }
+      const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+      // One sum of the fp32 weights normalises O and gives the LSE, so pieces of a
+      // split sequence merge back to the unsplit result (up to fp32 order); the
+      // PV product uses the same weights rounded to bf16.
+      float m_used = -INFINITY, lsum = 0.f;
+      bool have_o = false;
+      for (int j = a; j < e; ++j) {
+        int page;
+        const bool ok = page_ok(p, si, b, j, &page);
+        const int valid = min(kMlaBs, seq_len - (j * D + shard) * kMlaBs);
+        const uint32_t sb = gpage & 1u;
+        wait_or_die_warp(&misc->s_full[sb], (gpage >> 1) & 1u, dead, p.status);
+        tc_fence_after();
+        float s[64];
+        if (ok && !dead) {
+          tmem_ld32(tbase + lane_off + kColS + sb * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
+          tmem_ld32(tbase + lane_off + kColS + sb * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&misc->s_empty[sb]);
+        bool need = false;
+        float alpha = 1.f;
+        if (ok && !dead) {
+          float pmax = -INFINITY;
+#pragma unroll
+          for (int t = 0; t < 64; ++t) {
+            s[t] = t < valid ? s[t] * p.scale_log2 : -INFINITY;
+            pmax = fmaxf(pmax, s[t]);
+          }
+          if (m_used == -INFINITY || pmax > m_used + kRescaleThreshold) {
+            const float m_new = ceilf(pmax);  // integral reference: exact power-of-two rescale
+            alpha = exp2_int(m_used - m_new);
+            m_used = m_new;
+            need = have_o && head_thread;
+          }
+          float psum = 0.f;
+#pragma unroll
+          for (int t = 0; t < 64; ++t) {
+            s[t] = exp2f(s[t] - m_used);
+            psum += s[t];
+          }
+          lsum = lsum * alpha + psum;
+        }
+        if (j > a) {  // O^T of the previous page is complete: P and O^T may be touched
+          wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
+          od_ph ^= 1u;
+          tc_fence_after();
+        }
+        if (bar_red_or(2, kSoftmaxThreads, need)) {
+          if (head_thread) misc->alpha[h] = need ? alpha : 1.f;
+          named_bar_sync(2, kSoftmaxThreads);
+          if (!dead) {
+#pragma unroll 1
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll 1
+              for (int c = 0; c < 64; c += 32) {
+                float v[32];
+                const uint32_t ta = tbase + lane_off + kColO + mt * 64 + c;
+                tmem_ld32(ta, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= misc->alpha[c + i];
+                tmem_st32(ta, v);
+              }
+            tmem_st_wait();
+          }
+        }
+        if (ok && !dead) {
+          uint8_t* kv = smem + kOffKV + st * kTileBytes;
+          if (valid < kMlaBs) {  // zero the value rows of tokens past the end (dims 0..511)
+            const int nchunks = (kMlaBs - valid) * 64;
+            for (int i = ts; i < nchunks; i += kSoftmaxThreads) {
+              const int row = valid + (i >> 6), cb = (i >> 3) & 7, ch = i & 7;
+              *reinterpret_cast<uint4*>(kv + cb * kBlockBytes + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          if (head_thread) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4 w;
+              w.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
+              w.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
+              w.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
+              w.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
+              *reinterpret_cast<uint4*>(smem + kOffP + sw128((uint32_t)h, (uint32_t)c)) = w;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&misc->p_full);
+        have_o = have_o || ok;
+        ++gpage;
+        st ^= 1u;
+      }
+      // ---------------------------------------------------------- epilogue
+      wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
+      od_ph ^= 1u;
+      tc_fence_after();
+      if (head_thread) {
+        misc->inv_l[h] = (lsum > 0.f && have_o) ? 1.f / lsum : 0.f;
+        misc->lse2[h] = (lsum > 0.f && have_o) ? m_used + __log2f(lsum) : -INFINITY;
+      }
+      named_bar_sync(2, kSoftmaxThreads);
+      const bool complete = (c0 == c1);
+      const int slot = complete ? 0 : 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
+      float* dstO = complete ? Oout : p.slots + (size_t)slot * p.slot_floats;
+      float* dstL = complete ? Lout : p.slots + (size_t)slot * p.slot_floats + kMlaHeads * kMlaDv;
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll 1
+        for (int c = 0; c < 64; c += 32) {
+          float v[32];
+          if (!dead) {
+            tmem_ld32(tbase + lane_off + kColO + mt * 64 + c, v);
+            tmem_ld_wait();
+          }
+          const int dv = mt * 128 + 32 * q4 + lane;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float inv = misc->inv_l[c + i];
+            dstO[(size_t)(c + i) * kMlaDv + dv] = (inv == 0.f || dead) ? 0.f : v[i] * inv;
+          }
+        }
+      if (ts < kMlaHeads) dstL[ts] = complete ? misc->lse2[ts] * kLn2 : misc->lse2[ts];
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&misc->o_free);
+      if (!complete) {
+        __threadfence();
+        named_bar_sync(2, kSoftmaxThreads);
+        int* ctr = p.counters + sid;
+        if (ts == 0) misc->bcast = (atomicAdd(ctr, 1) == c1 - c0) ? 1 : 0;
+        named_bar_sync(2, kSoftmaxThreads);
+        if (misc->bcast) {
+          __threadfence();
+          const int w4 = ts >> 5;
+          for (int r = w4; r < kMlaHeads; r += 4) {
+            float mx = -INFINITY;
+            for (int c = c0; c <= c1; ++c) {
+              const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+              mx = fmaxf(mx, __ldcg(p.slots + (size_t)k * p.slot_floats + kMlaHeads * kMlaDv + r));
+            }
+            float4 acc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            float wsum = 0.f;
+            if (mx != -INFINITY) {
+              for (int c = c0; c <= c1; ++c) {
+                const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                const float* sl = p.slots + (size_t)k * p.slot_floats;
+                const float lk = __ldcg(sl + kMlaHeads * kMlaDv + r);
+                const float w = lk == -INFINITY ? 0.f : exp2f(lk - mx);
+                wsum += w;
+                const float4* src = reinterpret_cast<const float4*>(sl + (size_t)r * kMlaDv) + lane * 4;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float4 x = __ldcg(src + i);
+                  acc[i].x += w * x.x;
+                  acc[i].y += w * x.y;
+                  acc[i].z += w * x.z;
+                  acc[i].w += w * x.w;
+                }
+              }
+            }
+            const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+            float4* out = reinterpret_cast<float4*>(Oout + (size_t)r * kMlaDv) + lane * 4;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) out[i] = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
+            if (lane == 0) Lout[r] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+          }
+          if (ts == 0) *ctr = 0;  // ready for the next call
+        }
+      }
+      pre += n;
+    }
+  }
+
+  // ---------------------------------------------------------------- release TMEM
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------- host side
 int mla_ctas() { return device_sm_count(); }
 
-dcp_status launch_mla_decode(const dcp_attn_desc&, int, const ShardSet&, const void*, const int32_t*, void*, size_t,
-                             cudaStream_t) {
-  return DCP_ERR_UNSUPPORTED;
+dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
+                             const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  WorkspaceLayout L;
+  if (!workspace_layout(d, D, &L)) return DCP_ERR_UNSUPPORTED;
+  if (ws_bytes < L.total) return DCP_ERR_CAPACITY;
+  MlaParams p;
+  memset(&p, 0, sizeof(p));
+  p.n_si = set.n;
+  p.B = d.batch;
+  p.D = D;
+  p.mlb = d.max_local_blocks;
+  p.slot_floats = L.slot_floats;
+  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.seq_lens = seq_lens;
+  p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
+  p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);
+  p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slots_off);
+  if ((uint64_t)d.batch * kMlaHeads > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;
+  if (encode_tiled_2d(&p.qmap, q, kMlaDqk, (uint64_t)d.batch * kMlaHeads, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS)
+    return DCP_ERR_CUDA;
+  for (int si = 0; si < set.n; ++si) {
+    p.table[si] = set.table[si];
+    p.O[si] = set.O[si];
+    p.LSE[si] = set.LSE[si];
+    p.pool_pages[si] = set.pool_pages[si];
+    p.shard_of_si[si] = set.shard[si];
+    if (set.pool_pages[si] > 0) {
+      const uint64_t rows = (uint64_t)set.pool_pages[si] * kMlaBs;
+      if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+      if (encode_tiled_2d(&p.kvmap[si], set.pool[si], kMlaDqk, rows, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS)
+        return DCP_ERR_CUDA;
+    }
+  }
+  if (cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMlaSmem) !=
+      cudaSuccess)
+    return DCP_ERR_CUDA;
+  mla_decode_kernel<<<L.nctas, kMlaThreads, kMlaSmem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
 }
 
 }  // namespace dcp

@@ -108,7 +108,13 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 
 def values_bf16(seed: int, tensor: int, request: int, e0: int, n: int, amp: float) -> np.ndarray:
-    """bf16 bit patterns of elements ``e0 .. e0+n-1`` of one stream."""
+    """bf16 bit patterns of elements ``e0 .. e0+n-1`` of one stream (generated in chunks)."""
+    chunk = 1 << 23
+    if n > chunk:
+        out = np.empty(n, dtype=np.uint16)
+        for c0 in range(0, n, chunk):
+            out[c0:c0 + chunk] = values_bf16(seed, tensor, request, e0 + c0, min(chunk, n - c0), amp)
+        return out
     with np.errstate(over="ignore"):
         key = np.uint64(stream_key(seed, tensor, request))
         e = np.arange(e0, e0 + n, dtype=np.uint64)

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 import synth
-from gpu_cases import (D_INVARIANCE_TOL, LSE_TOL, O_TOL, assert_lse_close, assert_o_close, build_cache, host_kv,
+from gpu_cases import (D_INVARIANCE_TOL, LSE_TOL, O_BOUND_UNIT_AMP, O_TOL, assert_lse_close, assert_o_close, build_cache, host_kv,
                        host_q, oracle_request)
 
 pytestmark = pytest.mark.gpu
@@ -61,7 +61,7 @@ def test_tiny_workload_parity():
     cache.step(q)
     torch.cuda.synchronize()
     err = _check_against_oracle(w, 2, cache)
-    assert err < 5e-3  # bf16 P rounding only: far inside the 2e-2 bound
+    assert err < O_BOUND_UNIT_AMP  # bf16 rounding of the weights only
     assert cache.device_error() == 0
 
 
@@ -73,13 +73,19 @@ def test_tiny_workload_all_D(D):
     _check_against_oracle(w, D, cache)
 
 
-def test_per_shard_calls_equal_one_launch_bit_for_bit():
+def test_per_shard_calls_agree_with_one_launch():
     w = synth.custom(synth.GQA, [300, 17, 1000, 64], 16, 2, 128, 128, 16, seed=21)
     cache, q = build_cache(w, 4, perm_seed=3)
     cache.partials(q, per_shard=False)
     a = (cache.O_parts.clone(), cache.LSE_parts.clone())
     cache.partials(q, per_shard=True)
-    assert torch.equal(a[0], cache.O_parts) and torch.equal(a[1], cache.LSE_parts)
+    # different launches split the page lists differently; with integral softmax
+    # reference maxima the bf16 P values do not depend on the split, so the two
+    # agree to fp32 accumulation order
+    assert (a[0] - cache.O_parts).abs().max().item() <= 1e-4
+    inf = torch.isinf(a[1])
+    assert torch.equal(inf, torch.isinf(cache.LSE_parts))
+    assert (a[1][~inf] - cache.LSE_parts[~inf]).abs().max().item() <= LSE_TOL
 
 
 def test_repeated_steps_are_identical():

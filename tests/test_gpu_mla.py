@@ -1,0 +1,131 @@
+"""MLA (absorbed, 576-wide shared latent) parity on the GPU vs the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_cases import (D_INVARIANCE_TOL, LSE_TOL, O_BOUND_UNIT_AMP, O_TOL, assert_lse_close, assert_o_close, build_cache, host_kv)
+
+pytestmark = pytest.mark.gpu
+
+HEADS_SAMPLE = [(0, 8), (56, 64)]  # head ranges checked on the big workloads
+
+
+def _oracle(w, b, D, heads=None, src=None):
+    src = w.kv_source(b) if src is None else src
+    return oracle.sharded(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.query(b),
+                          src, w.softmax_scale, w.block_size, D, heads)
+
+
+def _check(w, D, cache, requests=None, heads=None):
+    reqs = range(w.batch) if requests is None else requests
+    Op = cache.O_parts.cpu().numpy()
+    Lp = cache.LSE_parts.cpu().numpy()
+    O = cache.O.cpu().numpy()
+    L = cache.LSE.cpu().numpy()
+    worst = 0.0
+    for b in reqs:
+        src = w.kv_source(b)
+        for hb, he in (heads or [(0, w.num_q_heads)]):
+            Ob, Lb, Opb, Lpb = _oracle(w, b, D, (hb, he), src)
+            for s in range(D):
+                worst = max(worst, assert_o_close(Op[s, b, hb:he], Opb[s, hb:he], O_TOL, f"O_{s}[{b}]"))
+                assert_lse_close(Lp[s, b, hb:he], Lpb[s, hb:he], LSE_TOL, f"LSE_{s}[{b}]")
+            worst = max(worst, assert_o_close(O[b, hb:he], Ob[hb:he], O_TOL, f"O[{b}]"))
+            assert_lse_close(L[b, hb:he], Lb[hb:he], LSE_TOL, f"LSE[{b}]")
+    return worst
+
+
+@pytest.mark.parametrize("case", [
+    ([1], 1), ([64], 1), ([65], 2), ([70, 3, 200], 2), ([0, 130, 64, 129], 4),
+    ([1000, 31, 257], 3), ([4097, 64], 8), ([300] * 5, 16),
+])
+def test_small_parity(case):
+    seq_lens, D = case
+    w = synth.custom(synth.MLA, seq_lens, 64, 1, 576, 512, 64, seed=sum(seq_lens) + D)
+    cache, q = build_cache(w, D, perm_seed=11)
+    cache.step(q)
+    torch.cuda.synchronize()
+    err = _check(w, D, cache)
+    assert err < O_BOUND_UNIT_AMP  # bf16 rounding of the weights only
+    assert cache.device_error() == 0
+
+
+def test_per_shard_calls_agree_with_one_launch():
+    w = synth.custom(synth.MLA, [2000, 65, 9000, 1], 64, 1, 576, 512, 64, seed=5)
+    cache, q = build_cache(w, 4)
+    cache.partials(q)
+    a = (cache.O_parts.clone(), cache.LSE_parts.clone())
+    cache.partials(q, per_shard=True)
+    # different launches split the page lists differently; with integral softmax
+    # reference maxima the bf16 P values do not depend on the split, so the two
+    # agree to fp32 accumulation order
+    assert (a[0] - cache.O_parts).abs().max().item() <= 1e-4
+    inf = torch.isinf(a[1])
+    assert torch.equal(inf, torch.isinf(cache.LSE_parts))
+    assert (a[1][~inf] - cache.LSE_parts[~inf]).abs().max().item() <= LSE_TOL
+    cache.partials(q)  # the same launch again: bit for bit
+    assert torch.equal(a[0], cache.O_parts) and torch.equal(a[1], cache.LSE_parts)
+
+
+def test_d_invariance():
+    w = synth.custom(synth.MLA, [5000, 700, 64, 12345, 3], 64, 1, 576, 512, 64, seed=6)
+    outs = []
+    for D in (1, 2, 4, 8):
+        cache, q = build_cache(w, D)
+        O, _ = cache.step(q)
+        outs.append(O.cpu().numpy())
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= D_INVARIANCE_TOL
+
+
+def test_out_of_range_page_is_reported_and_skipped():
+    w = synth.custom(synth.MLA, [200, 130], 64, 1, 576, 512, 64, seed=7)
+    cache, q = build_cache(w, 2)
+    bad = cache.tables[0].clone()
+    bad[1, 0] = int(cache.pool_pages[0]) + 3
+    cache.tables[0].copy_(bad)
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 1
+    assert torch.isfinite(cache.O).all()
+
+
+@pytest.mark.parametrize("name", ["mla_b32", "mla_long"])
+def test_full_size_workload_sampled(name):
+    w = synth.workload(name)
+    D = w.shards[0]
+    cache, q = build_cache(w, D, device_kv=True)
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    assert torch.isfinite(cache.O).all() and torch.isfinite(cache.LSE).all()
+    lens = np.array(w.seq_lens)
+    sample = sorted({int(lens.argmin()), int(np.argsort(lens)[len(lens) // 2])})
+    _check(w, D, cache, requests=sample, heads=HEADS_SAMPLE)
+    del cache
+    torch.cuda.empty_cache()
+
+
+def test_agentic_mix_all_D_sampled_and_invariant():
+    """256 requests, 17.8 M context tokens (20.5 GB of latent cache) at D = 1, 2, 4, 8."""
+    w = synth.workload("mla_mix")
+    lens = np.array(w.seq_lens)
+    sample = sorted({int(lens.argmin()), int(np.argsort(lens)[128])})
+    ref = None
+    for D in w.shards:
+        cache, q = build_cache(w, D, device_kv=True)
+        cache.step(q)
+        torch.cuda.synchronize()
+        assert cache.device_error() == 0
+        O = cache.O.cpu().numpy()
+        assert np.isfinite(O).all()
+        if D in (1, 8):
+            _check(w, D, cache, requests=sample, heads=[(0, 4)])
+        if ref is None:
+            ref = O
+        else:
+            assert np.abs(O - ref).max() <= D_INVARIANCE_TOL
+        del cache, q
+        torch.cuda.empty_cache()

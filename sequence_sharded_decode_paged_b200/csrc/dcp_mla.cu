@@ -25,7 +25,7 @@
 //                     operand, P^T from a 64 x 64 bf16 tile the softmax writes.
 //    S of page i+1 is issued before O of page i, so the tensor pipe works while
 //    the softmax runs.
-//  * Warps 2-5: softmax (one thread per head row of S), fp32, base-2; the
+//  * Warps 2-5: softmax (four threads per head row of S), fp32, base-2; the
 //    reference maximum is an integer and is only raised (O^T rescaled in TMEM
 //    by an exact power of two) when a page's maximum exceeds it by more than 8
 //    (a factor of 256); the result is unchanged because the final
@@ -60,6 +60,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                         // O^T: 4 tiles x 64 columns
 constexpr uint32_t kColS = 256;                       // S: 2 buffers x 64 columns
 constexpr float kRescaleThreshold = 8.0f;             // log2 units
+constexpr int kPrefetchPages = 4;                     // L2 prefetch distance of the producer, in pages
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSoftmaxThreads = 128;
 
@@ -79,6 +80,7 @@ static_assert(sizeof(MlaMisc) <= 2048, "misc block");
 struct MlaParams {
   CUtensorMap kvmap[kMaxShards];
   CUtensorMap qmap;
+  const uint8_t* pool[kMaxShards];
   const int32_t* table[kMaxShards];
   float* O[kMaxShards];
   float* LSE[kMaxShards];
@@ -179,6 +181,36 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       uint32_t st = 0, kv_ph = 0, q_ph = 0;
       long issued = 0;
       bool dead = false, q_issued = false;
+      // A second cursor walks the same page sequence kPrefetchPages ahead and pulls
+      // those pages into L2, so the HBM stream does not wait for a free stage.
+      int pf_sid = plan.sid0, pf_pre = plan.pre0, pf_j = 0, pf_e = 0, pf_si = 0, pf_b = 0;
+      bool pf_live = true;
+      long pf_count = 0;
+      auto pf_advance = [&]() {  // next page of the CTA's walk into (pf_si, pf_b, pf_j), false at the end
+        while (pf_live) {
+          if (pf_j < pf_e) return true;
+          if (pf_sid >= S) { pf_live = false; break; }
+          const int si2 = pf_sid / B, b2 = pf_sid - si2 * B;
+          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2]);
+          if (seg_first_cta(pf_pre, n2, T, P) > cta) { pf_live = false; break; }
+          pf_si = si2;
+          pf_b = b2;
+          pf_j = max(pf_pre, lo) - pf_pre;
+          pf_e = n2 > 0 ? min(pf_pre + n2, hi) - pf_pre : 0;
+          pf_pre += n2;
+          ++pf_sid;
+        }
+        return false;
+      };
+      auto pf_until = [&](long target) {  // prefetch pages with index < target
+        while (pf_count < target && pf_advance()) {
+          const int page = p.table[pf_si][(size_t)pf_b * p.mlb + pf_j];
+          if (page >= 0 && page < p.pool_pages[pf_si])
+            prefetch_l2_bulk(p.pool[pf_si] + (size_t)page * kTileBytes, kTileBytes);
+          ++pf_j;
+          ++pf_count;
+        }
+      };
       int pre = plan.pre0;
       for (int sid = plan.sid0; sid < S; ++sid) {
         const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
@@ -198,6 +230,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           int page;
           const bool ok = page_ok(p, si, b, j, &page);
           if (!ok) atomicOr(p.status, kDevBadPage);
+          pf_until(issued + 1 + kPrefetchPages);
           wait_or_die(&misc->kv_empty[st], kv_ph ^ 1u, dead, p.status);
           if (dead) break;
           if (ok) {
@@ -229,74 +262,118 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Two cursors over the CTA's page sequence: S = Q K^T of page js and
+    // O^T += V^T P^T of page jo < js, each issued as soon as its inputs are
+    // ready (O first: it frees a stage for the next load).  The tensor pipe
+    // executes in issue order, so this keeps a late page load from holding
+    // back the PV product of the page before it.
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64, false, false);
       const uint32_t idO = idesc_bf16_f32(128, 64, true, false);
       const uint32_t qa = smem_u32(smem + kOffQ), pa = smem_u32(smem + kOffP);
-      uint32_t st = 0, kv_ph = 0, q_ph = 0, p_ph = 0, of_ph = 0;
-      uint32_t gpage = 0;
-      bool dead = false;
-      int pre = plan.pre0;
-      for (int sid = plan.sid0; sid < S && !dead; ++sid) {
-        const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
-        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard);
-        if (seg_first_cta(pre, n, T, P) > cta) break;
-        const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
-        pre += n;
-        if (n == 0) continue;
-        wait_or_die(&misc->q_full, q_ph, dead, p.status);
-        q_ph ^= 1u;
-        tc_fence_after();
-        bool o_init = false, first_o = true;
-        int prev_st = -1;
-        bool prev_ok = false;
-        auto issue_o = [&](int ost, bool ook) {
-          wait_or_die(&misc->p_full, p_ph, dead, p.status);
+      struct PageRec {
+        bool ok, seg_first, seg_last;
+      };
+      PageRec ring[4];
+      uint32_t q_ph = 0, p_ph = 0, of_ph = 0;
+      long js = 0, jo = 0, known = 0;  // S issued, O issued, pages enumerated
+      bool dead = false, o_init = false;
+      // segment walk producing page records
+      int w_sid = plan.sid0, w_pre = plan.pre0, w_j = 0, w_e = 0, w_si = 0, w_b = 0, w_a = 0;
+      bool w_live = true;
+      auto enumerate = [&]() {  // append the next page record to the ring; false at the end
+        while (w_live) {
+          if (w_j < w_e) {
+            int page;
+            PageRec r;
+            r.ok = page_ok(p, w_si, w_b, w_j, &page);
+            r.seg_first = (w_j == w_a);
+            r.seg_last = (w_j == w_e - 1);
+            ring[known & 3] = r;
+            ++known;
+            ++w_j;
+            return true;
+          }
+          if (w_sid >= S) { w_live = false; break; }
+          const int si2 = w_sid / B, b2 = w_sid - si2 * B;
+          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2]);
+          if (seg_first_cta(w_pre, n2, T, P) > cta) { w_live = false; break; }
+          w_si = si2;
+          w_b = b2;
+          w_a = w_j = max(w_pre, lo) - w_pre;
+          w_e = n2 > 0 ? min(w_pre + n2, hi) - w_pre : 0;
+          w_pre += n2;
+          ++w_sid;
+        }
+        return false;
+      };
+      unsigned long long idle_since = 0;
+      while (!dead) {
+        if (known == js) enumerate();
+        bool progressed = false;
+        if (jo < js && mbar_test(&misc->p_full, p_ph)) {
+          const PageRec r = ring[jo & 3];
           p_ph ^= 1u;
-          if (first_o) {  // the previous segment's epilogue must have read O^T
+          if (r.seg_first) {  // the previous segment's epilogue must have read O^T
             wait_or_die(&misc->o_free, of_ph ^ 1u, dead, p.status);
             of_ph ^= 1u;
-            first_o = false;
+            o_init = false;
           }
           tc_fence_after();
-          if (ook && !dead) {
-            const uint32_t kva = smem_u32(smem + kOffKV + ost * kTileBytes);
+          const uint32_t ost = (uint32_t)(jo & 1);
+          if (r.ok && !dead) {
+            const uint64_t ad = sw128_desc(smem_u32(smem + kOffKV + ost * kTileBytes), kBlockBytes, 1024);
+            const uint64_t bd = sw128_desc(pa, 16, 1024);
+#pragma unroll
             for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(tbase + kColO + mt * 64, sw128_desc(kva + 2 * mt * kBlockBytes + ks * 2048, kBlockBytes, 1024),
-                          sw128_desc(pa + ks * 32, 16, 1024), idO, (o_init || ks > 0) ? 1u : 0u);
+                umma_bf16(tbase + kColO + mt * 64, ad + (uint64_t)((2 * mt * kBlockBytes + ks * 2048) >> 4),
+                          bd + (uint64_t)((ks * 32) >> 4), idO, (o_init || ks > 0) ? 1u : 0u);
             o_init = true;
           }
           umma_commit(&misc->o_done);
           umma_commit(&misc->kv_empty[ost]);
-        };
-        for (int j = a; j < e; ++j) {
-          int page;
-          const bool ok = page_ok(p, si, b, j, &page);
-          const uint32_t sb = gpage & 1u;
-          wait_or_die(&misc->kv_full[st], kv_ph, dead, p.status);
-          wait_or_die(&misc->s_empty[sb], ((gpage >> 1) & 1u) ^ 1u, dead, p.status);
-          tc_fence_after();
-          if (ok && !dead) {
-            const uint32_t kva = smem_u32(smem + kOffKV + st * kTileBytes);
-            for (int ks = 0; ks < 36; ++ks) {
-              const uint32_t off = (ks >> 2) * kBlockBytes + (ks & 3) * 32;
-              umma_bf16(tbase + kColS + sb * 64, sw128_desc(qa + off, 16, 1024), sw128_desc(kva + off, 16, 1024), idS,
-                        ks > 0 ? 1u : 0u);
+          ++jo;
+          progressed = true;
+        }
+        if (js < known && js - jo < 2) {
+          const PageRec r = ring[js & 3];
+          const uint32_t st = (uint32_t)(js & 1), par = (uint32_t)((js >> 1) & 1);
+          const bool ready = (!r.seg_first || mbar_test(&misc->q_full, q_ph)) && mbar_test(&misc->kv_full[st], par) &&
+                             mbar_test(&misc->s_empty[st], par ^ 1u);
+          if (ready) {
+            if (r.seg_first) q_ph ^= 1u;
+            tc_fence_after();
+            if (r.ok) {
+              // descriptors advance by adding (byte offset >> 4) to the start-address field
+              const uint64_t ad = sw128_desc(qa, 16, 1024);
+              const uint64_t bd = sw128_desc(smem_u32(smem + kOffKV + st * kTileBytes), 16, 1024);
+              const uint32_t dS = tbase + kColS + st * 64;
+#pragma unroll
+              for (int ks = 0; ks < 36; ++ks) {
+                const uint64_t off = (uint64_t)(((ks >> 2) * kBlockBytes + (ks & 3) * 32) >> 4);
+                umma_bf16(dS, ad + off, bd + off, idS, ks > 0 ? 1u : 0u);
+              }
             }
-          }
-          umma_commit(&misc->s_full[sb]);
-          if (prev_st >= 0) issue_o(prev_st, prev_ok);
-          prev_st = (int)st;
-          prev_ok = ok;
-          ++gpage;
-          if (++st == 2) {
-            st = 0;
-            kv_ph ^= 1u;
+            umma_commit(&misc->s_full[st]);
+            if (r.seg_last) umma_commit(&misc->q_empty);  // Q is free once these S products are done
+            ++js;
+            progressed = true;
           }
         }
-        umma_commit(&misc->q_empty);  // Q is free once the S products above are done
-        if (prev_st >= 0) issue_o(prev_st, prev_ok);
+        if (js == known && jo == js && !w_live) break;
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const unsigned long long now = global_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            atomicOr(p.status, kDevTimeout);
+            dead = true;
+          }
+        }
       }
       umma_commit(&misc->mma_done);  // everything issued has completed before TMEM is released
       bool d2 = false;
@@ -304,11 +381,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 2-5)
+    // Warp q (= warp % 4) owns head rows 16q..16q+15 of S (TMEM lanes 32q..32q+15);
+    // with the 16x256b load all 32 lanes share them: thread t holds heads
+    // hr0 = 16q + t/4 and hr1 = hr0 + 8, tokens 8k + 2*(t%4) + {0,1}, k = 0..7.
     const int q4 = warp & 3;
     const int ts = tid - 64;                       // 0..127
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const bool head_thread = lane < 16;
-    const int h = 16 * q4 + (lane & 15);           // head row of S held by this thread
+    const int quad = lane & 3;
+    const int hr0 = 16 * q4 + (lane >> 2), hr1 = hr0 + 8;
     uint32_t gpage = 0, od_ph = 0, st = 0;
     bool dead = false;
     int pre = plan.pre0;
@@ -331,8 +411,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
       // One sum of the fp32 weights normalises O and gives the LSE, so pieces of a
       // split sequence merge back to the unsplit result (up to fp32 order); the
-      // PV product uses the same weights rounded to bf16.
-      float m_used = -INFINITY, lsum = 0.f;
+      // PV product uses the same weights rounded to bf16.  l0 / l1 are this
+      // thread's partial sums (its 16 tokens of each page), reduced at the end.
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
       bool have_o = false;
       for (int j = a; j < e; ++j) {
         int page;
@@ -341,37 +422,64 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         const uint32_t sb = gpage & 1u;
         wait_or_die_warp(&misc->s_full[sb], (gpage >> 1) & 1u, dead, p.status);
         tc_fence_after();
-        float s[64];
+        float s[32];
         if (ok && !dead) {
-          tmem_ld32(tbase + lane_off + kColS + sb * 64, *reinterpret_cast<float(*)[32]>(&s[0]));
-          tmem_ld32(tbase + lane_off + kColS + sb * 64 + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+          tmem_ld16x256b_x8(tbase + lane_off + kColS + sb * 64, s);
           tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&misc->s_empty[sb]);
         bool need = false;
-        float alpha = 1.f;
+        float a0 = 1.f, a1 = 1.f;
         if (ok && !dead) {
-          float pmax = -INFINITY;
 #pragma unroll
-          for (int t = 0; t < 64; ++t) {
-            s[t] = t < valid ? s[t] * p.scale_log2 : -INFINITY;
-            pmax = fmaxf(pmax, s[t]);
-          }
-          if (m_used == -INFINITY || pmax > m_used + kRescaleThreshold) {
-            const float m_new = ceilf(pmax);  // integral reference: exact power-of-two rescale
-            alpha = exp2_int(m_used - m_new);
-            m_used = m_new;
-            need = have_o && head_thread;
-          }
-          float psum = 0.f;
+          for (int k = 0; k < 8; ++k)
 #pragma unroll
-          for (int t = 0; t < 64; ++t) {
-            s[t] = exp2f(s[t] - m_used);
-            psum += s[t];
+            for (int i = 0; i < 4; ++i) {
+              const int tok = 8 * k + 2 * quad + (i & 1);
+              s[4 * k + i] = tok < valid ? s[4 * k + i] * p.scale_log2 : -INFINITY;
+            }
+          float x0 = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5]));
+          float x1 = fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7]));
+          float y0 = fmaxf(fmaxf(s[8], s[9]), fmaxf(s[12], s[13]));
+          float y1 = fmaxf(fmaxf(s[10], s[11]), fmaxf(s[14], s[15]));
+          float z0 = fmaxf(fmaxf(s[16], s[17]), fmaxf(s[20], s[21]));
+          float z1 = fmaxf(fmaxf(s[18], s[19]), fmaxf(s[22], s[23]));
+          float w0 = fmaxf(fmaxf(s[24], s[25]), fmaxf(s[28], s[29]));
+          float w1 = fmaxf(fmaxf(s[26], s[27]), fmaxf(s[30], s[31]));
+          float pm0 = fmaxf(fmaxf(x0, y0), fmaxf(z0, w0));
+          float pm1 = fmaxf(fmaxf(x1, y1), fmaxf(z1, w1));
+          pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 1));
+          pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 2));
+          pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 1));
+          pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 2));
+          // integral reference maximum, raised only past the threshold (exact power-of-two rescale)
+          if (m0 == -INFINITY || pm0 > m0 + kRescaleThreshold) {
+            const float mn = ceilf(pm0);
+            a0 = exp2_int(m0 - mn);
+            m0 = mn;
+            need = have_o;
           }
-          lsum = lsum * alpha + psum;
+          if (m1 == -INFINITY || pm1 > m1 + kRescaleThreshold) {
+            const float mn = ceilf(pm1);
+            a1 = exp2_int(m1 - mn);
+            m1 = mn;
+            need = need || have_o;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            s[4 * k + 0] = ex2_approx(s[4 * k + 0] - m0);
+            s[4 * k + 1] = ex2_approx(s[4 * k + 1] - m0);
+            s[4 * k + 2] = ex2_approx(s[4 * k + 2] - m1);
+            s[4 * k + 3] = ex2_approx(s[4 * k + 3] - m1);
+          }
+          const float e0 = ((s[0] + s[1]) + (s[4] + s[5])) + ((s[8] + s[9]) + (s[12] + s[13]));
+          const float f0 = ((s[16] + s[17]) + (s[20] + s[21])) + ((s[24] + s[25]) + (s[28] + s[29]));
+          const float e1 = ((s[2] + s[3]) + (s[6] + s[7])) + ((s[10] + s[11]) + (s[14] + s[15]));
+          const float f1 = ((s[18] + s[19]) + (s[22] + s[23])) + ((s[26] + s[27]) + (s[30] + s[31]));
+          l0 = l0 * a0 + (e0 + f0);
+          l1 = l1 * a1 + (e1 + f1);
         }
         if (j > a) {  // O^T of the previous page is complete: P and O^T may be touched
           wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
@@ -379,7 +487,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           tc_fence_after();
         }
         if (bar_red_or(2, kSoftmaxThreads, need)) {
-          if (head_thread) misc->alpha[h] = need ? alpha : 1.f;
+          if (quad == 0) {
+            misc->alpha[hr0] = a0;
+            misc->alpha[hr1] = a1;
+          }
           named_bar_sync(2, kSoftmaxThreads);
           if (!dead) {
 #pragma unroll 1
@@ -406,16 +517,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               *reinterpret_cast<uint4*>(kv + cb * kBlockBytes + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
             }
           }
-          if (head_thread) {
+          // P^T tile (K-major, 128-byte swizzle): 4-byte pieces, the quad fills each 16-byte chunk
+          uint8_t* pt = smem + kOffP + 4 * quad;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint4 w;
-              w.x = pack_bf16x2(s[8 * c + 0], s[8 * c + 1]);
-              w.y = pack_bf16x2(s[8 * c + 2], s[8 * c + 3]);
-              w.z = pack_bf16x2(s[8 * c + 4], s[8 * c + 5]);
-              w.w = pack_bf16x2(s[8 * c + 6], s[8 * c + 7]);
-              *reinterpret_cast<uint4*>(smem + kOffP + sw128((uint32_t)h, (uint32_t)c)) = w;
-            }
+          for (int k = 0; k < 8; ++k) {
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr0, (uint32_t)k)) = pack_bf16x2(s[4 * k + 0], s[4 * k + 1]);
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr1, (uint32_t)k)) = pack_bf16x2(s[4 * k + 2], s[4 * k + 3]);
           }
         }
         fence_proxy_async_smem();
@@ -430,9 +537,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
       od_ph ^= 1u;
       tc_fence_after();
-      if (head_thread) {
-        misc->inv_l[h] = (lsum > 0.f && have_o) ? 1.f / lsum : 0.f;
-        misc->lse2[h] = (lsum > 0.f && have_o) ? m_used + __log2f(lsum) : -INFINITY;
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if (quad == 0) {
+        misc->inv_l[hr0] = (l0 > 0.f && have_o) ? 1.f / l0 : 0.f;
+        misc->lse2[hr0] = (l0 > 0.f && have_o) ? m0 + __log2f(l0) : -INFINITY;
+        misc->inv_l[hr1] = (l1 > 0.f && have_o) ? 1.f / l1 : 0.f;
+        misc->lse2[hr1] = (l1 > 0.f && have_o) ? m1 + __log2f(l1) : -INFINITY;
       }
       named_bar_sync(2, kSoftmaxThreads);
       const bool complete = (c0 == c1);
@@ -547,6 +660,7 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
     p.LSE[si] = set.LSE[si];
     p.pool_pages[si] = set.pool_pages[si];
     p.shard_of_si[si] = set.shard[si];
+    p.pool[si] = static_cast<const uint8_t*>(set.pool[si]);
     if (set.pool_pages[si] > 0) {
       const uint64_t rows = (uint64_t)set.pool_pages[si] * kMlaBs;
       if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32

@@ -16,7 +16,8 @@
 //    a segment cut by a range boundary are merged by the last CTA to arrive.
 //  * Warp 0 (one thread): TMA producer.  Per segment the query tile (64 x 576
 //    bf16, 72 KB) and per page the latent tile (64 tokens x 576, 72 KB), both
-//    as nine 64 x 64 boxes with 128-byte swizzle, into a 2-stage ring.
+//    as nine 64 x 64 boxes with 128-byte swizzle, into a 2-stage ring (two
+//    72 KB stages and the 72 KB query tile fill the shared memory).
 //  * Warp 1: TMEM allocator and the single MMA-issuing thread.
 //      S  = Q K^T   : tcgen05.mma M=64 (heads) N=64 (tokens) K=576, into one of
 //                     two 64-column TMEM buffers (head h in lane h%16 + 32*(h/16)).
@@ -44,7 +45,7 @@ namespace dcp {
 
 namespace {
 
-constexpr int kMlaThreads = 192;
+constexpr int kMlaThreads = 320;                      // producer warp, MMA warp, 8 softmax warps
 constexpr int kMlaHeads = 64;
 constexpr int kMlaDqk = 576;
 constexpr int kMlaDv = 512;
@@ -55,14 +56,14 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKV = kTileBytes;               // two stages
 constexpr uint32_t kOffP = 3 * kTileBytes;            // P^T tile: 64 heads x 64 tokens bf16
 constexpr uint32_t kOffMisc = kOffP + kBlockBytes;
-constexpr uint32_t kMlaSmem = kOffMisc + 2048;
+constexpr uint32_t kMlaSmem = kOffMisc + 3072;  // 232,448 bytes: the sm_100 per-block maximum
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                         // O^T: 4 tiles x 64 columns
 constexpr uint32_t kColS = 256;                       // S: 2 buffers x 64 columns
 constexpr float kRescaleThreshold = 8.0f;             // log2 units
-constexpr int kPrefetchPages = 4;                     // L2 prefetch distance of the producer, in pages
 constexpr float kLn2 = 0.69314718055994530942f;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxWarps = 8;
 
 struct MlaMisc {
   uint64_t q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, o_free, mma_done;
@@ -71,16 +72,17 @@ struct MlaMisc {
   float alpha[kMlaHeads];
   float inv_l[kMlaHeads];
   float lse2[kMlaHeads];
+  float pmax[2][2][kMlaHeads];  // [page parity][token half][head]: page maxima exchanged between halves
+  float lpart[kMlaHeads];       // token-half 1's row sums at the epilogue
   int scratch[32];
 };
-static_assert(sizeof(MlaMisc) <= 2048, "misc block");
+static_assert(sizeof(MlaMisc) <= 3072, "misc block");
 
 }  // namespace
 
 struct MlaParams {
   CUtensorMap kvmap[kMaxShards];
   CUtensorMap qmap;
-  const uint8_t* pool[kMaxShards];
   const int32_t* table[kMaxShards];
   float* O[kMaxShards];
   float* LSE[kMaxShards];
@@ -148,11 +150,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       mbar_init(&misc->kv_full[i], 1);
       mbar_init(&misc->kv_empty[i], 1);
       mbar_init(&misc->s_full[i], 1);
-      mbar_init(&misc->s_empty[i], 4);
+      mbar_init(&misc->s_empty[i], kSoftmaxWarps);
     }
-    mbar_init(&misc->p_full, 4);
+    mbar_init(&misc->p_full, kSoftmaxWarps);
     mbar_init(&misc->o_done, 1);
-    mbar_init(&misc->o_free, 4);
+    mbar_init(&misc->o_free, kSoftmaxWarps);
     mbar_init(&misc->mma_done, 1);
     fence_barrier_init();
   }
@@ -181,36 +183,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       uint32_t st = 0, kv_ph = 0, q_ph = 0;
       long issued = 0;
       bool dead = false, q_issued = false;
-      // A second cursor walks the same page sequence kPrefetchPages ahead and pulls
-      // those pages into L2, so the HBM stream does not wait for a free stage.
-      int pf_sid = plan.sid0, pf_pre = plan.pre0, pf_j = 0, pf_e = 0, pf_si = 0, pf_b = 0;
-      bool pf_live = true;
-      long pf_count = 0;
-      auto pf_advance = [&]() {  // next page of the CTA's walk into (pf_si, pf_b, pf_j), false at the end
-        while (pf_live) {
-          if (pf_j < pf_e) return true;
-          if (pf_sid >= S) { pf_live = false; break; }
-          const int si2 = pf_sid / B, b2 = pf_sid - si2 * B;
-          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2]);
-          if (seg_first_cta(pf_pre, n2, T, P) > cta) { pf_live = false; break; }
-          pf_si = si2;
-          pf_b = b2;
-          pf_j = max(pf_pre, lo) - pf_pre;
-          pf_e = n2 > 0 ? min(pf_pre + n2, hi) - pf_pre : 0;
-          pf_pre += n2;
-          ++pf_sid;
-        }
-        return false;
-      };
-      auto pf_until = [&](long target) {  // prefetch pages with index < target
-        while (pf_count < target && pf_advance()) {
-          const int page = p.table[pf_si][(size_t)pf_b * p.mlb + pf_j];
-          if (page >= 0 && page < p.pool_pages[pf_si])
-            prefetch_l2_bulk(p.pool[pf_si] + (size_t)page * kTileBytes, kTileBytes);
-          ++pf_j;
-          ++pf_count;
-        }
-      };
       int pre = plan.pre0;
       for (int sid = plan.sid0; sid < S; ++sid) {
         const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
@@ -230,7 +202,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           int page;
           const bool ok = page_ok(p, si, b, j, &page);
           if (!ok) atomicOr(p.status, kDevBadPage);
-          pf_until(issued + 1 + kPrefetchPages);
           wait_or_die(&misc->kv_empty[st], kv_ph ^ 1u, dead, p.status);
           if (dead) break;
           if (ok) {
@@ -381,11 +352,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 2-5)
-    // Warp q (= warp % 4) owns head rows 16q..16q+15 of S (TMEM lanes 32q..32q+15);
-    // with the 16x256b load all 32 lanes share them: thread t holds heads
-    // hr0 = 16q + t/4 and hr1 = hr0 + 8, tokens 8k + 2*(t%4) + {0,1}, k = 0..7.
+    // Warps 2-9: warp w reads TMEM sub-partition q = w % 4, which holds head rows
+    // 16q..16q+15 of S (lanes 32q..32q+15), and token half hf = (w - 2) / 4 of
+    // the page.  With the 16x256b load thread t holds heads hr0 = 16q + t/4 and
+    // hr1 = hr0 + 8, tokens 32*hf + 8k + 2*(t%4) + {0,1}, k = 0..3; the two
+    // halves exchange their page maxima through shared memory.
     const int q4 = warp & 3;
-    const int ts = tid - 64;                       // 0..127
+    const int hf = (warp - 2) >> 2;
+    const int ts = tid - 64;                       // 0..255
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const int quad = lane & 3;
     const int hr0 = 16 * q4 + (lane >> 2), hr1 = hr0 + 8;
@@ -422,38 +396,44 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         const uint32_t sb = gpage & 1u;
         wait_or_die_warp(&misc->s_full[sb], (gpage >> 1) & 1u, dead, p.status);
         tc_fence_after();
-        float s[32];
+        float s[16];
         if (ok && !dead) {
-          tmem_ld16x256b_x8(tbase + lane_off + kColS + sb * 64, s);
+          tmem_ld16x256b_x4(tbase + lane_off + kColS + sb * 64 + 32 * hf, s);
           tmem_ld_wait();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&misc->s_empty[sb]);
         bool need = false;
-        float a0 = 1.f, a1 = 1.f;
+        float a0 = 1.f, a1 = 1.f, pm0 = -INFINITY, pm1 = -INFINITY;
         if (ok && !dead) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < 4; ++k)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int tok = 8 * k + 2 * quad + (i & 1);
+              const int tok = 32 * hf + 8 * k + 2 * quad + (i & 1);
               s[4 * k + i] = tok < valid ? s[4 * k + i] * p.scale_log2 : -INFINITY;
             }
-          float x0 = fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5]));
-          float x1 = fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7]));
-          float y0 = fmaxf(fmaxf(s[8], s[9]), fmaxf(s[12], s[13]));
-          float y1 = fmaxf(fmaxf(s[10], s[11]), fmaxf(s[14], s[15]));
-          float z0 = fmaxf(fmaxf(s[16], s[17]), fmaxf(s[20], s[21]));
-          float z1 = fmaxf(fmaxf(s[18], s[19]), fmaxf(s[22], s[23]));
-          float w0 = fmaxf(fmaxf(s[24], s[25]), fmaxf(s[28], s[29]));
-          float w1 = fmaxf(fmaxf(s[26], s[27]), fmaxf(s[30], s[31]));
-          float pm0 = fmaxf(fmaxf(x0, y0), fmaxf(z0, w0));
-          float pm1 = fmaxf(fmaxf(x1, y1), fmaxf(z1, w1));
+          pm0 = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5])), fmaxf(fmaxf(s[8], s[9]), fmaxf(s[12], s[13])));
+          pm1 = fmaxf(fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7])), fmaxf(fmaxf(s[10], s[11]), fmaxf(s[14], s[15])));
           pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 1));
           pm0 = fmaxf(pm0, __shfl_xor_sync(0xffffffffu, pm0, 2));
           pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 1));
           pm1 = fmaxf(pm1, __shfl_xor_sync(0xffffffffu, pm1, 2));
+        }
+        {  // page maximum over both token halves (the partner warp holds the other half);
+           // the exchange runs on every page so both partners meet the barrier
+          float* xm = misc->pmax[gpage & 1][hf];
+          if (quad == 0) {
+            xm[hr0] = pm0;
+            xm[hr1] = pm1;
+          }
+          named_bar_sync(3 + q4, 64);
+          const float* om = misc->pmax[gpage & 1][hf ^ 1];
+          pm0 = fmaxf(pm0, om[hr0]);
+          pm1 = fmaxf(pm1, om[hr1]);
+        }
+        if (ok && !dead) {
           // integral reference maximum, raised only past the threshold (exact power-of-two rescale)
           if (m0 == -INFINITY || pm0 > m0 + kRescaleThreshold) {
             const float mn = ceilf(pm0);
@@ -468,18 +448,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             need = need || have_o;
           }
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 4; ++k) {
             s[4 * k + 0] = ex2_approx(s[4 * k + 0] - m0);
             s[4 * k + 1] = ex2_approx(s[4 * k + 1] - m0);
             s[4 * k + 2] = ex2_approx(s[4 * k + 2] - m1);
             s[4 * k + 3] = ex2_approx(s[4 * k + 3] - m1);
           }
-          const float e0 = ((s[0] + s[1]) + (s[4] + s[5])) + ((s[8] + s[9]) + (s[12] + s[13]));
-          const float f0 = ((s[16] + s[17]) + (s[20] + s[21])) + ((s[24] + s[25]) + (s[28] + s[29]));
-          const float e1 = ((s[2] + s[3]) + (s[6] + s[7])) + ((s[10] + s[11]) + (s[14] + s[15]));
-          const float f1 = ((s[18] + s[19]) + (s[22] + s[23])) + ((s[26] + s[27]) + (s[30] + s[31]));
-          l0 = l0 * a0 + (e0 + f0);
-          l1 = l1 * a1 + (e1 + f1);
+          l0 = l0 * a0 + (((s[0] + s[1]) + (s[4] + s[5])) + ((s[8] + s[9]) + (s[12] + s[13])));
+          l1 = l1 * a1 + (((s[2] + s[3]) + (s[6] + s[7])) + ((s[10] + s[11]) + (s[14] + s[15])));
         }
         if (j > a) {  // O^T of the previous page is complete: P and O^T may be touched
           wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
@@ -487,14 +463,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           tc_fence_after();
         }
         if (bar_red_or(2, kSoftmaxThreads, need)) {
-          if (quad == 0) {
+          if (quad == 0 && hf == 0) {
             misc->alpha[hr0] = a0;
             misc->alpha[hr1] = a1;
           }
           named_bar_sync(2, kSoftmaxThreads);
           if (!dead) {
 #pragma unroll 1
-            for (int mt = 0; mt < 4; ++mt)
+            for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
 #pragma unroll 1
               for (int c = 0; c < 64; c += 32) {
                 float v[32];
@@ -520,9 +496,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           // P^T tile (K-major, 128-byte swizzle): 4-byte pieces, the quad fills each 16-byte chunk
           uint8_t* pt = smem + kOffP + 4 * quad;
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr0, (uint32_t)k)) = pack_bf16x2(s[4 * k + 0], s[4 * k + 1]);
-            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr1, (uint32_t)k)) = pack_bf16x2(s[4 * k + 2], s[4 * k + 3]);
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t ch = (uint32_t)(4 * hf + k);
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr0, ch)) = pack_bf16x2(s[4 * k + 0], s[4 * k + 1]);
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr1, ch)) = pack_bf16x2(s[4 * k + 2], s[4 * k + 3]);
           }
         }
         fence_proxy_async_smem();
@@ -541,7 +518,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-      if (quad == 0) {
+      if (quad == 0 && hf == 1) {
+        misc->lpart[hr0] = l0;
+        misc->lpart[hr1] = l1;
+      }
+      named_bar_sync(2, kSoftmaxThreads);
+      if (quad == 0 && hf == 0) {
+        l0 += misc->lpart[hr0];
+        l1 += misc->lpart[hr1];
         misc->inv_l[hr0] = (l0 > 0.f && have_o) ? 1.f / l0 : 0.f;
         misc->lse2[hr0] = (l0 > 0.f && have_o) ? m0 + __log2f(l0) : -INFINITY;
         misc->inv_l[hr1] = (l1 > 0.f && have_o) ? 1.f / l1 : 0.f;
@@ -553,7 +537,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       float* dstO = complete ? Oout : p.slots + (size_t)slot * p.slot_floats;
       float* dstL = complete ? Lout : p.slots + (size_t)slot * p.slot_floats + kMlaHeads * kMlaDv;
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt)
+      for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
 #pragma unroll 1
         for (int c = 0; c < 64; c += 32) {
           float v[32];
@@ -580,8 +564,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         named_bar_sync(2, kSoftmaxThreads);
         if (misc->bcast) {
           __threadfence();
-          const int w4 = ts >> 5;
-          for (int r = w4; r < kMlaHeads; r += 4) {
+          const int w8 = ts >> 5;
+          for (int r = w8; r < kMlaHeads; r += kSoftmaxWarps) {
             float mx = -INFINITY;
             for (int c = c0; c <= c1; ++c) {
               const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
@@ -660,7 +644,6 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
     p.LSE[si] = set.LSE[si];
     p.pool_pages[si] = set.pool_pages[si];
     p.shard_of_si[si] = set.shard[si];
-    p.pool[si] = static_cast<const uint8_t*>(set.pool[si]);
     if (set.pool_pages[si] > 0) {
       const uint64_t rows = (uint64_t)set.pool_pages[si] * kMlaBs;
       if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32

@@ -93,3 +93,92 @@ class ShardedPagedCache:
         d = self.desc
         per = 2 * d.num_kv_heads * d.head_dim_qk * 2 if d.layout == dcp.DCP_LAYOUT_GQA else d.head_dim_qk * 2
         return int(sum(self.seq_lens)) * per
+
+
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
+class HostStepPipeline:
+    """Decode steps fed from, and returned to, pinned host memory.
+
+    Per step there is one host-to-device copy of the step's packed inputs (the
+    query, the sequence lengths and the D block tables) and one device-to-host
+    copy of its packed results (O and LSE).  Two buffer sets alternate between
+    steps and three streams (upload, compute, download) are ordered with
+    events, so step i's inputs upload while step i-1 computes and step i-1's
+    results download while step i computes.  The compute itself is
+    ``dcp_decode_partial_all`` + ``dcp_lse_merge`` on the cache's pools.
+    """
+
+    def __init__(self, cache: ShardedPagedCache):
+        self.cache = c = cache
+        d = c.desc
+        self.q_elems = c.batch * d.num_q_heads * d.head_dim_qk
+        self.q_off, self.sl_off = 0, _align(self.q_elems * 2)
+        self.tab_off = self.sl_off + _align(c.batch * 4)
+        self.tab_elems = c.batch * c.max_local_blocks
+        self.in_bytes = self.tab_off + c.D * self.tab_elems * 4
+        self.o_elems = c.batch * d.num_q_heads * d.head_dim_v
+        self.lse_off = self.o_elems * 4
+        self.out_bytes = self.lse_off + c.batch * d.num_q_heads * 4
+        dev = c.device
+        self.dev_in = [torch.empty(self.in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.dev_out = [torch.empty(self.out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(dev) for _ in range(3))
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_comp = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+
+    # ------------------------------------------------------------------ host buffers
+    def pack_inputs(self, q_bits, seq_lens, tables_host) -> torch.Tensor:
+        """Pinned host buffer holding one step's inputs in the device layout."""
+        buf = torch.zeros(self.in_bytes, dtype=torch.uint8).pin_memory()
+        a = buf.numpy()
+        a[self.q_off:self.q_off + self.q_elems * 2] = np.ascontiguousarray(q_bits).view(np.uint8).ravel()
+        a[self.sl_off:self.sl_off + self.cache.batch * 4] = np.ascontiguousarray(seq_lens, np.int32).view(np.uint8)
+        a[self.tab_off:] = np.ascontiguousarray(tables_host, np.int32).view(np.uint8).ravel()
+        return buf
+
+    def host_output(self) -> torch.Tensor:
+        return torch.empty(self.out_bytes, dtype=torch.uint8).pin_memory()
+
+    def unpack_output(self, buf: torch.Tensor):
+        d = self.cache.desc
+        O = buf[:self.lse_off].view(torch.float32).view(self.cache.batch, d.num_q_heads, d.head_dim_v)
+        L = buf[self.lse_off:].view(torch.float32).view(self.cache.batch, d.num_q_heads)
+        return O, L
+
+    # ------------------------------------------------------------------ one step
+    def step(self, i: int, host_in: torch.Tensor, host_out: torch.Tensor) -> None:
+        c, k = self.cache, i & 1
+        din, dout = self.dev_in[k], self.dev_out[k]
+        with torch.cuda.stream(self.s_in):
+            if self.used[k]:
+                self.s_in.wait_event(self.ev_comp[k])      # slot k's inputs are no longer read
+            din.copy_(host_in, non_blocking=True)
+            self.ev_in[k].record(self.s_in)
+        q = din[self.q_off:self.q_off + self.q_elems * 2]
+        sl = din[self.sl_off:self.sl_off + c.batch * 4]
+        tabs = [din[self.tab_off + s * self.tab_elems * 4:self.tab_off + (s + 1) * self.tab_elems * 4]
+                for s in range(c.D)]
+        o_dev = dout[:self.lse_off]
+        l_dev = dout[self.lse_off:]
+        self.s_comp.wait_event(self.ev_in[k])
+        if self.used[k]:
+            self.s_comp.wait_event(self.ev_out[k])         # slot k's results have been read back
+        dcp.dcp_decode_partial_all(c.desc, q, c.pools, c.pool_pages, tabs, sl, c.D, list(c.O_parts),
+                                   list(c.LSE_parts), c.workspace, stream=self.s_comp)
+        dcp.dcp_lse_merge(list(c.O_parts), list(c.LSE_parts), c.D, c.batch * c.desc.num_q_heads,
+                          c.desc.head_dim_v, o_dev, l_dev, stream=self.s_comp)
+        self.ev_comp[k].record(self.s_comp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_comp[k])
+            host_out.copy_(dout, non_blocking=True)
+            self.ev_out[k].record(self.s_out)
+        self.used[k] = True
+
+    def synchronize(self) -> None:
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.synchronize()

@@ -66,7 +66,10 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
 
 struct MlaMisc {
-  uint64_t q_full, q_empty, kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full, o_done, o_free, mma_done;
+  // kv_empty[st][g]: the groups of a stage that become free at different times --
+  // g = 0 the rope box (read by QK^T only), g = 1 value boxes 0-3 (PV tiles 0-1),
+  // g = 2 value boxes 4-7 (PV tiles 2-3) -- so the next page streams in early.
+  uint64_t q_full, q_empty, kv_full[2], kv_empty[2][3], s_full[2], s_empty[2], p_full, o_done, o_free, mma_done;
   uint32_t tmem_base;
   int bcast;
   float alpha[kMlaHeads];
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     mbar_init(&misc->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&misc->kv_full[i], 1);
-      mbar_init(&misc->kv_empty[i], 1);
+      for (int g = 0; g < 3; ++g) mbar_init(&misc->kv_empty[i][g], 1);
       mbar_init(&misc->s_full[i], 1);
       mbar_init(&misc->s_empty[i], kSoftmaxWarps);
     }
@@ -202,16 +205,24 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           int page;
           const bool ok = page_ok(p, si, b, j, &page);
           if (!ok) atomicOr(p.status, kDevBadPage);
-          wait_or_die(&misc->kv_empty[st], kv_ph ^ 1u, dead, p.status);
-          if (dead) break;
-          if (ok) {
-            mbar_arrive_expect_tx(&misc->kv_full[st], kTileBytes);
-            uint8_t* dst = smem + kOffKV + st * kTileBytes;
-            for (int cb = 0; cb < 9; ++cb)
-              tma_load_2d(dst + cb * kBlockBytes, &p.kvmap[si], cb * 64, page * kMlaBs, &misc->kv_full[st]);
-          } else {
-            mbar_arrive(&misc->kv_full[st]);
+          uint8_t* dst = smem + kOffKV + st * kTileBytes;
+          // box groups in the order they are freed: rope box, value boxes 0-3, value boxes 4-7
+          for (int g = 0; g < 3 && !dead; ++g) {
+            wait_or_die(&misc->kv_empty[st][g], kv_ph ^ 1u, dead, p.status);
+            if (dead) break;
+            if (ok) {
+              if (g == 0) {
+                mbar_arrive_expect_tx(&misc->kv_full[st], kTileBytes);
+                tma_load_2d(dst + 8 * kBlockBytes, &p.kvmap[si], 8 * 64, page * kMlaBs, &misc->kv_full[st]);
+              } else {
+                for (int cb = 4 * (g - 1); cb < 4 * g; ++cb)
+                  tma_load_2d(dst + cb * kBlockBytes, &p.kvmap[si], cb * 64, page * kMlaBs, &misc->kv_full[st]);
+              }
+            } else if (g == 2) {
+              mbar_arrive(&misc->kv_full[st]);
+            }
           }
+          if (dead) break;
           ++issued;
           if (++st == 2) {
             st = 0;
@@ -296,15 +307,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             const uint64_t ad = sw128_desc(smem_u32(smem + kOffKV + ost * kTileBytes), kBlockBytes, 1024);
             const uint64_t bd = sw128_desc(pa, 16, 1024);
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
+            for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
                 umma_bf16(tbase + kColO + mt * 64, ad + (uint64_t)((2 * mt * kBlockBytes + ks * 2048) >> 4),
                           bd + (uint64_t)((ks * 32) >> 4), idO, (o_init || ks > 0) ? 1u : 0u);
+              if (mt == 1) umma_commit(&misc->kv_empty[ost][1]);  // value boxes 0-3 are free
+            }
             o_init = true;
+          } else {
+            umma_commit(&misc->kv_empty[ost][1]);
           }
+          umma_commit(&misc->kv_empty[ost][2]);  // value boxes 4-7 are free
           umma_commit(&misc->o_done);
-          umma_commit(&misc->kv_empty[ost]);
           ++jo;
           progressed = true;
         }
@@ -328,6 +343,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               }
             }
             umma_commit(&misc->s_full[st]);
+            umma_commit(&misc->kv_empty[st][0]);           // the rope box is read by QK^T only
             if (r.seg_last) umma_commit(&misc->q_empty);  // Q is free once these S products are done
             ++js;
             progressed = true;

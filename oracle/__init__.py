@@ -50,6 +50,8 @@ def _load():
             lib.oracle_token_local_block.argtypes = [C.c_int64, C.c_int, C.c_int]
             lib.oracle_block_tables.restype = C.c_int
             lib.oracle_block_tables.argtypes = [p, C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_int, p, p, p]
+            lib.oracle_grow_tables.restype = C.c_int
+            lib.oracle_grow_tables.argtypes = [p, p, C.c_int, C.c_int, C.c_int, C.c_int, p, p, p, p]
             lib.oracle_place_request.restype = None
             lib.oracle_place_request.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                                  C.c_int, p, C.c_int64, p, p]
@@ -99,6 +101,18 @@ def block_tables(seq_lens: Sequence[int], block_size: int, D: int, perm_seed: in
     if rc != 0:
         raise ValueError(f"oracle_block_tables failed ({rc})")
     return tables, local_len, num_pages
+
+
+def grow_tables(old_lens: Sequence[int], new_lens: Sequence[int], block_size: int, D: int, tables: np.ndarray,
+                local_len: np.ndarray, next_page: np.ndarray, pool_pages: Sequence[int]) -> int:
+    """Grow ``tables[D][B][mlb]`` / ``local_len[D][B]`` / ``next_page[D]`` in place; returns the C status."""
+    o = np.ascontiguousarray(old_lens, dtype=np.int32)
+    n = np.ascontiguousarray(new_lens, dtype=np.int32)
+    pp = np.ascontiguousarray(pool_pages, dtype=np.int32)
+    for a in (tables, local_len, next_page):
+        assert a.dtype == np.int32 and a.flags.c_contiguous
+    return _load().oracle_grow_tables(_ptr(o), _ptr(n), o.shape[0], block_size, D, tables.shape[2], _ptr(tables),
+                                      _ptr(local_len), _ptr(next_page), _ptr(pp))
 
 
 def place(layout: int, Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray,

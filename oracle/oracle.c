@@ -136,6 +136,40 @@ int oracle_block_tables(const int32_t *seq_lens, int B, int block_size, int D, u
 }
 
 /*
+ * Incremental growth of the shard tables when requests gain tokens
+ * ([P3] §6.2: when a sequence grows only its newly added blocks are remapped;
+ * existing entries keep their pages).  Walking the new tokens
+ * t in [old_len[b], new_len[b]) of every request in order, a (shard, local
+ * block) seen for the first time takes the next free page of its shard,
+ * next_page[s]++; local_len[s][b] counts the tokens added to shard s.
+ * Returns 0, -1 on bad arguments (new < old, negative lengths), -2 when a
+ * local block index reaches max_local_blocks, -3 when a shard runs out of
+ * pages (next_page[s] == pool_pages[s]).  Tables of a failed call are partly
+ * updated.
+ */
+int oracle_grow_tables(const int32_t *old_lens, const int32_t *new_lens, int B, int block_size, int D,
+                       int max_local_blocks, int32_t *tables, int32_t *local_len, int32_t *next_page,
+                       const int32_t *pool_pages) {
+    if (B < 0 || block_size <= 0 || D <= 0 || max_local_blocks < 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (old_lens[b] < 0 || new_lens[b] < old_lens[b]) return -1;
+    for (int b = 0; b < B; ++b) {
+        for (int64_t t = old_lens[b]; t < new_lens[b]; ++t) {
+            int s = oracle_token_shard(t, block_size, D);
+            int64_t j = oracle_token_local_block(t, block_size, D);
+            if (j >= max_local_blocks) return -2;
+            int32_t *entry = &tables[((int64_t)s * B + b) * max_local_blocks + j];
+            if (*entry < 0) {
+                if (next_page[s] >= pool_pages[s]) return -3;
+                *entry = next_page[s]++;
+            }
+            local_len[(int64_t)s * B + b] += 1;
+        }
+    }
+    return 0;
+}
+
+/*
  * Reference placement of one request's unsharded KV rows into the shard
  * pools (the cache write that precedes decoding).  Token t of request b goes
  * to pool shard(t), page table[shard][b][local block], slot t mod bs.

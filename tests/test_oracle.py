@@ -315,3 +315,51 @@ def test_workload_recipes():
     lg = synth.workload("mla_long").seq_lens
     assert len(lg) == 4 and min(lg) >= 204800 and max(lg) <= 262144
     assert synth.workload("gqa_tiny").seq_lens == [100, 257]
+
+
+# ---------------------------------------------------------------------------
+# incremental growth of the tables (new blocks only)
+# ---------------------------------------------------------------------------
+def test_grow_from_empty_equals_full_build():
+    seq_lens = [100, 257, 0, 64, 1]
+    for D in (1, 2, 3, 4):
+        t_full, l_full, n_full = oracle.block_tables(seq_lens, 16, D)
+        t = np.full(t_full.shape, -1, np.int32)
+        l = np.zeros(l_full.shape, np.int32)
+        nxt = np.zeros(D, np.int32)
+        assert oracle.grow_tables([0] * 5, seq_lens, 16, D, t, l, nxt, [10 ** 6] * D) == 0
+        np.testing.assert_array_equal(t, t_full)
+        np.testing.assert_array_equal(l, l_full)
+        np.testing.assert_array_equal(nxt, n_full)
+
+
+def test_grow_keeps_existing_pages_and_covers_new_tokens():
+    rng = np.random.default_rng(8)
+    D, bs, B = 3, 16, 6
+    lens = rng.integers(0, 200, size=B).astype(np.int32)
+    t, l, n = oracle.block_tables(lens, bs, D, max_local_blocks=40)
+    nxt = n.copy()
+    for step in range(30):
+        new = lens + rng.integers(0, 40, size=B).astype(np.int32)
+        before = t.copy()
+        assert oracle.grow_tables(lens, new, bs, D, t, l, nxt, [10 ** 6] * D) == 0
+        assert ((before < 0) | (t == before)).all()            # old entries never move
+        for b in range(B):
+            assert int(l[:, b].sum()) == new[b]
+            for tok in range(0, int(new[b]), 7):
+                s = (tok // bs) % D
+                assert t[s, b, (tok // bs) // D] >= 0
+        used = [sorted(t[s][t[s] >= 0].tolist()) for s in range(D)]
+        for s in range(D):                                       # pages stay a bijection onto 0..next-1
+            assert used[s] == list(range(int(nxt[s])))
+        lens = new
+
+
+def test_grow_errors():
+    t = np.full((2, 1, 2), -1, np.int32)
+    l = np.zeros((2, 1), np.int32)
+    nxt = np.zeros(2, np.int32)
+    assert oracle.grow_tables([5], [3], 16, 2, t, l, nxt, [9, 9]) == -1        # shrinking
+    assert oracle.grow_tables([0], [16 * 5], 16, 2, t, l, nxt, [9, 9]) == -2   # local block 2 > capacity 2
+    t[:] = -1; l[:] = 0; nxt[:] = 0
+    assert oracle.grow_tables([0], [16 * 3], 16, 2, t, l, nxt, [1, 9]) == -3   # shard 0 has one page only

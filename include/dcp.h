@@ -161,6 +161,43 @@ DCP_API dcp_status dcp_place_kv(const dcp_attn_desc *desc, int32_t D, const void
                         const int32_t *pool_pages, int32_t *device_error, void *stream);
 
 /*
+ * Incremental table growth (host only) for requests that gained tokens since
+ * the tables were built.  [P3 §6.2: when a sequence grows only the newly
+ * added blocks are remapped; existing entries keep their pages.]  For each
+ * request b in order and each new logical block g in
+ * [ceil(old_seq_lens[b]/bs), ceil(new_seq_lens[b]/bs)) in order, shard s =
+ * g % D gives local block g / D the page next_page[s]++.  local_len (may be
+ * NULL) gains the tokens each shard received.  Growing from all-zero lengths
+ * with next_page = 0 reproduces dcp_build_block_table (perm_seed 0).
+ *   old_seq_lens, new_seq_lens  host int32[batch], new >= old.
+ *   tables      in/out, host int32[D][batch][max_local_blocks].
+ *   local_len   in/out, host int32[D][batch], or NULL.
+ *   next_page   in/out, host int32[D]: first free page of each shard pool.
+ *   pool_pages  host int32[D]: pages each pool holds.
+ * Errors: DCP_ERR_INVALID_ARG (nulls, a shrinking request, bad sizes);
+ * DCP_ERR_CAPACITY if a local block index reaches max_local_blocks or a pool
+ * runs out of pages.  On error nothing is modified.
+ */
+DCP_API dcp_status dcp_grow_block_table(const int32_t *old_seq_lens, const int32_t *new_seq_lens, int32_t batch,
+                                        int32_t block_size, int32_t D, int32_t max_local_blocks, int32_t *tables,
+                                        int32_t *local_len, int32_t *next_page, const int32_t *pool_pages);
+
+/*
+ * Cache write of new tokens (the decode step's append).  [P3 §3.2, §6.2]
+ * Request b's new rows are rows [cu_rows[b], cu_rows[b+1]) of kv_new and hold
+ * tokens first_pos[b], first_pos[b]+1, ...; each goes to shard
+ * (t / block_size) % D, page tables[shard][b][(t / block_size) / D], slot
+ * t % block_size (layouts as in dcp_place_kv).
+ *   kv_new      device bf16 rows ([2][Hkv][head_dim] GQA, [576] MLA).
+ *   cu_rows     device int64[batch+1];  first_pos  device int32[batch].
+ *   tables, kv_pools, pool_pages, device_error: as in dcp_place_kv (tables
+ *               already grown to cover the new tokens).
+ */
+DCP_API dcp_status dcp_append_kv(const dcp_attn_desc *desc, int32_t D, const void *kv_new, const int64_t *cu_rows,
+                                 const int32_t *first_pos, const int32_t *const *tables, void *const *kv_pools,
+                                 const int32_t *pool_pages, int32_t *device_error, void *stream);
+
+/*
  * Workspace bytes the decode calls need for `desc` and D shards on the
  * current device (split partials, arrival counters, a status word).  The
  * workspace must be zeroed once by dcp_workspace_init before its first use;

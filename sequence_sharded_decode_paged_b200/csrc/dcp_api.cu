@@ -230,7 +230,60 @@ dcp_status dcp_place_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_src
     if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
   }
   if ((reinterpret_cast<uintptr_t>(kv_src) & 15u) != 0) return DCP_ERR_INVALID_ARG;
-  return launch_place_kv(*desc, D, kv_src, cu_seqlens, seq_lens, tables, kv_pools, pool_pages, device_error,
+  return launch_place_kv(*desc, D, kv_src, cu_seqlens, nullptr, tables, kv_pools, pool_pages, device_error,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dcp_status dcp_grow_block_table(const int32_t* old_seq_lens, const int32_t* new_seq_lens, int32_t batch,
+                                int32_t block_size, int32_t D, int32_t max_local_blocks, int32_t* tables,
+                                int32_t* local_len, int32_t* next_page, const int32_t* pool_pages) {
+  if (old_seq_lens == nullptr || new_seq_lens == nullptr || tables == nullptr || next_page == nullptr ||
+      pool_pages == nullptr || batch < 0 || block_size <= 0 || D < 1 || D > kMaxShardsHost || max_local_blocks < 0)
+    return DCP_ERR_INVALID_ARG;
+  std::vector<int64_t> need(D, 0);
+  for (int b = 0; b < batch; ++b) {
+    if (old_seq_lens[b] < 0 || new_seq_lens[b] < old_seq_lens[b]) return DCP_ERR_INVALID_ARG;
+    const int64_t g0 = (old_seq_lens[b] + block_size - 1) / block_size;  // first block without a page
+    const int64_t g1 = ((int64_t)new_seq_lens[b] + block_size - 1) / block_size;
+    for (int64_t g = g0; g < g1; ++g) {
+      if (g / D >= max_local_blocks) return DCP_ERR_CAPACITY;
+      ++need[g % D];
+    }
+  }
+  for (int s = 0; s < D; ++s)
+    if (next_page[s] < 0 || (int64_t)next_page[s] + need[s] > pool_pages[s]) return DCP_ERR_CAPACITY;
+  // checks passed: apply (new blocks take their shard's next free page, requests in order)
+  for (int b = 0; b < batch; ++b) {
+    const int64_t old_len = old_seq_lens[b], new_len = new_seq_lens[b];
+    const int64_t g0 = (old_len + block_size - 1) / block_size;
+    const int64_t g1 = (new_len + block_size - 1) / block_size;
+    for (int64_t g = g0; g < g1; ++g)
+      tables[((size_t)(g % D) * batch + b) * max_local_blocks + g / D] = next_page[g % D]++;
+    if (local_len != nullptr)
+      for (int64_t g = old_len / block_size; g < g1; ++g) {
+        const int64_t lo = g * block_size > old_len ? g * block_size : old_len;
+        const int64_t hi = (g + 1) * block_size < new_len ? (g + 1) * block_size : new_len;
+        if (hi > lo) local_len[(size_t)(g % D) * batch + b] += (int32_t)(hi - lo);
+      }
+  }
+  return DCP_OK;
+}
+
+dcp_status dcp_append_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_new, const int64_t* cu_rows,
+                         const int32_t* first_pos, const int32_t* const* tables, void* const* kv_pools,
+                         const int32_t* pool_pages, int32_t* device_error, void* stream) {
+  if (desc == nullptr || kv_new == nullptr || cu_rows == nullptr || first_pos == nullptr || tables == nullptr ||
+      kv_pools == nullptr || pool_pages == nullptr)
+    return DCP_ERR_INVALID_ARG;
+  dcp_status why;
+  if (!desc_supported(*desc, D, &why)) return why;
+  for (int s = 0; s < D; ++s) {
+    if (tables[s] == nullptr || pool_pages[s] < 0 || (pool_pages[s] > 0 && kv_pools[s] == nullptr))
+      return DCP_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(kv_new) & 15u) != 0) return DCP_ERR_INVALID_ARG;
+  return launch_place_kv(*desc, D, kv_new, cu_rows, first_pos, tables, kv_pools, pool_pages, device_error,
                          static_cast<cudaStream_t>(stream));
 }
 

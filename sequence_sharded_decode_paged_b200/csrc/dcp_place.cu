@@ -7,6 +7,8 @@
 //
 // One warp per source row (token): the warp finds its request by binary
 // search over cu_seqlens, then copies the row with 16-byte loads and stores.
+// The same kernel appends new tokens (the decode step's cache write): the rows
+// of request b then start at token position token_begin[b] instead of 0.
 //   GQA: source row [2][Hkv][d] -> pool page [2][Hkv][bs][d], slot t % bs.
 //   MLA: source row [576]       -> pool page [bs][576],        slot t % bs.
 #include "dcp_device.cuh"
@@ -20,7 +22,7 @@ struct PlaceParams {
   int pool_pages[kMaxShards];
   const uint8_t* src;
   const int64_t* cu_seqlens;
-  const int32_t* seq_lens;
+  const int32_t* token_begin;  // position of each request's first source row (nullptr: 0)
   int32_t* err;
   int layout, B, Hkv, d, bs, D, mlb;
 };
@@ -39,7 +41,11 @@ __global__ void __launch_bounds__(256) place_kv_kernel(const __grid_constant__ P
       if (p.cu_seqlens[mid] <= r) lo = mid; else hi = mid - 1;
     }
     const int b = lo;
-    const long t = r - p.cu_seqlens[b];
+    const long t = r - p.cu_seqlens[b] + (p.token_begin != nullptr ? p.token_begin[b] : 0);
+    if (t < 0) {  // a negative start position names no slot
+      if (lane == 0 && p.err != nullptr) atomicOr(p.err, kDevBadPage);
+      continue;
+    }
     const long g = t / p.bs;
     const int s = (int)(g % p.D);
     const long j = g / p.D;
@@ -68,7 +74,7 @@ __global__ void __launch_bounds__(256) place_kv_kernel(const __grid_constant__ P
 }
 
 dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, const int64_t* cu_seqlens,
-                           const int32_t* seq_lens, const int32_t* const* tables, void* const* pools,
+                           const int32_t* token_begin, const int32_t* const* tables, void* const* pools,
                            const int32_t* pool_pages, int32_t* device_error, cudaStream_t st) {
   PlaceParams p;
   memset(&p, 0, sizeof(p));
@@ -79,7 +85,7 @@ dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, co
   }
   p.src = static_cast<const uint8_t*>(kv_src);
   p.cu_seqlens = cu_seqlens;
-  p.seq_lens = seq_lens;
+  p.token_begin = token_begin;
   p.err = device_error;
   p.layout = d.layout;
   p.B = d.batch;

@@ -25,7 +25,7 @@ DCP_LAYOUT_GQA, DCP_LAYOUT_MLA = 0, 1
 EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_build_block_table",
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
-            "dcp_validate_config", "dcp_decode_partial_all_noalloc"]
+            "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_grow_block_table", "dcp_append_kv"]
 
 
 class DcpError(RuntimeError):
@@ -61,6 +61,8 @@ def _load() -> C.CDLL:
         "dcp_read_device_error": (C.c_int, [p, p, p]),
         "dcp_validate_config": (C.c_int, [i32, i32, i32, i32]),
         "dcp_decode_partial_all_noalloc": (C.c_int, [p, p, p, p, p, p, i32, p, p, p]),
+        "dcp_grow_block_table": (C.c_int, [p, p, i32, i32, i32, i32, p, p, p, p]),
+        "dcp_append_kv": (C.c_int, [p, i32, p, p, p, p, p, p, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -138,6 +140,18 @@ def dcp_build_block_table(seq_lens: Sequence[int], block_size: int, D: int, perm
     return tables, local_len
 
 
+def dcp_grow_block_table(old_seq_lens, new_seq_lens, block_size: int, D: int, tables: np.ndarray,
+                         local_len: Optional[np.ndarray], next_page: np.ndarray, pool_pages) -> None:
+    """Grow ``tables`` (int32[D][B][mlb]), ``local_len`` and ``next_page`` (int32[D]) in place."""
+    o, n, pp = _i32(old_seq_lens), _i32(new_seq_lens), _i32(pool_pages)
+    for a in (tables, next_page) + ((local_len,) if local_len is not None else ()):
+        if a.dtype != np.int32 or not a.flags.c_contiguous:
+            raise TypeError("tables, local_len and next_page must be C-contiguous int32 arrays")
+    _check("dcp_grow_block_table", _lib.dcp_grow_block_table(
+        o.ctypes.data, n.ctypes.data, o.shape[0], block_size, D, tables.shape[2], tables.ctypes.data,
+        None if local_len is None else local_len.ctypes.data, next_page.ctypes.data, pp.ctypes.data))
+
+
 def dcp_kv_page_bytes(desc: dcp_attn_desc) -> int:
     return int(_lib.dcp_kv_page_bytes(C.byref(desc)))
 
@@ -158,6 +172,14 @@ def dcp_place_kv(desc: dcp_attn_desc, D: int, kv_src, cu_seqlens, seq_lens, tabl
     _check("dcp_place_kv", _lib.dcp_place_kv(
         C.byref(desc), D, _addr(kv_src), _addr(cu_seqlens), _addr(seq_lens), _ptr_array(tables),
         _ptr_array(kv_pools), pp.ctypes.data, _addr(device_error), _stream(stream)))
+
+
+def dcp_append_kv(desc: dcp_attn_desc, D: int, kv_new, cu_rows, first_pos, tables, kv_pools, pool_pages,
+                  device_error=None, stream=None) -> None:
+    pp = _i32(pool_pages)
+    _check("dcp_append_kv", _lib.dcp_append_kv(
+        C.byref(desc), D, _addr(kv_new), _addr(cu_rows), _addr(first_pos), _ptr_array(tables), _ptr_array(kv_pools),
+        pp.ctypes.data, _addr(device_error), _stream(stream)))
 
 
 def dcp_workspace_init(workspace, workspace_bytes: Optional[int] = None, stream=None) -> None:

@@ -105,3 +105,54 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == dcp.DCP_ERR_INVALID_ARG
     lib.dcp_lse_merge.restype = ctypes.c_int
     assert lib.dcp_lse_merge(null, null, 2, 4, 64, null, null, null) == dcp.DCP_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8])
+def test_grow_block_table_bit_exact_vs_oracle(D):
+    rng = np.random.default_rng(D + 40)
+    bs, B, mlb = 16, 7, 64
+    lens = rng.integers(0, 300, size=B).astype(np.int32)
+    t_lib = np.full((D, B, mlb), -1, np.int32)
+    l_lib = np.zeros((D, B), np.int32)
+    n_lib = np.zeros(D, np.int32)
+    t_or, l_or, n_or = t_lib.copy(), l_lib.copy(), n_lib.copy()
+    pool = [10 ** 6] * D
+    dcp.dcp_grow_block_table([0] * B, lens, bs, D, t_lib, l_lib, n_lib, pool)
+    assert oracle.grow_tables([0] * B, lens, bs, D, t_or, l_or, n_or, pool) == 0
+    for step in range(25):
+        new = lens + rng.integers(0, 50, size=B).astype(np.int32) * (rng.random(B) < 0.7)
+        dcp.dcp_grow_block_table(lens, new, bs, D, t_lib, l_lib, n_lib, pool)
+        assert oracle.grow_tables(lens, new, bs, D, t_or, l_or, n_or, pool) == 0
+        np.testing.assert_array_equal(t_lib, t_or)
+        np.testing.assert_array_equal(l_lib, l_or)
+        np.testing.assert_array_equal(n_lib, n_or)
+        lens = new
+
+
+def test_grow_from_empty_equals_build():
+    lens = [100, 257, 0, 64, 1, 3000]
+    for D in (1, 2, 4):
+        t_b, l_b = dcp.dcp_build_block_table(lens, 16, D)
+        t = np.full(t_b.shape, -1, np.int32)
+        l = np.zeros(l_b.shape, np.int32)
+        nxt = np.zeros(D, np.int32)
+        dcp.dcp_grow_block_table([0] * len(lens), lens, 16, D, t, l, nxt, [10 ** 6] * D)
+        np.testing.assert_array_equal(t, t_b)
+        np.testing.assert_array_equal(l, l_b)
+        assert list(nxt) == list(dcp.dcp_block_table_extent(lens, 16, D)[1])
+
+
+def test_grow_errors_leave_tables_untouched():
+    t = np.full((2, 1, 3), -1, np.int32)
+    l = np.zeros((2, 1), np.int32)
+    nxt = np.zeros(2, np.int32)
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_grow_block_table([5], [3], 16, 2, t, l, nxt, [9, 9])
+    assert e.value.status == dcp.DCP_ERR_INVALID_ARG
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_grow_block_table([0], [16 * 3], 16, 2, t, l, nxt, [1, 9])  # shard 0 needs 2 pages, has 1
+    assert e.value.status == dcp.DCP_ERR_CAPACITY
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_grow_block_table([0], [16 * 7], 16, 2, t, l, nxt, [9, 9])  # local block 3 >= 3
+    assert e.value.status == dcp.DCP_ERR_CAPACITY
+    assert (t == -1).all() and (l == 0).all() and (nxt == 0).all()

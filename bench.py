@@ -329,8 +329,26 @@ def run_ours(args, rank, world, local):
     h2d, d2h = pipe.in_bytes, pipe.out_bytes
     assert np.isfinite(pipe.unpack_output(host_out[0])[0].numpy()).all()
 
+    # cache write of one new token per request (the append that precedes each decode step),
+    # timed on its own; it rewrites each request's last slot, after which the cache is not reused
+    from sequence_sharded_decode_paged_b200 import dcp
+    row_elems = w.kv_bytes_per_token // 2
+    kv_row = torch.zeros((w.batch, row_elems), dtype=torch.int16, device=dev)
+    cu_rows = torch.arange(w.batch + 1, dtype=torch.int64, device=dev)
+    last_pos = (cache.seq_lens_dev - 1).clamp_min(0).contiguous()
+    for _ in range(3):
+        dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools, cache.pool_pages)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(20):
+        dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools, cache.pool_pages)
+    a1.record()
+    torch.cuda.synchronize()
+    append_ms = a0.elapsed_time(a1) / 20
+
     kv_b, dec_b, mrg_b = algorithmic_bytes(w, D)
     step_ms_max = reduce_max(step_ms, world, dev)
+    append_ms_max = reduce_max(append_ms, world, dev)
     part_ms_max = reduce_max(part_ms, world, dev)
     merge_ms_max = reduce_max(merge_ms, world, dev)
     e2e_ms_max = reduce_max(e2e_ms, world, dev)
@@ -381,6 +399,8 @@ def run_ours(args, rank, world, local):
         "decode_kernel_us": round(part_ms_max * 1e3, 2),
         "merge_kernel_us": round(merge_ms_max * 1e3, 2),
         "merge_gbs": round(mrg_b / merge_ms_max / 1e6, 1),
+        "append_kernel_us": round(append_ms_max * 1e3, 2),
+        "append_bytes_per_step": 2 * w.batch * w.kv_bytes_per_token,
         "context_tokens_per_s": round(world * w.total_tokens / step_ms_max * 1e3, 1),
         "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
         "tensor": tensor_figures(w, part_ms_max, peaks, peaks_kind),

@@ -189,6 +189,41 @@ def sharded(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, 
     return Of, Lf, Op, Lp
 
 
+# ---------------------------------------------------------------------------
+# multi-token decode (q_len query tokens per request, causal within the draft)
+# ---------------------------------------------------------------------------
+def visible_tokens(seq_len: int, q_len: int, j: int) -> int:
+    """Tokens that query token ``j`` of a ``q_len``-token draft sees: the draft tokens are the last
+    ``q_len`` of the ``seq_len`` cached ones, and token j sees itself and everything before it."""
+    return max(0, seq_len - (q_len - 1 - j))
+
+
+def attend_mtp(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
+               q_len: int, block_size: int = 1, D: int = 1, shard: int = -1,
+               heads: Optional[Tuple[int, int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention of the ``q_len`` query tokens of one request: ``q`` bf16 bits [q_len][Hq][d_qk] ->
+    (O[q_len][Hq][d_v], LSE[q_len][Hq]).  Token j is ``attend`` over the first
+    ``visible_tokens(len(src), q_len, j)`` source rows (restricted to ``shard`` as in ``attend``)."""
+    q = np.ascontiguousarray(q, dtype=np.uint16).reshape(q_len, Hq, d_qk)
+    L = src.shape[0]
+    O = np.empty((q_len, Hq, d_v))
+    LSE = np.empty((q_len, Hq))
+    for j in range(q_len):
+        O[j], LSE[j] = attend(layout, Hq, Hkv, d_qk, d_v, q[j], src[:visible_tokens(L, q_len, j)], scale,
+                              block_size, D, shard, heads)
+    return O, LSE
+
+
+def sharded_mtp(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
+                q_len: int, block_size: int, D: int):
+    """Per-shard multi-token partials and their merge: (O[q_len][Hq][d_v], LSE[q_len][Hq], O_parts[D], LSE_parts[D])."""
+    parts = [attend_mtp(layout, Hq, Hkv, d_qk, d_v, q, src, scale, q_len, block_size, D, s) for s in range(D)]
+    Op = np.stack([p[0] for p in parts])
+    Lp = np.stack([p[1] for p in parts])
+    O, LSE = merge(Op.reshape(D, q_len * Hq, d_v), Lp.reshape(D, q_len * Hq))
+    return O.reshape(q_len, Hq, d_v), LSE.reshape(q_len, Hq), Op, Lp
+
+
 def kv_bytes_per_token(num_kv_heads: int, head_dim: int, elem_bytes: int) -> int:
     return _load().oracle_kv_bytes_per_token(num_kv_heads, head_dim, elem_bytes)
 

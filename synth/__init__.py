@@ -28,7 +28,8 @@ Element indices (logical, unsharded tensors; the caller never sees shards):
 * GQA key  ``K[b][t][h][k]``: tensor ``T_K``, ``e = (t*Hkv + h)*d + k``.
 * GQA value``V[b][t][h][k]``: tensor ``T_V``, same ``e``.
 * MLA latent row ``C[b][t][k]`` (k < 576): tensor ``T_LATENT``, ``e = t*576 + k``.
-* query ``q[b][h][k]``: tensor ``T_Q``, ``e = h*d_qk + k``.
+* query ``q[b][h][k]``: tensor ``T_Q``, ``e = h*d_qk + k``; with ``q_len`` query tokens,
+  ``q[b][j][h][k]`` has ``e = (j*Hq + h)*d_qk + k`` (token 0 is the single-token query).
 
 The unsharded KV source layout consumed by the cache-placement call is
 ``[token][2][Hkv][d]`` for GQA and ``[token][d_qk]`` for MLA, with requests
@@ -162,6 +163,7 @@ class Workload:
     perm_seed: int = 0
     note: str = ""
     extra: dict = field(default_factory=dict)
+    q_len: int = 1  # query tokens per request (multi-token decode when > 1)
 
     @property
     def kv_bytes_per_token(self) -> int:
@@ -177,6 +179,12 @@ class Workload:
     def query(self, b: int) -> np.ndarray:
         n = self.num_q_heads * self.head_dim_qk
         return values_bf16(self.seed, T_Q, b, 0, n, self.q_amp).reshape(self.num_q_heads, self.head_dim_qk)
+
+    def queries(self, b: int) -> np.ndarray:
+        """All ``q_len`` query tokens of request ``b``: ``[q_len][Hq][d_qk]``; token 0 is ``query(b)``."""
+        n = self.q_len * self.num_q_heads * self.head_dim_qk
+        return values_bf16(self.seed, T_Q, b, 0, n, self.q_amp).reshape(self.q_len, self.num_q_heads,
+                                                                        self.head_dim_qk)
 
     def kv_source_head(self, b: int, h: int, n_tok: Optional[int] = None) -> np.ndarray:
         """GQA: request ``b``'s rows of KV head ``h`` only, as a one-head source ``[n][2][1][d]``
@@ -271,9 +279,10 @@ WORKLOADS = ["gqa_tiny", "gqa_70b", "mla_b32", "mla_long", "mla_mix"]
 
 def custom(layout: int, seq_lens, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
            block_size: int, seed: int, softmax_scale: Optional[float] = None, q_amp: float = 1.0,
-           kv_amp: float = 1.0, name: str = "custom") -> Workload:
+           kv_amp: float = 1.0, name: str = "custom", q_len: int = 1) -> Workload:
     """Ad-hoc workload for edge-case tests (same generator, any shape)."""
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(head_dim_qk if layout == GQA else 192)
     return Workload(name, layout, len(seq_lens), num_q_heads, num_kv_heads, head_dim_qk, head_dim_v,
-                    block_size, [1], list(int(s) for s in seq_lens), softmax_scale, seed, q_amp, kv_amp)
+                    block_size, [1], list(int(s) for s in seq_lens), softmax_scale, seed, q_amp, kv_amp,
+                    q_len=q_len)

@@ -59,9 +59,12 @@ def cu_seqlens(w: Workload, device) -> torch.Tensor:
 
 
 def query(w: Workload, device) -> torch.Tensor:
-    """q[B][Hq][d_qk] bf16 on the device."""
-    q = torch.empty((w.batch, w.num_q_heads, w.head_dim_qk), dtype=torch.bfloat16, device=device)
-    _fill(q, None, w.batch, 2, w.num_q_heads, w.head_dim_qk, w.seed, w.q_amp, w.batch * w.num_q_heads)
+    """q[B][Hq][d_qk] bf16 on the device; q[B][q_len][Hq][d_qk] when the workload has q_len > 1."""
+    rows = w.q_len * w.num_q_heads  # per request, in the order of Workload.queries
+    shape = (w.batch, w.num_q_heads, w.head_dim_qk) if w.q_len == 1 else \
+        (w.batch, w.q_len, w.num_q_heads, w.head_dim_qk)
+    q = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    _fill(q, None, w.batch, 2, rows, w.head_dim_qk, w.seed, w.q_amp, w.batch * rows)
     return q
 
 

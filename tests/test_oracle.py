@@ -363,3 +363,96 @@ def test_grow_errors():
     assert oracle.grow_tables([0], [16 * 5], 16, 2, t, l, nxt, [9, 9]) == -2   # local block 2 > capacity 2
     t[:] = -1; l[:] = 0; nxt[:] = 0
     assert oracle.grow_tables([0], [16 * 3], 16, 2, t, l, nxt, [1, 9]) == -3   # shard 0 has one page only
+
+
+# ---------------------------------------------------------------------------
+# multi-token decode (causal within the draft)
+# ---------------------------------------------------------------------------
+MTP_CASES = [(GQA, 8, 2, 64, 64), (MLA, 4, 1, 576, 512)]
+
+
+@pytest.mark.parametrize("case", MTP_CASES)
+def test_mtp_single_token_is_plain_decode(case):
+    layout, Hq, Hkv, dqk, dv = case
+    w = synth.custom(layout, [77], Hq, Hkv, dqk, dv, 16, seed=21, q_len=1)
+    O, L = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, w.queries(0), w.kv_source(0), w.softmax_scale, 1)
+    O1, L1 = oracle.attend(layout, Hq, Hkv, dqk, dv, w.query(0), w.kv_source(0), w.softmax_scale)
+    np.testing.assert_array_equal(O[0], O1)
+    np.testing.assert_array_equal(L[0], L1)
+
+
+@pytest.mark.parametrize("case", MTP_CASES)
+@pytest.mark.parametrize("q_len", [2, 3, 4])
+def test_mtp_causal_boundary_by_perturbation(case, q_len):
+    # Query token j must see exactly the first L - (q_len - 1 - j) tokens: replacing every
+    # token after them changes nothing, replacing the last visible one changes the result.
+    layout, Hq, Hkv, dqk, dv = case
+    L = 41
+    w = synth.custom(layout, [L], Hq, Hkv, dqk, dv, 16, seed=30 + q_len, q_len=q_len)
+    other = synth.custom(layout, [L], Hq, Hkv, dqk, dv, 16, seed=999, q_len=q_len).kv_source(0)
+    q, src = w.queries(0), w.kv_source(0)
+    O, LSE = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, q_len)
+    for j in range(q_len):
+        n = L - (q_len - 1 - j)
+        tail = src.copy()
+        tail[n:] = other[n:]
+        Ot, Lt = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, q, tail, w.softmax_scale, q_len)
+        np.testing.assert_array_equal(Ot[j], O[j])
+        np.testing.assert_array_equal(Lt[j], LSE[j])
+        last = src.copy()
+        last[n - 1] = other[n - 1]
+        Ol, Ll = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, q, last, w.softmax_scale, q_len)
+        assert np.abs(Ol[j] - O[j]).max() > 1e-6 and np.abs(Ll[j] - LSE[j]).max() > 1e-9
+
+
+@pytest.mark.parametrize("case", MTP_CASES)
+def test_mtp_matches_masked_torch_sdpa(case):
+    # Library reference: torch float64 SDPA with a boolean mask built from token counts
+    # (token j of the draft sits at position L - q_len + j and sees positions <= its own).
+    layout, Hq, Hkv, dqk, dv = case
+    q_len, L = 3, 29
+    w = synth.custom(layout, [L], Hq, Hkv, dqk, dv, 16, seed=44, q_len=q_len)
+    q, src = w.queries(0), w.kv_source(0)
+    O, LSE = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, q_len)
+    pos_q = torch.arange(L - q_len, L)
+    allowed = torch.arange(L)[None, :] <= pos_q[:, None]  # [q_len][L]
+    qd = torch.from_numpy(_f64(q)).permute(1, 0, 2)  # [Hq][q_len][d]
+    if layout == GQA:
+        kv = torch.from_numpy(_f64(src))
+        K = kv[:, 0].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+        V = kv[:, 1].permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0)
+    else:
+        c = torch.from_numpy(_f64(src))
+        K = c.unsqueeze(0).expand(Hq, -1, -1)
+        V = c[:, :dv].unsqueeze(0).expand(Hq, -1, -1)
+    Ot = torch.nn.functional.scaled_dot_product_attention(qd, K, V, attn_mask=allowed, scale=w.softmax_scale)
+    S = torch.einsum("hjd,hnd->hjn", qd, K) * w.softmax_scale
+    Lt = torch.logsumexp(S.masked_fill(~allowed, -math.inf), dim=2)
+    np.testing.assert_allclose(O, Ot.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE, Lt.permute(1, 0).numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("D", [2, 3, 4])
+def test_mtp_sharded_merge_equals_direct(D):
+    for layout, Hq, Hkv, dqk, dv in MTP_CASES:
+        for L in [3, 16, 17, 50]:  # draft straddling a block boundary, and L < q_len + block
+            w = synth.custom(layout, [L], Hq, Hkv, dqk, dv, 16, seed=L * D, q_len=4)
+            q, src = w.queries(0), w.kv_source(0)
+            O, LSE = oracle.attend_mtp(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, 4)
+            Om, Lm, _, _ = oracle.sharded_mtp(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, 4, 16, D)
+            np.testing.assert_allclose(Om, O, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(Lm, LSE, rtol=0, atol=1e-12)
+
+
+def test_mtp_short_sequence_sees_nothing():
+    # seq_len 2 with a 4-token draft: tokens 0 and 1 see no cached token at all.
+    w = synth.custom(GQA, [2], 4, 2, 64, 64, 16, seed=5, q_len=4)
+    O, LSE = oracle.attend_mtp(GQA, 4, 2, 64, 64, w.queries(0), w.kv_source(0), 0.125, 4)
+    assert (O[:2] == 0).all() and (LSE[:2] == -np.inf).all()
+    assert np.isfinite(LSE[2:]).all()
+    np.testing.assert_array_equal(O[3], oracle.attend(GQA, 4, 2, 64, 64, w.queries(0)[3], w.kv_source(0), 0.125)[0])
+
+
+def test_queries_extend_the_single_token_query():
+    w = synth.custom(MLA, [5], 64, 1, 576, 512, 64, seed=8, q_len=3)
+    np.testing.assert_array_equal(w.queries(0)[0], w.query(0))

@@ -42,6 +42,8 @@
  *       MLA: Hq == 64, Hkv == 1, head_dim_qk == 576, head_dim_v == 512,
  *            block_size == 64.
  *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.
+ *       Multi-token decode: 1 <= q_len <= 4 query tokens per request
+ *       (GQA and MLA).
  */
 #ifndef DCP_H
 #define DCP_H
@@ -76,7 +78,7 @@ typedef enum dcp_layout {
 /*
  * Problem description shared by the decode calls.
  *   layout           dcp_layout.
- *   batch            B, number of requests (one decode token each).
+ *   batch            B, number of requests (q_len decode tokens each).
  *   num_q_heads      Hq.
  *   num_kv_heads     Hkv (GQA); must be 1 for MLA.
  *   head_dim_qk      query/key width (GQA head_dim; MLA 576 = 512 latent + 64 rope).
@@ -84,6 +86,14 @@ typedef enum dcp_layout {
  *   block_size       tokens per KV page.
  *   max_local_blocks row length of each shard's block table (>= the largest local block count).
  *   softmax_scale    multiplier of q.k (e.g. 1/sqrt(head_dim); MLA 1/sqrt(192)).
+ *   q_len            query tokens per request: 1 = single-token decode; 2..4 = multi-token
+ *                    decode (MTP / speculative drafts; [P1] "A5 结论", future-work item 3,
+ *                    names MTP and speculative decoding as what DCP must support next).
+ *                    The q_len new tokens are the LAST q_len tokens of the request and their
+ *                    KV is already in the cache (seq_len counts them); query token j
+ *                    (0-based) attends the tokens t < seq_len - (q_len - 1 - j), i.e.
+ *                    causally within the draft.  A query token with no visible token in a
+ *                    shard gets O = 0, LSE = -inf there.
  */
 typedef struct dcp_attn_desc {
     int32_t layout;
@@ -95,6 +105,7 @@ typedef struct dcp_attn_desc {
     int32_t block_size;
     int32_t max_local_blocks;
     float softmax_scale;
+    int32_t q_len;
 } dcp_attn_desc;
 
 /* Library version, major * 10000 + minor * 100 + patch. */
@@ -218,12 +229,14 @@ DCP_API dcp_status dcp_workspace_init(void *workspace, size_t workspace_bytes, v
  * GQA: k_t, v_t are KV head h / (Hq/Hkv) of token t.  MLA: k_t is the whole
  * 576-wide latent row, v_t its first 512 entries.  A request with no token
  * in this shard gets O_i = 0 and LSE_i = -inf.
- *   q           device bf16 [batch][Hq][head_dim_qk] (the full query: every shard reads it).
+ *   q           device bf16 [batch][q_len][Hq][head_dim_qk] (the full query: every shard reads it).
  *   kv_pool     device, this shard's pool (layout as in dcp_place_kv), pool_pages pages.
  *   table       device int32 [batch][max_local_blocks], this shard's block table.
  *   seq_lens    device int32 [batch], GLOBAL lengths; the local token count is
  *               derived from (seq_len, block_size, shard, D).
- *   O_i         device fp32 [batch][Hq][head_dim_v];  LSE_i  device fp32 [batch][Hq].
+ *   O_i         device fp32 [batch][q_len][Hq][head_dim_v];  LSE_i  device fp32 [batch][q_len][Hq].
+ * With q_len > 1 each (request, query token j, head) row follows the same
+ * formulas over the visible tokens t < seq_len - (q_len - 1 - j).
  *   workspace   device, >= dcp_decode_workspace_bytes(desc, D) bytes, initialised.
  * Page ids outside [0, pool_pages) are not read (their tokens count as zero
  * keys and values) and set the workspace status (see dcp_read_device_error).
@@ -284,7 +297,7 @@ DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc *desc, con
  *   LSE_out[r] = max_j LSE_j[r] + ln sum_i w_i.
  * Parts with LSE = -inf weigh 0; if all are -inf then O = 0, LSE_out = -inf.
  *   O_parts, LSE_parts  host arrays of D device pointers: fp32 [rows][d_v] and fp32 [rows].
- *   rows                number of (request, head) rows (batch * Hq).
+ *   rows                number of (request, query token, head) rows (batch * q_len * Hq).
  *   O                   device fp32 [rows][d_v]; LSE_out device fp32 [rows] or NULL.
  * d_v must be a multiple of 4 and all pointers 16-byte aligned.
  */

@@ -20,8 +20,9 @@ from . import dcp
 class ShardedPagedCache:
     def __init__(self, layout: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
                  block_size: int, D: int, seq_lens: Sequence[int], softmax_scale: float, perm_seed: int = 0,
-                 device="cuda", pool_fill: Optional[int] = None):
+                 device="cuda", pool_fill: Optional[int] = None, q_len: int = 1):
         self.D = D
+        self.q_len = q_len
         self.device = torch.device(device)
         self.seq_lens = [int(x) for x in seq_lens]
         self.batch = len(self.seq_lens)
@@ -31,7 +32,7 @@ class ShardedPagedCache:
         self.tables_host, self.local_len = dcp.dcp_build_block_table(self.seq_lens, block_size, D, perm_seed,
                                                                      self.max_local_blocks)
         self.desc = dcp.make_desc(layout, self.batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v,
-                                  block_size, self.max_local_blocks, softmax_scale)
+                                  block_size, self.max_local_blocks, softmax_scale, q_len)
         self.page_bytes = dcp.dcp_kv_page_bytes(self.desc)
         if self.page_bytes == 0:
             raise ValueError("unsupported attention shape")
@@ -52,10 +53,12 @@ class ShardedPagedCache:
         self.ws_bytes = dcp.dcp_decode_workspace_bytes(self.desc, D)
         self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         dcp.dcp_workspace_init(self.workspace)
-        self.O_parts = torch.empty((D, self.batch, num_q_heads, head_dim_v), dtype=torch.float32, device=self.device)
-        self.LSE_parts = torch.empty((D, self.batch, num_q_heads), dtype=torch.float32, device=self.device)
-        self.O = torch.empty((self.batch, num_q_heads, head_dim_v), dtype=torch.float32, device=self.device)
-        self.LSE = torch.empty((self.batch, num_q_heads), dtype=torch.float32, device=self.device)
+        # outputs [B][Hq](...) for single-token decode, [B][q_len][Hq](...) for multi-token decode
+        rows = (self.batch, num_q_heads) if q_len == 1 else (self.batch, q_len, num_q_heads)
+        self.O_parts = torch.empty((D, *rows, head_dim_v), dtype=torch.float32, device=self.device)
+        self.LSE_parts = torch.empty((D, *rows), dtype=torch.float32, device=self.device)
+        self.O = torch.empty((*rows, head_dim_v), dtype=torch.float32, device=self.device)
+        self.LSE = torch.empty(rows, dtype=torch.float32, device=self.device)
 
     # ------------------------------------------------------------------ cache write
     def place(self, kv_src: torch.Tensor, device_error: Optional[torch.Tensor] = None) -> None:
@@ -74,7 +77,7 @@ class ShardedPagedCache:
                                        self.D, list(self.O_parts), list(self.LSE_parts), self.workspace)
 
     def merge(self, with_lse: bool = True) -> None:
-        rows = self.batch * self.desc.num_q_heads
+        rows = self.batch * self.q_len * self.desc.num_q_heads
         dcp.dcp_lse_merge(list(self.O_parts), list(self.LSE_parts), self.D, rows, self.desc.head_dim_v, self.O,
                           self.LSE if with_lse else None)
 
@@ -114,14 +117,15 @@ class HostStepPipeline:
     def __init__(self, cache: ShardedPagedCache):
         self.cache = c = cache
         d = c.desc
-        self.q_elems = c.batch * d.num_q_heads * d.head_dim_qk
+        self.rows = c.batch * c.q_len * d.num_q_heads  # (request, query token, head) rows
+        self.q_elems = self.rows * d.head_dim_qk
         self.q_off, self.sl_off = 0, _align(self.q_elems * 2)
         self.tab_off = self.sl_off + _align(c.batch * 4)
         self.tab_elems = c.batch * c.max_local_blocks
         self.in_bytes = self.tab_off + c.D * self.tab_elems * 4
-        self.o_elems = c.batch * d.num_q_heads * d.head_dim_v
+        self.o_elems = self.rows * d.head_dim_v
         self.lse_off = self.o_elems * 4
-        self.out_bytes = self.lse_off + c.batch * d.num_q_heads * 4
+        self.out_bytes = self.lse_off + self.rows * 4
         dev = c.device
         self.dev_in = [torch.empty(self.in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
         self.dev_out = [torch.empty(self.out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
@@ -146,8 +150,8 @@ class HostStepPipeline:
 
     def unpack_output(self, buf: torch.Tensor):
         d = self.cache.desc
-        O = buf[:self.lse_off].view(torch.float32).view(self.cache.batch, d.num_q_heads, d.head_dim_v)
-        L = buf[self.lse_off:].view(torch.float32).view(self.cache.batch, d.num_q_heads)
+        O = buf[:self.lse_off].view(torch.float32).view(self.cache.O.shape)
+        L = buf[self.lse_off:].view(torch.float32).view(self.cache.LSE.shape)
         return O, L
 
     # ------------------------------------------------------------------ one step
@@ -170,7 +174,7 @@ class HostStepPipeline:
             self.s_comp.wait_event(self.ev_out[k])         # slot k's results have been read back
         dcp.dcp_decode_partial_all(c.desc, q, c.pools, c.pool_pages, tabs, sl, c.D, list(c.O_parts),
                                    list(c.LSE_parts), c.workspace, stream=self.s_comp)
-        dcp.dcp_lse_merge(list(c.O_parts), list(c.LSE_parts), c.D, c.batch * c.desc.num_q_heads,
+        dcp.dcp_lse_merge(list(c.O_parts), list(c.LSE_parts), c.D, self.rows,
                           c.desc.head_dim_v, o_dev, l_dev, stream=self.s_comp)
         self.ev_comp[k].record(self.s_comp)
         with torch.cuda.stream(self.s_out):

@@ -69,8 +69,11 @@ CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elem
 bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
   *why = DCP_ERR_INVALID_ARG;
   if (D < 1 || D > kMaxShardsHost || d.batch < 1 || d.num_q_heads < 1 || d.num_kv_heads < 1 || d.block_size < 1 ||
-      d.max_local_blocks < 1 || d.head_dim_qk < 1 || d.head_dim_v < 1 || !(d.softmax_scale == d.softmax_scale))
+      d.max_local_blocks < 1 || d.head_dim_qk < 1 || d.head_dim_v < 1 || !(d.softmax_scale == d.softmax_scale) ||
+      d.q_len < 1)
     return false;
+  *why = DCP_ERR_UNSUPPORTED;
+  if (d.q_len > kMaxQLen) return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.layout == DCP_LAYOUT_GQA) {
     if (d.head_dim_qk != d.head_dim_v || (d.head_dim_qk != 64 && d.head_dim_qk != 128)) return false;
@@ -86,21 +89,22 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
   return false;
 }
 
-int mla_ctas();
+int mla_ctas(int q_len);
 
 bool workspace_layout(const dcp_attn_desc& d, int D, WorkspaceLayout* L) {
   dcp_status why;
   if (!desc_supported(d, D, &why)) return false;
   const int sms = device_sm_count();
   if (d.layout == DCP_LAYOUT_GQA) {
-    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size, d.head_dim_qk);
+    const int G = d.num_q_heads / d.num_kv_heads;
+    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size, d.head_dim_qk, gqa_row_tiles(G, d.q_len));
     L->n_hg = d.num_kv_heads / hpc;
-    L->rows_per_hg = hpc * (d.num_q_heads / d.num_kv_heads);
+    L->rows_per_hg = hpc * G * d.q_len;
     L->nctas = sms / L->n_hg > 0 ? sms / L->n_hg : 1;
   } else {
-    L->n_hg = 1;
+    L->n_hg = d.q_len;  // one group per query token (blockIdx.y)
     L->rows_per_hg = d.num_q_heads;
-    L->nctas = mla_ctas();
+    L->nctas = mla_ctas(d.q_len);
   }
   L->slot_floats = (L->rows_per_hg * (d.head_dim_v + 1) + 3) & ~3;
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };

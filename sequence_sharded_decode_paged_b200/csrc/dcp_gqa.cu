@@ -15,12 +15,15 @@
 //  * One producer thread streams whole pages of the CTA's KV-head group into
 //    a ring of shared-memory stages with 2-D TMA tiles (128-byte swizzle, no
 //    multicast); K and V of all heads of one page arrive on one mbarrier.
-//  * Eight consumer warps; each owns one KV head and all G <= 16 query heads
-//    sharing it (16-row mma tile).  Per 16-token chunk: S = Q K^T with
+//  * Eight consumer warps; each owns one KV head and one 16-row mma tile of
+//    the R = q_len * G query rows sharing it (row r = query token r / G, head
+//    r % G; R <= 16 is one tile per head).  Per 16-token chunk: S = Q K^T with
 //    mma.m16n8k16 (K fragments by ldmatrix), online softmax in fp32 with quad
 //    shuffles, P rounded to bf16 in registers and O += P V (V by
 //    ldmatrix.trans).  Tokens past the sequence end are masked in both S and
 //    the V fragments, so stale cache contents (even NaN) never leak in.
+//  * Multi-token decode (q_len > 1): row r sees only the tokens before
+//    seq_len - (q_len - 1 - r / G); the rest of its scores are masked.
 #include <float.h>
 
 #include "dcp_device.cuh"
@@ -47,10 +50,18 @@ struct GqaParams {
   float* slots;
   float scale_log2;
   int n_si, B, Hq, Hkv, G, bs, D, mlb;
+  int q_len, R, rt;  // query tokens per request, rows per KV head (q_len * G), 16-row tiles per head
   int hpc, n_hg, stages, wph;
   uint32_t stage_bytes;
   int slot_floats;
 };
+
+// Output row of head-group row rr = h * R + r (KV head kv0 + h, local row r =
+// query token r / G, head r % G) of request b: [b][r / G][(kv0 + h) * G + r % G].
+__device__ __forceinline__ size_t gqa_out_row(int rr, int b, int ql, int Hq, int kv0, int G, int R) {
+  const int h = rr / R, r = rr - h * R, jq = r / G;
+  return ((size_t)b * ql + jq) * Hq + (size_t)(kv0 + h) * G + (r - jq * G);
+}
 
 template <int HEAD_DIM>
 struct GqaGeom {
@@ -60,7 +71,9 @@ struct GqaGeom {
   static constexpr int kCombineFloats = kNTiles * 4 + 4;  // per lane per warp
 };
 
-template <int HEAD_DIM>
+// MULTI: multi-token decode (q_len > 1, per-row causal limits); the single-token
+// instantiation keeps the plain end-of-sequence mask and its register budget.
+template <int HEAD_DIM, bool MULTI>
 __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid_constant__ GqaParams p) {
   using Geo = GqaGeom<HEAD_DIM>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -154,12 +167,13 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   }
 
   // ------------------------------------------------------------------ consumers
-  const int hpc = p.hpc, G = p.G, wph = p.wph;
-  const bool active = warp < hpc * wph;
-  const int hh = warp % hpc, sub = warp / hpc;
+  const int hpc = p.hpc, G = p.G, wph = p.wph, R = MULTI ? p.R : p.G, ql = MULTI ? p.q_len : 1;
+  const int hu = MULTI ? hpc * p.rt : hpc;  // (KV head, row tile) units of one CTA; one tile if q_len = 1
+  const bool active = warp < hu * wph;
+  const int u = warp % hu, sub = warp / hu;
+  const int hh = MULTI ? u % hpc : u, tile = MULTI ? u / hpc : 0;
   const int g4 = lane >> 2, c4 = lane & 3;
-  const int rows_hg = hpc * G;
-  const int qrow0 = hg * rows_hg;  // first query head of this head group
+  const int rows_hg = hpc * R;  // rows of one head group: (head hh, row r) at hh * R + r
   int stage = 0;
   uint32_t phase = 0;
   int pre = plan.pre0;
@@ -172,28 +186,42 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     const int c0 = seg_first_cta(pre, n, T, P);
     if (c0 > cta) break;
     const int c1 = seg_last_cta(pre, n, T, P);
-    float* Oout = p.O[si] + ((size_t)b * p.Hq + qrow0) * HEAD_DIM;
-    float* Lout = p.LSE[si] + (size_t)b * p.Hq + qrow0;
     if (n == 0) {  // no token of this request in this shard
-      for (int i = tid; i < rows_hg * HEAD_DIM; i += kGqaConsumerWarps * 32) Oout[i] = 0.f;
-      for (int i = tid; i < rows_hg; i += kGqaConsumerWarps * 32) Lout[i] = -INFINITY;
+      float* Obase = p.O[si];
+      float* Lbase = p.LSE[si];
+      for (int i = tid; i < rows_hg * HEAD_DIM; i += kGqaConsumerWarps * 32)
+        Obase[gqa_out_row(i / HEAD_DIM, b, ql, p.Hq, hg * hpc, G, R) * HEAD_DIM + i % HEAD_DIM] = 0.f;
+      for (int i = tid; i < rows_hg; i += kGqaConsumerWarps * 32)
+        Lbase[gqa_out_row(i, b, ql, p.Hq, hg * hpc, G, R)] = -INFINITY;
       pre += n;
       continue;
     }
     const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
 
-    // query fragments (16-row A tile; rows >= G are zero)
+    // query fragments (16-row A tile; rows >= R are zero)
     uint32_t qa[Geo::kKTiles][4];
     const int kvh = hg * hpc + hh;
+    int lim0 = seq_len, lim1 = seq_len;  // tokens each row may see
     {
-      const uint32_t* qb = reinterpret_cast<const uint32_t*>(p.q + ((size_t)b * p.Hq + (size_t)kvh * G) * HEAD_DIM);
+      // this thread's two accumulator rows (r and r + 8 of the warp's tile), their query tokens
+      const int r0 = tile * 16 + g4, r1 = r0 + 8;
+      const bool row0 = active && r0 < R, row1 = active && r1 < R;
+      const int j0 = (MULTI && row0) ? r0 / G : 0, j1 = (MULTI && row1) ? r1 / G : 0;
+      const size_t q0 = (((size_t)b * ql + j0) * p.Hq + (size_t)kvh * G + (r0 - j0 * G)) * HEAD_DIM;
+      const size_t q1 = (((size_t)b * ql + j1) * p.Hq + (size_t)kvh * G + (r1 - j1 * G)) * HEAD_DIM;
+      const uint32_t* qb0 = reinterpret_cast<const uint32_t*>(p.q + (row0 ? q0 : 0));
+      const uint32_t* qb1 = reinterpret_cast<const uint32_t*>(p.q + (row1 ? q1 : 0));
 #pragma unroll
       for (int kt = 0; kt < Geo::kKTiles; ++kt) {
         const int col = kt * 16 + c4 * 2;
-        qa[kt][0] = (active && g4 < G) ? __ldg(qb + (g4 * HEAD_DIM + col) / 2) : 0u;
-        qa[kt][1] = (active && g4 + 8 < G) ? __ldg(qb + ((g4 + 8) * HEAD_DIM + col) / 2) : 0u;
-        qa[kt][2] = (active && g4 < G) ? __ldg(qb + (g4 * HEAD_DIM + col + 8) / 2) : 0u;
-        qa[kt][3] = (active && g4 + 8 < G) ? __ldg(qb + ((g4 + 8) * HEAD_DIM + col + 8) / 2) : 0u;
+        qa[kt][0] = row0 ? __ldg(qb0 + col / 2) : 0u;
+        qa[kt][1] = row1 ? __ldg(qb1 + col / 2) : 0u;
+        qa[kt][2] = row0 ? __ldg(qb0 + (col + 8) / 2) : 0u;
+        qa[kt][3] = row1 ? __ldg(qb1 + (col + 8) / 2) : 0u;
+      }
+      if (MULTI) {  // up to the row's own draft position
+        lim0 = seq_len - (ql - 1 - j0);
+        lim1 = seq_len - (ql - 1 - j1);
       }
     }
     float o[Geo::kNTiles][4];
@@ -230,12 +258,14 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           }
           // ---- online softmax (log2 domain), rows g4 and g4 + 8
           const int vrem = valid - t0;
+          const int vr0 = MULTI ? lim0 - (gblk * bs + t0) : vrem;
+          const int vr1 = MULTI ? lim1 - (gblk * bs + t0) : vrem;
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int tok = nt * 8 + c4 * 2 + (i & 1);
-              s[nt][i] = tok < vrem ? s[nt][i] * p.scale_log2 : -INFINITY;
+              s[nt][i] = tok < (i < 2 ? vr0 : vr1) ? s[nt][i] * p.scale_log2 : -INFINITY;
             }
           float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
           float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -248,12 +278,16 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
           m0 = mn0;
           m1 = mn1;
+          // a row that has seen no visible token yet keeps -inf: subtract 0 so exp2 gives 0
+          // (single-token decode always has a visible token in every chunk it processes)
+          const float sub0 = (MULTI && mn0 == -INFINITY) ? 0.f : mn0;
+          const float sub1 = (MULTI && mn1 == -INFINITY) ? 0.f : mn1;
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            s[nt][0] = exp2f(s[nt][0] - mn0);
-            s[nt][1] = exp2f(s[nt][1] - mn0);
-            s[nt][2] = exp2f(s[nt][2] - mn1);
-            s[nt][3] = exp2f(s[nt][3] - mn1);
+            s[nt][0] = exp2f(s[nt][0] - sub0);
+            s[nt][1] = exp2f(s[nt][1] - sub0);
+            s[nt][2] = exp2f(s[nt][2] - sub1);
+            s[nt][3] = exp2f(s[nt][3] - sub1);
           }
           l0 = l0 * al0 + (s[0][0] + s[0][1] + s[1][0] + s[1][1]);
           l1 = l1 * al1 + (s[0][2] + s[0][3] + s[1][2] + s[1][3]);
@@ -316,7 +350,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       named_bar_sync(1, kGqaConsumerWarps * 32);
       if (active && sub == 0) {
         for (int w2 = 1; w2 < wph; ++w2) {
-          const float* other = combine + (size_t)(w2 * hpc + hh) * Geo::kCombineFloats * 32;
+          const float* other = combine + (size_t)(w2 * hu + u) * Geo::kCombineFloats * 32;
           const float om0 = other[(Geo::kNTiles * 4 + 0) * 32 + lane];
           const float om1 = other[(Geo::kNTiles * 4 + 1) * 32 + lane];
           const float ol0 = other[(Geo::kNTiles * 4 + 2) * 32 + lane];
@@ -348,31 +382,28 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       const float lse0 = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
       const float lse1 = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
       const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-      float* dstO;
-      float* dstL;
-      size_t stride;
-      if (complete) {
-        dstO = Oout + (size_t)hh * G * HEAD_DIM;
-        dstL = Lout + hh * G;
-        stride = HEAD_DIM;
-      } else {
-        float* sl = p.slots + ((size_t)slot * p.n_hg + hg) * p.slot_floats;
-        dstO = sl + (size_t)hh * G * HEAD_DIM;
-        dstL = sl + (size_t)rows_hg * HEAD_DIM + hh * G;
-        stride = HEAD_DIM;
-      }
-      if (g4 < G) {
+      // destination rows: the outputs, or this CTA's slot (rows in head-group order)
+      float* Obase = p.O[si];
+      float* Lbase = p.LSE[si];
+      auto out_row = [=](int rr) { return gqa_out_row(rr, b, ql, p.Hq, hg * hpc, G, R); };
+      const int r0 = tile * 16 + g4, r1 = r0 + 8;
+      const bool row0 = r0 < R, row1 = r1 < R;
+      float* sl = p.slots + ((size_t)slot * p.n_hg + hg) * p.slot_floats;
+      float* dO0 = complete ? Obase + out_row(hh * R + r0) * HEAD_DIM : sl + (size_t)(hh * R + r0) * HEAD_DIM;
+      float* dO1 = complete ? Obase + out_row(hh * R + r1) * HEAD_DIM : sl + (size_t)(hh * R + r1) * HEAD_DIM;
+      float* dL0 = complete ? Lbase + out_row(hh * R + r0) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r0;
+      float* dL1 = complete ? Lbase + out_row(hh * R + r1) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r1;
+      if (row0) {
 #pragma unroll
         for (int i = 0; i < Geo::kNTiles; ++i)
-          *reinterpret_cast<float2*>(dstO + g4 * stride + i * 8 + c4 * 2) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
-        if (c4 == 0) dstL[g4] = complete ? lse0 * kLn2 : lse0;
+          *reinterpret_cast<float2*>(dO0 + i * 8 + c4 * 2) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
+        if (c4 == 0) *dL0 = complete ? lse0 * kLn2 : lse0;
       }
-      if (g4 + 8 < G) {
+      if (row1) {
 #pragma unroll
         for (int i = 0; i < Geo::kNTiles; ++i)
-          *reinterpret_cast<float2*>(dstO + (g4 + 8) * stride + i * 8 + c4 * 2) =
-              make_float2(o[i][2] * inv1, o[i][3] * inv1);
-        if (c4 == 0) dstL[g4 + 8] = complete ? lse1 * kLn2 : lse1;
+          *reinterpret_cast<float2*>(dO1 + i * 8 + c4 * 2) = make_float2(o[i][2] * inv1, o[i][3] * inv1);
+        if (c4 == 0) *dL1 = complete ? lse1 * kLn2 : lse1;
       }
     }
     if (!complete) {
@@ -408,9 +439,12 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
             }
           }
           const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+          const size_t orow = gqa_out_row(r, b, ql, p.Hq, hg * hpc, G, R);
+          float* Obase = p.O[si];
+          float* Lbase = p.LSE[si];
 #pragma unroll
-          for (int i = 0; i < kPer; ++i) Oout[(size_t)r * HEAD_DIM + lane * kPer + i] = acc[i] * inv;
-          if (lane == 0) Lout[r] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+          for (int i = 0; i < kPer; ++i) Obase[orow * HEAD_DIM + lane * kPer + i] = acc[i] * inv;
+          if (lane == 0) Lbase[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
         }
         if (tid == 0) *ctr = 0;  // leave the counter ready for the next call
       }
@@ -420,11 +454,14 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
 }
 
 // ---------------------------------------------------------------------------- host side
-// KV heads one CTA streams per page: a divisor of Hkv, at most 8 (one consumer
-// warp each), a TMA box of at most 256 rows, and a stage (K and V of those
-// heads for one page) of at most 64 KB so that three or more stages fit.
-int gqa_heads_per_cta(int Hkv, int bs, int head_dim) {
-  int cap = min(kGqaConsumerWarps, 256 / bs);
+// KV heads one CTA streams per page: a divisor of Hkv, at most 8 / row_tiles
+// (one consumer warp per head and 16-row tile), a TMA box of at most 256 rows,
+// and a stage (K and V of those heads for one page) of at most 64 KB so that
+// three or more stages fit.
+int gqa_row_tiles(int G, int q_len) { return (G * q_len + 15) / 16; }
+
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles) {
+  int cap = min(kGqaConsumerWarps / row_tiles, 256 / bs);
   cap = min(cap, 65536 / (bs * head_dim * 4));
   int best = 1;
   for (int h = 1; h <= cap; ++h)
@@ -438,7 +475,7 @@ static int gqa_stage_count(uint32_t stage_bytes, size_t fixed_bytes) {
   return st > 8 ? 8 : st;
 }
 
-template <int HEAD_DIM>
+template <int HEAD_DIM, bool MULTI>
 static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                                   const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
   WorkspaceLayout L;
@@ -454,9 +491,12 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.bs = d.block_size;
   p.D = D;
   p.mlb = d.max_local_blocks;
-  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs, HEAD_DIM);
+  p.q_len = d.q_len;
+  p.R = p.G * p.q_len;
+  p.rt = gqa_row_tiles(p.G, p.q_len);
+  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs, HEAD_DIM, p.rt);
   p.n_hg = p.Hkv / p.hpc;
-  p.wph = kGqaConsumerWarps / p.hpc;
+  p.wph = kGqaConsumerWarps / (p.hpc * p.rt);
   p.stage_bytes = (uint32_t)(2 * p.hpc * p.bs * HEAD_DIM * 2);
   const size_t combine_bytes =
       p.wph > 1 ? (size_t)kGqaConsumerWarps * GqaGeom<HEAD_DIM>::kCombineFloats * 32 * sizeof(float) : 0;
@@ -485,7 +525,7 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
     }
   }
   const size_t smem = (size_t)p.stages * p.stage_bytes + fixed;
-  auto kern = gqa_decode_kernel<HEAD_DIM>;
+  auto kern = gqa_decode_kernel<HEAD_DIM, MULTI>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return DCP_ERR_CUDA;
   dim3 grid(L.nctas, p.n_hg);
@@ -495,8 +535,13 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
 
 dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
-  if (d.head_dim_qk == 128) return launch_gqa_impl<128>(d, D, set, q, seq_lens, ws, ws_bytes, st);
-  if (d.head_dim_qk == 64) return launch_gqa_impl<64>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+  const bool multi = d.q_len > 1;
+  if (d.head_dim_qk == 128)
+    return multi ? launch_gqa_impl<128, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                 : launch_gqa_impl<128, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+  if (d.head_dim_qk == 64)
+    return multi ? launch_gqa_impl<64, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                 : launch_gqa_impl<64, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
   return DCP_ERR_UNSUPPORTED;
 }
 

@@ -11,6 +11,7 @@
 namespace dcp {
 
 constexpr int kMaxShardsHost = 16;
+constexpr int kMaxQLen = 4;  // query tokens per request (multi-token decode)
 
 // The shards one decode launch works on: slot si computes shard shard[si].
 struct ShardSet {
@@ -56,6 +57,7 @@ dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, co
                            const int32_t* pool_pages, int32_t* device_error, cudaStream_t st);
 
 // GQA geometry helpers (shared by the workspace sizing and the launcher).
-int gqa_heads_per_cta(int Hkv, int bs, int head_dim);
+int gqa_row_tiles(int G, int q_len);
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles);
 
 }  // namespace dcp

@@ -35,6 +35,11 @@
 //    shared memory before the PV product, so stale cache contents never leak in.
 //    Epilogue: O^T rows (value dims) are read from TMEM, normalised per head
 //    and stored with coalesced 128-byte writes.
+//  * Multi-token decode (q_len > 1): blockIdx.y is the query token j; the
+//    q_len CTAs of one page range run side by side (the grid keeps q_len x
+//    ranges within one wave), so each latent page is fetched from HBM about
+//    once and the other reads hit L2.  Token j masks the scores of tokens at
+//    or past seq_len - (q_len - 1 - j).
 #include <float.h>
 
 #include "dcp_device.cuh"
@@ -96,7 +101,7 @@ struct MlaParams {
   int* counters;
   float* slots;
   float scale_log2;
-  int n_si, B, D, mlb, slot_floats;
+  int n_si, B, D, mlb, slot_floats, q_len;
 };
 
 namespace {
@@ -140,6 +145,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
   MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x, nctas = gridDim.x;
+  const int jq = blockIdx.y, ql = p.q_len;  // query token of this CTA
   const int B = p.B, D = p.D;
 
   if ((smem_u32(smem) & 1023u) != 0u) {  // swizzled tiles need 1024-byte alignment
@@ -199,7 +205,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         if (dead) break;
         mbar_arrive_expect_tx(&misc->q_full, kTileBytes);
         for (int cb = 0; cb < 9; ++cb)
-          tma_load_2d(smem + kOffQ + cb * kBlockBytes, &p.qmap, cb * 64, b * kMlaHeads, &misc->q_full);
+          tma_load_2d(smem + kOffQ + cb * kBlockBytes, &p.qmap, cb * 64, (b * ql + jq) * kMlaHeads, &misc->q_full);
         q_issued = true;
         for (int j = a; j < e; ++j) {
           int page;
@@ -389,8 +395,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       const int c0 = seg_first_cta(pre, n, T, P);
       if (c0 > cta) break;
       const int c1 = seg_last_cta(pre, n, T, P);
-      float* Oout = p.O[si] + (size_t)b * kMlaHeads * kMlaDv;
-      float* Lout = p.LSE[si] + (size_t)b * kMlaHeads;
+      float* Oout = p.O[si] + ((size_t)b * ql + jq) * kMlaHeads * kMlaDv;
+      float* Lout = p.LSE[si] + ((size_t)b * ql + jq) * kMlaHeads;
+      const int lim = seq_len - (ql - 1 - jq);  // tokens this query token sees
       if (n == 0) {
         for (int i = ts; i < kMlaHeads * kMlaDv / 4; i += kSoftmaxThreads)
           reinterpret_cast<float4*>(Oout)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -409,6 +416,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         int page;
         const bool ok = page_ok(p, si, b, j, &page);
         const int valid = min(kMlaBs, seq_len - (j * D + shard) * kMlaBs);
+        const int vis = lim - (j * D + shard) * kMlaBs;  // visible tokens of this page (may be <= 0)
         const uint32_t sb = gpage & 1u;
         wait_or_die_warp(&misc->s_full[sb], (gpage >> 1) & 1u, dead, p.status);
         tc_fence_after();
@@ -428,7 +436,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int tok = 32 * hf + 8 * k + 2 * quad + (i & 1);
-              s[4 * k + i] = tok < valid ? s[4 * k + i] * p.scale_log2 : -INFINITY;
+              s[4 * k + i] = tok < vis ? s[4 * k + i] * p.scale_log2 : -INFINITY;
             }
           pm0 = fmaxf(fmaxf(fmaxf(s[0], s[1]), fmaxf(s[4], s[5])), fmaxf(fmaxf(s[8], s[9]), fmaxf(s[12], s[13])));
           pm1 = fmaxf(fmaxf(fmaxf(s[2], s[3]), fmaxf(s[6], s[7])), fmaxf(fmaxf(s[10], s[11]), fmaxf(s[14], s[15])));
@@ -463,12 +471,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             m1 = mn;
             need = need || have_o;
           }
+          // a row with no visible token so far keeps -inf: subtract 0 so ex2 gives 0
+          const float sub0 = m0 == -INFINITY ? 0.f : m0, sub1 = m1 == -INFINITY ? 0.f : m1;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            s[4 * k + 0] = ex2_approx(s[4 * k + 0] - m0);
-            s[4 * k + 1] = ex2_approx(s[4 * k + 1] - m0);
-            s[4 * k + 2] = ex2_approx(s[4 * k + 2] - m1);
-            s[4 * k + 3] = ex2_approx(s[4 * k + 3] - m1);
+            s[4 * k + 0] = ex2_approx(s[4 * k + 0] - sub0);
+            s[4 * k + 1] = ex2_approx(s[4 * k + 1] - sub0);
+            s[4 * k + 2] = ex2_approx(s[4 * k + 2] - sub1);
+            s[4 * k + 3] = ex2_approx(s[4 * k + 3] - sub1);
           }
           l0 = l0 * a0 + (((s[0] + s[1]) + (s[4] + s[5])) + ((s[8] + s[9]) + (s[12] + s[13])));
           l1 = l1 * a1 + (((s[2] + s[3]) + (s[6] + s[7])) + ((s[10] + s[11]) + (s[14] + s[15])));
@@ -550,8 +560,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       named_bar_sync(2, kSoftmaxThreads);
       const bool complete = (c0 == c1);
       const int slot = complete ? 0 : 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
-      float* dstO = complete ? Oout : p.slots + (size_t)slot * p.slot_floats;
-      float* dstL = complete ? Lout : p.slots + (size_t)slot * p.slot_floats + kMlaHeads * kMlaDv;
+      float* slot_base = p.slots + ((size_t)slot * ql + jq) * p.slot_floats;
+      float* dstO = complete ? Oout : slot_base;
+      float* dstL = complete ? Lout : slot_base + kMlaHeads * kMlaDv;
 #pragma unroll 1
       for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
 #pragma unroll 1
@@ -575,7 +586,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       if (!complete) {
         __threadfence();
         named_bar_sync(2, kSoftmaxThreads);
-        int* ctr = p.counters + sid;
+        int* ctr = p.counters + (size_t)sid * ql + jq;
         if (ts == 0) misc->bcast = (atomicAdd(ctr, 1) == c1 - c0) ? 1 : 0;
         named_bar_sync(2, kSoftmaxThreads);
         if (misc->bcast) {
@@ -585,7 +596,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             float mx = -INFINITY;
             for (int c = c0; c <= c1; ++c) {
               const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-              mx = fmaxf(mx, __ldcg(p.slots + (size_t)k * p.slot_floats + kMlaHeads * kMlaDv + r));
+              mx = fmaxf(mx, __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + r));
             }
             float4 acc[4];
 #pragma unroll
@@ -594,7 +605,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             if (mx != -INFINITY) {
               for (int c = c0; c <= c1; ++c) {
                 const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-                const float* sl = p.slots + (size_t)k * p.slot_floats;
+                const float* sl = p.slots + ((size_t)k * ql + jq) * p.slot_floats;
                 const float lk = __ldcg(sl + kMlaHeads * kMlaDv + r);
                 const float w = lk == -INFINITY ? 0.f : exp2f(lk - mx);
                 wsum += w;
@@ -632,7 +643,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
 }
 
 // ---------------------------------------------------------------------------- host side
-int mla_ctas() { return device_sm_count(); }
+// CTAs per query token: q_len x ranges fill one wave (one CTA per SM).
+int mla_ctas(int q_len) {
+  const int n = device_sm_count() / q_len;
+  return n > 0 ? n : 1;
+}
 
 dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream) {
@@ -647,13 +662,14 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   p.mlb = d.max_local_blocks;
   p.slot_floats = L.slot_floats;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  p.q_len = d.q_len;
   p.seq_lens = seq_lens;
   p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
   p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);
   p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slots_off);
-  if ((uint64_t)d.batch * kMlaHeads > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;
-  if (encode_tiled_2d(&p.qmap, q, kMlaDqk, (uint64_t)d.batch * kMlaHeads, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS)
-    return DCP_ERR_CUDA;
+  const uint64_t q_rows = (uint64_t)d.batch * d.q_len * kMlaHeads;  // q: [batch][q_len][64][576]
+  if (q_rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;
+  if (encode_tiled_2d(&p.qmap, q, kMlaDqk, q_rows, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS) return DCP_ERR_CUDA;
   for (int si = 0; si < set.n; ++si) {
     p.table[si] = set.table[si];
     p.O[si] = set.O[si];
@@ -670,7 +686,7 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   if (cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMlaSmem) !=
       cudaSuccess)
     return DCP_ERR_CUDA;
-  mla_decode_kernel<<<L.nctas, kMlaThreads, kMlaSmem, stream>>>(p);
+  mla_decode_kernel<<<dim3(L.nctas, d.q_len), kMlaThreads, kMlaSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
 }
 

@@ -37,7 +37,8 @@ class DcpError(RuntimeError):
 class dcp_attn_desc(C.Structure):
     _fields_ = [("layout", C.c_int32), ("batch", C.c_int32), ("num_q_heads", C.c_int32),
                 ("num_kv_heads", C.c_int32), ("head_dim_qk", C.c_int32), ("head_dim_v", C.c_int32),
-                ("block_size", C.c_int32), ("max_local_blocks", C.c_int32), ("softmax_scale", C.c_float)]
+                ("block_size", C.c_int32), ("max_local_blocks", C.c_int32), ("softmax_scale", C.c_float),
+                ("q_len", C.c_int32)]
 
 
 def _load() -> C.CDLL:
@@ -107,9 +108,9 @@ def _i32(a) -> np.ndarray:
 
 
 def make_desc(layout: int, batch: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
-              block_size: int, max_local_blocks: int, softmax_scale: float) -> dcp_attn_desc:
+              block_size: int, max_local_blocks: int, softmax_scale: float, q_len: int = 1) -> dcp_attn_desc:
     return dcp_attn_desc(layout, batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v, block_size,
-                         max_local_blocks, softmax_scale)
+                         max_local_blocks, softmax_scale, q_len)
 
 
 # --------------------------------------------------------------------------- host calls

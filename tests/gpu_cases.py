@@ -24,14 +24,15 @@ def host_kv(w: synth.Workload, requests=None) -> np.ndarray:
 
 
 def host_q(w: synth.Workload) -> np.ndarray:
-    return np.stack([w.query(b) for b in range(w.batch)])
+    """[B][Hq][d] queries, or [B][q_len][Hq][d] for multi-token decode."""
+    return np.stack([w.query(b) if w.q_len == 1 else w.queries(b) for b in range(w.batch)])
 
 
 def build_cache(w: synth.Workload, D: int, perm_seed: int = 0, pool_fill=0xFFFF, device_kv: bool = False):
     """Cache with the workload's KV placed in D shard pools; returns (cache, q on device)."""
     import synth.device as sdev
     cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size, D,
-                              w.seq_lens, w.softmax_scale, perm_seed, "cuda", pool_fill)
+                              w.seq_lens, w.softmax_scale, perm_seed, "cuda", pool_fill, q_len=w.q_len)
     if w.total_tokens > 0:
         if device_kv:
             kv = sdev.kv_source(w, "cuda", cache.cu_seqlens)

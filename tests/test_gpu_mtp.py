@@ -1,0 +1,104 @@
+"""Multi-token decode (q_len 2..4 query tokens per request, causal within the draft) on the GPU:
+CUDA path through the C ABI vs the float64 oracle, per shard and merged."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_cases import D_INVARIANCE_TOL, LSE_TOL, O_TOL, assert_lse_close, assert_o_close, build_cache
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(w, D, cache, requests=None):
+    Op = cache.O_parts.cpu().numpy()
+    Lp = cache.LSE_parts.cpu().numpy()
+    O = cache.O.cpu().numpy()
+    L = cache.LSE.cpu().numpy()
+    for b in (range(w.batch) if requests is None else requests):
+        Ob, Lb, Opb, Lpb = oracle.sharded_mtp(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v,
+                                              w.queries(b), w.kv_source(b), w.softmax_scale, w.q_len,
+                                              w.block_size, D)
+        for s in range(D):
+            assert_o_close(Op[s, b], Opb[s], O_TOL, f"O_{s}[{b}]")
+            assert_lse_close(Lp[s, b], Lpb[s], LSE_TOL, f"LSE_{s}[{b}]")
+        assert_o_close(O[b], Ob, O_TOL, f"O[{b}]")
+        assert_lse_close(L[b], Lb, LSE_TOL, f"LSE[{b}]")
+
+
+# lengths: shorter than the draft, block boundaries on both sides, several pages, a few CTAs' worth
+GQA_LENS = [1, 2, 3, 16, 17, 33, 300, 1000]
+
+
+@pytest.mark.parametrize("q_len", [2, 3, 4])
+@pytest.mark.parametrize("D", [1, 3])
+def test_gqa_small_heads(q_len, D):
+    w = synth.custom(synth.GQA, GQA_LENS, 8, 2, 64, 64, 16, seed=40 + q_len, q_len=q_len)
+    cache, q = build_cache(w, D, perm_seed=D)
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, D, cache)
+    assert cache.device_error() == 0
+
+
+@pytest.mark.parametrize("q_len", [2, 4])
+def test_gqa_70b_heads(q_len):
+    # G = 8: q_len 2 fills one 16-row tile per KV head, q_len 4 takes two tiles (two warps per head)
+    w = synth.custom(synth.GQA, [5, 129, 2000, 4097], 64, 8, 128, 128, 16, seed=7 * q_len, q_len=q_len,
+                     kv_amp=0.5)
+    cache, q = build_cache(w, 4)
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, 4, cache)
+
+
+def test_gqa_sixteen_heads_per_kv_head():
+    # G = 16, q_len 4: 64 rows per KV head, four row tiles
+    w = synth.custom(synth.GQA, [4, 70, 513], 32, 2, 128, 128, 32, seed=5, q_len=4)
+    cache, q = build_cache(w, 2)
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, 2, cache)
+
+
+@pytest.mark.parametrize("q_len", [2, 4])
+@pytest.mark.parametrize("D", [1, 2])
+def test_mla(q_len, D):
+    w = synth.custom(synth.MLA, [1, 3, 64, 65, 130, 700], 64, 1, 576, 512, 64, seed=60 + q_len, q_len=q_len)
+    cache, q = build_cache(w, D)
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, D, cache)
+    assert cache.device_error() == 0
+
+
+@pytest.mark.parametrize("layout", [synth.GQA, synth.MLA])
+def test_last_draft_token_is_single_token_decode(layout):
+    # the last draft token sees the whole cache: it must agree with a q_len = 1 call on that token
+    shape = (16, 2, 128, 128, 16) if layout == synth.GQA else (64, 1, 576, 512, 64)
+    lens = [37, 500, 1200]
+    wm = synth.custom(layout, lens, *shape, seed=9, q_len=3)
+    cm, qm = build_cache(wm, 2)
+    cm.step(qm)
+    c1, _ = build_cache(synth.custom(layout, lens, *shape, seed=9), 2)
+    q_last = qm[:, 2].contiguous()
+    c1.step(q_last)
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(cm.O[:, 2].cpu().numpy(), c1.O.cpu().numpy(), rtol=0, atol=D_INVARIANCE_TOL)
+    np.testing.assert_allclose(cm.LSE[:, 2].cpu().numpy(), c1.LSE.cpu().numpy(), rtol=0, atol=D_INVARIANCE_TOL)
+
+
+@pytest.mark.parametrize("layout", [synth.GQA, synth.MLA])
+def test_d_invariance(layout):
+    shape = (8, 2, 64, 64, 16) if layout == synth.GQA else (64, 1, 576, 512, 64)
+    w = synth.custom(layout, [3, 150, 2100], *shape, seed=12, q_len=4)
+    outs = []
+    for D in (1, 2, 4):
+        cache, q = build_cache(w, D)
+        cache.step(q)
+        outs.append((cache.O.cpu().numpy(), cache.LSE.cpu().numpy()))
+    for O, L in outs[1:]:
+        np.testing.assert_allclose(O, outs[0][0], rtol=0, atol=D_INVARIANCE_TOL)
+        np.testing.assert_allclose(L, outs[0][1], rtol=0, atol=D_INVARIANCE_TOL)
+

@@ -156,3 +156,21 @@ def test_grow_errors_leave_tables_untouched():
         dcp.dcp_grow_block_table([0], [16 * 7], 16, 2, t, l, nxt, [9, 9])  # local block 3 >= 3
     assert e.value.status == dcp.DCP_ERR_CAPACITY
     assert (t == -1).all() and (l == 0).all() and (nxt == 0).all()
+
+
+def test_q_len_validation_and_workspace_growth():
+    # q_len outside 1..4 is refused; a multi-token workspace holds q_len times the rows
+    for ql in (0, 5, -1):
+        desc = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 4, 0.125, ql)
+        assert dcp.dcp_decode_workspace_bytes(desc, 2) == 0
+    base = dcp.dcp_decode_workspace_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 4, 8, 2, 64, 64, 16, 4, 0.125, 1), 2)
+    multi = dcp.dcp_decode_workspace_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 4, 8, 2, 64, 64, 16, 4, 0.125, 4), 2)
+    assert base > 0 and multi > base
+    mla = dcp.dcp_decode_workspace_bytes(dcp.make_desc(dcp.DCP_LAYOUT_MLA, 4, 64, 1, 576, 512, 64, 4, 0.07, 3), 2)
+    assert mla > 0
+
+
+def test_descriptor_layout_matches_header():
+    import ctypes
+    assert ctypes.sizeof(dcp.dcp_attn_desc) == 10 * 4
+    assert dcp.dcp_attn_desc.q_len.offset == 36

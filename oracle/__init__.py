@@ -58,6 +58,20 @@ def _load():
             lib.oracle_attend.restype = None
             lib.oracle_attend.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, C.c_int64, p,
                                           C.c_double, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, p]
+            lib.oracle_attend_f64.restype = None
+            lib.oracle_attend_f64.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, C.c_int64, p,
+                                              C.c_double, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, p]
+            lib.oracle_e4m3_decode.restype = C.c_double
+            lib.oracle_e4m3_decode.argtypes = [C.c_uint8]
+            lib.oracle_e4m3_encode.restype = C.c_uint8
+            lib.oracle_e4m3_encode.argtypes = [C.c_double]
+            lib.oracle_quantize_e4m3.restype = None
+            lib.oracle_quantize_e4m3.argtypes = [p, C.c_int64, C.c_float, p]
+            lib.oracle_dequantize_e4m3.restype = None
+            lib.oracle_dequantize_e4m3.argtypes = [p, C.c_int64, C.c_double, p]
+            lib.oracle_place_request_u8.restype = None
+            lib.oracle_place_request_u8.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                    p, C.c_int64, p, p]
             lib.oracle_merge.restype = None
             lib.oracle_merge.argtypes = [p, p, C.c_int, C.c_int64, C.c_int, p, p]
             lib.oracle_merge_ml.restype = None
@@ -151,6 +165,95 @@ def attend(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, s
     _load().oracle_attend(layout, Hq, Hkv, d_qk, d_v, _ptr(q), src.shape[0], _ptr(src), scale, block_size, D,
                           shard, hb, he, _ptr(O), _ptr(LSE))
     return O, LSE
+
+
+def attend_values(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray,
+                  scale: float, block_size: int = 1, D: int = 1, shard: int = -1,
+                  heads: Optional[Tuple[int, int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """``attend`` with the key/value source given as float64 values (same row layout)."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    src = np.ascontiguousarray(src, dtype=np.float64)
+    hb, he = heads if heads is not None else (0, Hq)
+    O = np.full((Hq, d_v), np.nan)
+    LSE = np.full((Hq,), np.nan)
+    _load().oracle_attend_f64(layout, Hq, Hkv, d_qk, d_v, _ptr(q), src.shape[0], _ptr(src), scale, block_size, D,
+                              shard, hb, he, _ptr(O), _ptr(LSE))
+    return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) KV cache
+# ---------------------------------------------------------------------------
+def e4m3_decode(codes) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    return np.array([_load().oracle_e4m3_decode(int(x)) for x in c.ravel()]).reshape(c.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float64)
+    return np.array([_load().oracle_e4m3_encode(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def inv_scale(scale: float) -> np.float32:
+    """float32 of 1 / scale (how the cache write turns a scale into a multiplier)."""
+    return np.float32(1.0) / np.float32(scale)
+
+
+def quantize_e4m3(bits: np.ndarray, scale: float) -> np.ndarray:
+    """bf16 bit patterns -> E4M3 codes of float32(x) * float32(1 / scale)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(b.shape, dtype=np.uint8)
+    _load().oracle_quantize_e4m3(_ptr(b), b.size, float(inv_scale(scale)), _ptr(out))
+    return out
+
+
+def dequantize_e4m3(codes: np.ndarray, scale: float) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    _load().oracle_dequantize_e4m3(_ptr(c), c.size, float(np.float32(scale)), _ptr(out))
+    return out
+
+
+def quantize_kv_gqa(src: np.ndarray, k_scale: float, v_scale: float) -> np.ndarray:
+    """GQA source rows [n][2][Hkv][d] (bf16 bits) -> E4M3 codes, K with k_scale and V with v_scale."""
+    codes = np.empty(src.shape, dtype=np.uint8)
+    codes[:, 0] = quantize_e4m3(src[:, 0], k_scale)
+    codes[:, 1] = quantize_e4m3(src[:, 1], v_scale)
+    return codes
+
+
+def dequantize_kv_gqa(codes: np.ndarray, k_scale: float, v_scale: float) -> np.ndarray:
+    """The float64 values an FP8 GQA cache stands for: [n][2][Hkv][d]."""
+    out = np.empty(codes.shape, dtype=np.float64)
+    out[:, 0] = dequantize_e4m3(codes[:, 0], k_scale)
+    out[:, 1] = dequantize_e4m3(codes[:, 1], v_scale)
+    return out
+
+
+def place_u8(Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray, codes: List[np.ndarray],
+             num_pages: np.ndarray, fill: int = 0xFF) -> List[np.ndarray]:
+    """Reference placement of quantised GQA rows: D byte pools, unused bytes set to ``fill``."""
+    B = len(codes)
+    mlb = tables.shape[2]
+    page = 2 * Hkv * block_size * d
+    pools = [np.full(int(num_pages[s]) * page, fill, dtype=np.uint8) for s in range(D)]
+    arr = (C.c_void_p * D)(*[p.ctypes.data for p in pools])
+    t = np.ascontiguousarray(tables, dtype=np.int32)
+    for b, c in enumerate(codes):
+        c = np.ascontiguousarray(c, dtype=np.uint8)
+        _load().oracle_place_request_u8(Hkv, d, block_size, D, B, b, mlb, _ptr(t), c.shape[0], _ptr(c),
+                                        C.cast(arr, C.c_void_p))
+    return pools
+
+
+def sharded_values(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray,
+                   scale: float, block_size: int, D: int):
+    """``sharded`` over a float64-valued source (e.g. a dequantised FP8 cache)."""
+    parts = [attend_values(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s) for s in range(D)]
+    Op = np.stack([p[0] for p in parts])
+    Lp = np.stack([p[1] for p in parts])
+    O, LSE = merge(Op, Lp)
+    return O, LSE, Op, Lp
 
 
 def merge(O_parts: np.ndarray, LSE_parts: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:

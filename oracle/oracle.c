@@ -216,9 +216,9 @@ void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int
  * Heads are computed for h in [h_begin, h_end); outputs are indexed by the
  * absolute head: O[h][d_v], LSE[h].
  */
-void oracle_attend(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
-                   const uint16_t *src, double scale, int block_size, int D, int shard, int h_begin, int h_end,
-                   double *O, double *LSE) {
+void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
+                       const double *src, double scale, int block_size, int D, int shard, int h_begin, int h_end,
+                       double *O, double *LSE) {
     double *s = (double *)malloc((size_t)(n_tok > 0 ? n_tok : 1) * sizeof(double));
     double *qd = (double *)malloc((size_t)d_qk * sizeof(double));
     int group = (layout == OR_GQA) ? Hq / Hkv : Hq;
@@ -229,10 +229,10 @@ void oracle_attend(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_
         int64_t count = 0;
         for (int64_t t = 0; t < n_tok; ++t) {
             if (shard >= 0 && oracle_token_shard(t, block_size, D) != shard) continue;
-            const uint16_t *krow = (layout == OR_GQA) ? src + ((t * 2 + 0) * Hkv + kvh) * (int64_t)d_qk
-                                                      : src + t * (int64_t)d_qk;
+            const double *krow = (layout == OR_GQA) ? src + ((t * 2 + 0) * Hkv + kvh) * (int64_t)d_qk
+                                                    : src + t * (int64_t)d_qk;
             double acc = 0.0;
-            for (int k = 0; k < d_qk; ++k) acc += qd[k] * bf16_to_double(krow[k]);
+            for (int k = 0; k < d_qk; ++k) acc += qd[k] * krow[k];
             s[t] = scale * acc;
             if (s[t] > M) M = s[t];
             ++count;
@@ -246,17 +246,110 @@ void oracle_attend(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_
         double Z = 0.0;
         for (int64_t t = 0; t < n_tok; ++t) {
             if (shard >= 0 && oracle_token_shard(t, block_size, D) != shard) continue;
-            const uint16_t *vrow = (layout == OR_GQA) ? src + ((t * 2 + 1) * Hkv + kvh) * (int64_t)d_qk
-                                                      : src + t * (int64_t)d_qk;
+            const double *vrow = (layout == OR_GQA) ? src + ((t * 2 + 1) * Hkv + kvh) * (int64_t)d_qk
+                                                    : src + t * (int64_t)d_qk;
             double w = exp(s[t] - M);
             Z += w;
-            for (int k = 0; k < d_v; ++k) o[k] += w * bf16_to_double(vrow[k]);
+            for (int k = 0; k < d_v; ++k) o[k] += w * vrow[k];
         }
         for (int k = 0; k < d_v; ++k) o[k] /= Z;
         LSE[h] = M + log(Z);
     }
     free(qd);
     free(s);
+}
+
+/* The same attention with the key/value source given as bf16 bit patterns
+ * (widened exactly to double first). */
+void oracle_attend(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
+                   const uint16_t *src, double scale, int block_size, int D, int shard, int h_begin, int h_end,
+                   double *O, double *LSE) {
+    int64_t row = (layout == OR_GQA) ? 2 * (int64_t)Hkv * d_qk : d_qk;
+    int64_t n = n_tok * row;
+    double *wide = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    for (int64_t i = 0; i < n; ++i) wide[i] = bf16_to_double(src[i]);
+    oracle_attend_f64(layout, Hq, Hkv, d_qk, d_v, q, n_tok, wide, scale, block_size, D, shard, h_begin, h_end, O,
+                      LSE);
+    free(wide);
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 KV cache: E4M3 codes with a per-tensor scale                    */
+/* ------------------------------------------------------------------ */
+
+/*
+ * The FP8 E4M3 format (the OCP 8-bit floating-point specification's E4M3,
+ * "fn" variant): bit 7 sign, bits 6..3 exponent e (bias 7), bits 2..0
+ * mantissa m.  e = 0: subnormal, value m/8 * 2^-6; e = 1..15: (1 + m/8) *
+ * 2^(e-7), except e = 15, m = 7 which is NaN.  No infinities; the largest
+ * finite magnitude is 448 (e = 15, m = 6).
+ */
+double oracle_e4m3_decode(uint8_t c) {
+    int sign = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/*
+ * Nearest E4M3 code to x, ties to the even code (even mantissa), magnitudes
+ * above 448 saturated to +-448 (the "satfinite" rule); NaN -> 0x7F.  Found by
+ * scanning the 127 non-negative finite codes, which are increasing in value.
+ */
+uint8_t oracle_e4m3_encode(double x) {
+    if (x != x) return 0x7F;
+    uint8_t sign = (x < 0.0 || (x == 0.0 && signbit(x))) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int best = 0;
+    for (int c = 1; c <= 0x7E; ++c) {
+        double dc = fabs(oracle_e4m3_decode((uint8_t)c) - a), db = fabs(oracle_e4m3_decode((uint8_t)best) - a);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+    }
+    return (uint8_t)(sign | best);
+}
+
+/*
+ * Quantisation of bf16 cache values to E4M3 codes with a per-tensor scale:
+ * code = e4m3(float32(x) * inv_scale), the product rounded to float32 first
+ * (the decision is taken in the kernel's precision), inv_scale = float32 of
+ * 1 / scale.  The value a code stands for is scale * e4m3_value(code).
+ */
+void oracle_quantize_e4m3(const uint16_t *src, int64_t n, float inv_scale, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) {
+        float x = (float)bf16_to_double(src[i]);
+        float p = x * inv_scale;
+        out[i] = oracle_e4m3_encode((double)p);
+    }
+}
+
+/* scale * value(code) for n codes (exact in double). */
+void oracle_dequantize_e4m3(const uint8_t *codes, int64_t n, double scale, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = scale * oracle_e4m3_decode(codes[i]);
+}
+
+/*
+ * Placement of one request's quantised GQA rows (codes [n_tok][2][Hkv][d],
+ * one byte per element) into byte pools whose pages are [2][Hkv][bs][d]:
+ * the same token walk as oracle_place_request, one byte per element.
+ */
+void oracle_place_request_u8(int Hkv, int d, int block_size, int D, int B, int b, int max_local_blocks,
+                             const int32_t *tables, int64_t n_tok, const uint8_t *src, uint8_t **pools) {
+    for (int64_t t = 0; t < n_tok; ++t) {
+        int s = oracle_token_shard(t, block_size, D);
+        int64_t j = oracle_token_local_block(t, block_size, D);
+        int64_t page = tables[((int64_t)s * B + b) * max_local_blocks + j];
+        int64_t slot = t % block_size;
+        for (int kv = 0; kv < 2; ++kv)
+            for (int h = 0; h < Hkv; ++h)
+                for (int k = 0; k < d; ++k)
+                    pools[s][(((page * 2 + kv) * Hkv + h) * block_size + slot) * d + k] =
+                        src[((t * 2 + kv) * Hkv + h) * d + k];
+    }
 }
 
 /* ------------------------------------------------------------------ */

@@ -456,3 +456,92 @@ def test_mtp_short_sequence_sees_nothing():
 def test_queries_extend_the_single_token_query():
     w = synth.custom(MLA, [5], 64, 1, 576, 512, 64, seed=8, q_len=3)
     np.testing.assert_array_equal(w.queries(0)[0], w.query(0))
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) cache: code definition, rounding, scales, placement
+# ---------------------------------------------------------------------------
+def test_e4m3_values_from_the_format_definition():
+    # sign | exponent (bias 7) | mantissa: hand-decoded codes
+    cases = {0x38: 1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x40: 2.0,
+             0x3C: 1.5, 0x30: 0.5, 0xB8: -1.0, 0x00: 0.0, 0x77: 240.0, 0x7D: 416.0}
+    for c, v in cases.items():
+        assert oracle.e4m3_decode(np.array([c], np.uint8))[0] == v, hex(c)
+    assert np.isnan(oracle.e4m3_decode(np.array([0x7F, 0xFF], np.uint8))).all()
+    z = oracle.e4m3_decode(np.array([0x80], np.uint8))[0]
+    assert z == 0.0 and math.copysign(1.0, z) == -1.0
+
+
+def test_e4m3_decode_matches_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ours)
+    np.testing.assert_array_equal(ours[ok], ref[ok])
+
+
+def test_e4m3_encode_matches_torch_float8_in_range():
+    # torch's float32 -> float8_e4m3fn cast rounds to nearest even; within +-448 it must agree
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.normal(0, 1, 4000), rng.normal(0, 60, 2000), rng.uniform(-448, 448, 2000),
+                        rng.normal(0, 2.0 ** -8, 2000)]).astype(np.float32)
+    vals = oracle.e4m3_decode(np.arange(127, dtype=np.uint8)).astype(np.float32)
+    mids = ((vals[:-1].astype(np.float64) + vals[1:]) / 2).astype(np.float32)  # exact ties
+    x = np.concatenate([x, mids, -mids, vals, -vals])
+    ours = oracle.e4m3_encode(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_e4m3_saturates_and_ties_to_even():
+    assert list(oracle.e4m3_encode([449.0, 1e6, -1e6, 464.0, 447.0])) == [0x7E, 0x7E, 0xFE, 0x7E, 0x7E]
+    # halfway between 1.0 (0x38, even) and 1.125 (0x39): to 0x38; between 1.125 and 1.25: to 0x3A
+    assert list(oracle.e4m3_encode([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10])) == [0x38, 0x3A, 0x00, 0x02]
+
+
+def test_quantize_rounds_the_product_in_float32_then_to_e4m3():
+    w = synth.custom(GQA, [300], 8, 2, 64, 64, 16, seed=19, kv_amp=0.5)
+    src = w.kv_source(0)
+    for scale in (1.0, 0.75, 1.0 / 64, 3.3):
+        codes = oracle.quantize_e4m3(src, scale)
+        prod = synth.bf16_bits_to_f64(src).astype(np.float32) * oracle.inv_scale(scale)
+        np.testing.assert_array_equal(codes, oracle.e4m3_encode(prod.astype(np.float64)))
+        # dequantised values are within half a unit of the third mantissa bit (relative 2^-4)
+        back = oracle.dequantize_e4m3(codes, scale)
+        x = synth.bf16_bits_to_f64(src)
+        big = np.abs(x / scale) >= 2.0 ** -6
+        assert (np.abs(back[big] - x[big]) <= 2.0 ** -4 * np.abs(x[big]) * (1 + 1e-6)).all()
+
+
+def test_quantize_roundtrips_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF, 0x80)], dtype=np.uint8)
+    vals = oracle.e4m3_decode(codes)
+    bits = synth.f32_to_bf16_bits(vals.astype(np.float32))  # E4M3 values are exact in bf16
+    np.testing.assert_array_equal(oracle.quantize_e4m3(bits, 1.0), codes)
+
+
+def test_attend_values_equals_attend_on_widened_bf16():
+    w = synth.custom(GQA, [90], 8, 2, 64, 64, 16, seed=23)
+    q, src = w.query(0), w.kv_source(0)
+    for D, s in [(1, -1), (3, 1)]:
+        a = oracle.attend(GQA, 8, 2, 64, 64, q, src, 0.125, 16, D, s)
+        b = oracle.attend_values(GQA, 8, 2, 64, 64, q, synth.bf16_bits_to_f64(src), 0.125, 16, D, s)
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_fp8_placement_roundtrip():
+    w = synth.custom(GQA, [70, 5, 33], 8, 2, 128, 128, 16, seed=4)
+    D = 3
+    tables, _, pages = oracle.block_tables(w.seq_lens, 16, D)
+    codes = [oracle.quantize_kv_gqa(w.kv_source(b), 1.0, 0.5) for b in range(w.batch)]
+    pools = oracle.place_u8(2, 128, 16, D, tables, codes, pages, fill=0x7F)
+    for b in range(w.batch):
+        for t in range(w.seq_lens[b]):
+            s, j = oracle.token_shard(t, 16, D), oracle.token_local_block(t, 16, D)
+            page = tables[s, b, j]
+            pg = pools[s][page * 2 * 2 * 16 * 128:(page + 1) * 2 * 2 * 16 * 128].reshape(2, 2, 16, 128)
+            np.testing.assert_array_equal(pg[:, :, t % 16], codes[b][t])
+    used = sum(int(w.seq_lens[b]) for b in range(w.batch)) * 2 * 2 * 128
+    assert sum(int((p != 0x7F).sum()) for p in pools) <= used

@@ -50,6 +50,10 @@ def parse(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline time budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="query tokens per request (multi-token decode, causal within the draft; 1..4)")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="cache element type (fp8: E4M3 codes, per-tensor scales 2^-7; GQA head_dim 128)")
     ap.add_argument("--batch-limit", type=int, default=None,
                     help="keep only the first N requests (small cases for profiling)")
     return ap.parse_args(argv)
@@ -176,17 +180,31 @@ def load_workload(args):
         w.seq_lens = w.seq_lens[:args.batch_limit]
         w.batch = args.batch_limit
         w.name = f"{w.name}[:{args.batch_limit}]"
+    if args.q_len != 1:
+        w.q_len = args.q_len
+        w.name = f"{w.name} q_len={args.q_len}"
+    w.extra["kv_dtype"] = args.kv_dtype
+    if args.kv_dtype == "fp8":
+        w.name = f"{w.name} fp8"
     return w
+
+
+FP8_SCALE = 2.0 ** -7  # per-tensor K and V scale of the FP8 cache: |x| <= 3.5 maps inside E4M3's 448
+
+
+def cache_elem_bytes(w) -> int:
+    return 1 if w.extra.get("kv_dtype") == "fp8" else 2
 
 
 def tensor_figures(w, decode_ms: float, peaks: dict, peaks_kind: str):
     """Tensor-pipe side of the roofline: the method's flops per launch vs the dense bf16 peak.
 
-    Per context token and query head: 2*d_qk (q.k) + 2*d_v (p*v) flops."""
-    flops = w.total_tokens * w.num_q_heads * 2 * (w.head_dim_qk + w.head_dim_v)
+    Per context token, query token and query head: 2*d_qk (q.k) + 2*d_v (p*v) flops (the few
+    draft tokens a causal row does not see are not subtracted)."""
+    flops = w.total_tokens * w.q_len * w.num_q_heads * 2 * (w.head_dim_qk + w.head_dim_v)
     tf = flops / decode_ms / 1e9
     peak = peaks["bf16_tflops"]
-    bytes_time = w.total_tokens * w.kv_bytes_per_token / (peaks["hbm_gbs"] * 1e9)
+    bytes_time = w.total_tokens * w.kv_bytes_per_token * cache_elem_bytes(w) / 2 / (peaks["hbm_gbs"] * 1e9)
     flop_time = flops / (peak * 1e12)
     return {"flops_per_launch": flops, "achieved_tflops": round(tf, 1), "peak_tflops": peak,
             "frac": round(tf / peak, 4), "peak_kind": f"{peaks_kind} dense bf16 (burst)",
@@ -196,8 +214,8 @@ def tensor_figures(w, decode_ms: float, peaks: dict, peaks_kind: str):
 
 def algorithmic_bytes(w, D: int):
     """(KV bytes, decode-kernel bytes, merge bytes) the method must move per step."""
-    rows = w.batch * w.num_q_heads
-    kv = w.total_tokens * w.kv_bytes_per_token
+    rows = w.batch * w.q_len * w.num_q_heads
+    kv = w.total_tokens * w.kv_bytes_per_token * cache_elem_bytes(w) // 2
     q = rows * w.head_dim_qk * 2
     partial_out = rows * (w.head_dim_v + 1) * 4
     decode = kv + D * q + D * partial_out
@@ -265,7 +283,9 @@ def run_ours(args, rank, world, local):
 
     def build(Dx):
         cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v,
-                                  w.block_size, Dx, w.seq_lens, w.softmax_scale, device=dev)
+                                  w.block_size, Dx, w.seq_lens, w.softmax_scale, device=dev, q_len=w.q_len,
+                                  kv_dtype=1 if cache_elem_bytes(w) == 1 else 0, k_scale=FP8_SCALE,
+                                  v_scale=FP8_SCALE)
         kv = sdev.kv_source(w, dev, cache.cu_seqlens)
         cache.place(kv)
         del kv
@@ -336,15 +356,28 @@ def run_ours(args, rank, world, local):
     kv_row = torch.zeros((w.batch, row_elems), dtype=torch.int16, device=dev)
     cu_rows = torch.arange(w.batch + 1, dtype=torch.int64, device=dev)
     last_pos = (cache.seq_lens_dev - 1).clamp_min(0).contiguous()
-    for _ in range(3):
-        dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools, cache.pool_pages)
+    # 20 appends captured in one CUDA graph, so the events time the kernels, not the host calls
+    side = torch.cuda.Stream(dev)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
+                              cache.pool_pages, stream=side)
+    side.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for _ in range(20):
+            dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
+                              cache.pool_pages, stream=side)
+    graph.replay()
+    torch.cuda.synchronize()
     a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a0.record()
-    for _ in range(20):
-        dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools, cache.pool_pages)
+    for _ in range(5):
+        graph.replay()
     a1.record()
     torch.cuda.synchronize()
-    append_ms = a0.elapsed_time(a1) / 20
+    append_ms = a0.elapsed_time(a1) / 100
+    del graph
 
     kv_b, dec_b, mrg_b = algorithmic_bytes(w, D)
     step_ms_max = reduce_max(step_ms, world, dev)
@@ -384,9 +417,9 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if cache_elem_bytes(w) == 2 else "fp8-e4m3 cache, f16 products, f32 accumulate",
         "data": "synthetic",
-        "config": {"workload": f"{w.name}: {w.note}", "D": D, "batch": w.batch,
+        "config": {"workload": f"{w.name}: {w.note}", "D": D, "batch": w.batch, "q_len": w.q_len,
                    "context_tokens": w.total_tokens, "kv_bytes_per_step": kv_b,
                    "l2": "flushed before every step (write of 2x L2), outside the timed events",
                    "parallelism": "replicas" if world > 1 else "single GPU (D shard pools in one HBM)"},
@@ -400,8 +433,9 @@ def run_ours(args, rank, world, local):
         "merge_kernel_us": round(merge_ms_max * 1e3, 2),
         "merge_gbs": round(mrg_b / merge_ms_max / 1e6, 1),
         "append_kernel_us": round(append_ms_max * 1e3, 2),
-        "append_bytes_per_step": 2 * w.batch * w.kv_bytes_per_token,
+        "append_bytes_per_step": w.batch * w.kv_bytes_per_token * (2 + cache_elem_bytes(w)) // 2,
         "context_tokens_per_s": round(world * w.total_tokens / step_ms_max * 1e3, 1),
+        "query_tokens_per_s": round(world * w.batch * w.q_len / step_ms_max * 1e3, 1),
         "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
         "tensor": tensor_figures(w, part_ms_max, peaks, peaks_kind),
         "median_step_ms": round(step_med, 4),
@@ -413,7 +447,7 @@ def run_ours(args, rank, world, local):
                                                 "overlapped with neighbouring steps)"},
         "other_D": other,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and w.q_len == 1 and cache_elem_bytes(w) == 2:
         gbs, secs, desc = cpu_baseline(w, D, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                 "sample": desc, "seconds": round(secs, 2)}

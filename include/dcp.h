@@ -44,6 +44,7 @@
  *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.
  *       Multi-token decode: 1 <= q_len <= 4 query tokens per request
  *       (GQA and MLA).
+ *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA with head_dim 128 only.
  */
 #ifndef DCP_H
 #define DCP_H
@@ -76,6 +77,27 @@ typedef enum dcp_layout {
 } dcp_layout;
 
 /*
+ * Element type of the KV cache pools.  [P3 §7: an FP8 KV cache complements
+ * DCP by shrinking the cache further; the page does not fix a format.]
+ *   DCP_KV_BF16      bf16 values.
+ *   DCP_KV_FP8_E4M3  one byte per value: an E4M3 code (the OCP FP8 E4M3 "fn"
+ *                    format: bias 7, no infinities, largest finite 448) and a
+ *                    per-tensor scale, value = scale * e4m3(code); K uses
+ *                    k_scale, V uses v_scale.  The cache writes quantise bf16
+ *                    rows as code = e4m3_rn_satfinite(float32(x) * inv), inv =
+ *                    float32(1 / scale): the product rounded to float32, then to
+ *                    the nearest code (ties to even), magnitudes past 448
+ *                    saturated.  The decode kernel feeds the codes (exact in
+ *                    f16) and the query converted to f16 to f16 tensor-core
+ *                    products; query elements outside f16's normal range
+ *                    (|q| > 65504 or |q| < 2^-14) lose precision there.
+ */
+typedef enum dcp_kv_dtype {
+    DCP_KV_BF16 = 0,
+    DCP_KV_FP8_E4M3 = 1
+} dcp_kv_dtype;
+
+/*
  * Problem description shared by the decode calls.
  *   layout           dcp_layout.
  *   batch            B, number of requests (q_len decode tokens each).
@@ -94,6 +116,8 @@ typedef enum dcp_layout {
  *                    (0-based) attends the tokens t < seq_len - (q_len - 1 - j), i.e.
  *                    causally within the draft.  A query token with no visible token in a
  *                    shard gets O = 0, LSE = -inf there.
+ *   kv_dtype         dcp_kv_dtype of the pools.
+ *   k_scale, v_scale per-tensor scales of an FP8 cache (positive, finite); ignored for bf16.
  */
 typedef struct dcp_attn_desc {
     int32_t layout;
@@ -106,6 +130,9 @@ typedef struct dcp_attn_desc {
     int32_t max_local_blocks;
     float softmax_scale;
     int32_t q_len;
+    int32_t kv_dtype;
+    float k_scale;
+    float v_scale;
 } dcp_attn_desc;
 
 /* Library version, major * 10000 + minor * 100 + patch. */
@@ -147,7 +174,8 @@ DCP_API dcp_status dcp_build_block_table(const int32_t *seq_lens, int32_t batch,
                                  uint64_t perm_seed, int32_t max_local_blocks, int32_t *tables,
                                  int32_t *local_len);
 
-/* Bytes of one KV page for `desc` (GQA: 2*Hkv*block_size*head_dim*2; MLA: block_size*576*2); 0 if invalid. */
+/* Bytes of one KV page for `desc` (GQA: 2*Hkv*block_size*head_dim*e; MLA: block_size*576*2; e = 2 for
+ * bf16, 1 for FP8); 0 if invalid. */
 DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
 
 /*
@@ -160,7 +188,8 @@ DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
  *   tables      host array of D device pointers, each int32[batch][max_local_blocks]
  *               (as built by dcp_build_block_table).
  *   kv_pools    host array of D device pointers; pool s holds pool_pages[s] pages:
- *               GQA page [2 (K,V)][Hkv][block_size][head_dim] bf16;
+ *               GQA page [2 (K,V)][Hkv][block_size][head_dim] of the pool's
+ *               kv_dtype (bf16, or FP8 codes quantised on the way in);
  *               MLA page [block_size][576] bf16.
  *   pool_pages  host int32[D].
  *   device_error optional device int32 (may be NULL): set to 1 if a table entry

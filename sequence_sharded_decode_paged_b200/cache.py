@@ -20,7 +20,8 @@ from . import dcp
 class ShardedPagedCache:
     def __init__(self, layout: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
                  block_size: int, D: int, seq_lens: Sequence[int], softmax_scale: float, perm_seed: int = 0,
-                 device="cuda", pool_fill: Optional[int] = None, q_len: int = 1):
+                 device="cuda", pool_fill: Optional[int] = None, q_len: int = 1, kv_dtype: int = 0,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
         self.D = D
         self.q_len = q_len
         self.device = torch.device(device)
@@ -32,7 +33,8 @@ class ShardedPagedCache:
         self.tables_host, self.local_len = dcp.dcp_build_block_table(self.seq_lens, block_size, D, perm_seed,
                                                                      self.max_local_blocks)
         self.desc = dcp.make_desc(layout, self.batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v,
-                                  block_size, self.max_local_blocks, softmax_scale, q_len)
+                                  block_size, self.max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale,
+                                  v_scale)
         self.page_bytes = dcp.dcp_kv_page_bytes(self.desc)
         if self.page_bytes == 0:
             raise ValueError("unsupported attention shape")
@@ -94,7 +96,8 @@ class ShardedPagedCache:
     def kv_bytes(self) -> int:
         """KV bytes the method reads per step (tokens x bytes per token; padding excluded)."""
         d = self.desc
-        per = 2 * d.num_kv_heads * d.head_dim_qk * 2 if d.layout == dcp.DCP_LAYOUT_GQA else d.head_dim_qk * 2
+        eb = 1 if d.kv_dtype == dcp.DCP_KV_FP8_E4M3 else 2
+        per = 2 * d.num_kv_heads * d.head_dim_qk * eb if d.layout == dcp.DCP_LAYOUT_GQA else d.head_dim_qk * 2
         return int(sum(self.seq_lens)) * per
 
 

@@ -6,6 +6,7 @@
 // to shard g % D as local block g / D, so shard s holds
 // nloc(s) = nblk > s ? (nblk - 1 - s) / D + 1 : 0 blocks, all full except the
 // request's last block when that one falls in shard s.
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -54,14 +55,14 @@ static EncodeTiledFn encode_fn() {
 }
 
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return CUDA_ERROR_NOT_SUPPORTED;
   cuuint64_t dims[2] = {inner_elems, rows};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
@@ -72,8 +73,13 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
       d.max_local_blocks < 1 || d.head_dim_qk < 1 || d.head_dim_v < 1 || !(d.softmax_scale == d.softmax_scale) ||
       d.q_len < 1)
     return false;
+  if (d.kv_dtype != DCP_KV_BF16 && d.kv_dtype != DCP_KV_FP8_E4M3) return false;
+  if (d.kv_dtype == DCP_KV_FP8_E4M3 &&
+      !(d.k_scale > 0.f && d.k_scale < INFINITY && d.v_scale > 0.f && d.v_scale < INFINITY))
+    return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.q_len > kMaxQLen) return false;
+  if (d.kv_dtype == DCP_KV_FP8_E4M3 && (d.layout != DCP_LAYOUT_GQA || d.head_dim_qk != 128)) return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.layout == DCP_LAYOUT_GQA) {
     if (d.head_dim_qk != d.head_dim_v || (d.head_dim_qk != 64 && d.head_dim_qk != 128)) return false;
@@ -97,7 +103,8 @@ bool workspace_layout(const dcp_attn_desc& d, int D, WorkspaceLayout* L) {
   const int sms = device_sm_count();
   if (d.layout == DCP_LAYOUT_GQA) {
     const int G = d.num_q_heads / d.num_kv_heads;
-    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size, d.head_dim_qk, gqa_row_tiles(G, d.q_len));
+    const int hpc = gqa_heads_per_cta(d.num_kv_heads, d.block_size, d.head_dim_qk, gqa_row_tiles(G, d.q_len),
+                                      kv_elem_bytes(d));
     L->n_hg = d.num_kv_heads / hpc;
     L->rows_per_hg = hpc * G * d.q_len;
     L->nctas = sms / L->n_hg > 0 ? sms / L->n_hg : 1;
@@ -216,7 +223,7 @@ size_t dcp_kv_page_bytes(const dcp_attn_desc* desc) {
   if (d.max_local_blocks < 1) d.max_local_blocks = 1;
   dcp_status why;
   if (!desc_supported(d, 1, &why)) return 0;
-  if (d.layout == DCP_LAYOUT_GQA) return (size_t)2 * d.num_kv_heads * d.block_size * d.head_dim_qk * 2;
+  if (d.layout == DCP_LAYOUT_GQA) return (size_t)2 * d.num_kv_heads * d.block_size * d.head_dim_qk * kv_elem_bytes(d);
   return (size_t)d.block_size * d.head_dim_qk * 2;
 }
 
@@ -234,7 +241,7 @@ dcp_status dcp_place_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_src
     if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
   }
   if ((reinterpret_cast<uintptr_t>(kv_src) & 15u) != 0) return DCP_ERR_INVALID_ARG;
-  return launch_place_kv(*desc, D, kv_src, cu_seqlens, nullptr, tables, kv_pools, pool_pages, device_error,
+  return launch_place_kv(*desc, D, kv_src, cu_seqlens, nullptr, tables, kv_pools, pool_pages, device_error, false,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -287,7 +294,7 @@ dcp_status dcp_append_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_ne
     if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
   }
   if ((reinterpret_cast<uintptr_t>(kv_new) & 15u) != 0) return DCP_ERR_INVALID_ARG;
-  return launch_place_kv(*desc, D, kv_new, cu_rows, first_pos, tables, kv_pools, pool_pages, device_error,
+  return launch_place_kv(*desc, D, kv_new, cu_rows, first_pos, tables, kv_pools, pool_pages, device_error, true,
                          static_cast<cudaStream_t>(stream));
 }
 

@@ -24,6 +24,18 @@
 //    the V fragments, so stale cache contents (even NaN) never leak in.
 //  * Multi-token decode (q_len > 1): row r sees only the tokens before
 //    seq_len - (q_len - 1 - r / G); the rest of its scores are masked.
+//  * FP8 cache (KV8, head_dim 128): pages hold E4M3 codes, a 128-byte row per
+//    token and head, so one swizzled box carries a head's K (or V) block and a
+//    stage is half the size.  Codes convert exactly to f16 and the products
+//    run as f16 mma.  K: each lane reads 4 consecutive codes of a token with
+//    one 32-bit load; the query's dimensions are permuted the same way inside
+//    each 16-wide k-tile (dims 4c..4c+3 play k = 2c, 2c+1, 2c+8, 2c+9).  V:
+//    each lane reads 16 codes (dims 16g..16g+15) of tokens 2c, 2c+1, 2c+8 and
+//    2c+9 with 16-byte loads and pairs them by byte permutes, so n-tile nt,
+//    column n stands for dim 16n + nt; the output store undoes that order.
+//    k_scale is folded into the score scale and v_scale into the final
+//    normalisation.  The K products of a chunk run as four independent chains
+//    (two token halves x two k halves) so that their latencies overlap.
 #include <float.h>
 
 #include "dcp_device.cuh"
@@ -49,6 +61,7 @@ struct GqaParams {
   int* counters;
   float* slots;
   float scale_log2;
+  float v_scale;  // multiplies O (FP8 cache); 1 for bf16
   int n_si, B, Hq, Hkv, G, bs, D, mlb;
   int q_len, R, rt;  // query tokens per request, rows per KV head (q_len * G), 16-row tiles per head
   int hpc, n_hg, stages, wph;
@@ -63,9 +76,11 @@ __device__ __forceinline__ size_t gqa_out_row(int rr, int b, int ql, int Hq, int
   return ((size_t)b * ql + jq) * Hq + (size_t)(kv0 + h) * G + (r - jq * G);
 }
 
-template <int HEAD_DIM>
+template <int HEAD_DIM, bool KV8>
 struct GqaGeom {
-  static constexpr int kBoxes = HEAD_DIM / 64;  // 64-element (128-byte) swizzled boxes per row
+  // 128-byte swizzled boxes per row: 64 bf16 or 128 FP8 codes each
+  static constexpr int kBoxes = KV8 ? HEAD_DIM / 128 : HEAD_DIM / 64;
+  static constexpr int kBoxElems = KV8 ? 128 : 64;
   static constexpr int kNTiles = HEAD_DIM / 8;  // n-tiles of O
   static constexpr int kKTiles = HEAD_DIM / 16; // k-tiles of Q K^T
   static constexpr int kCombineFloats = kNTiles * 4 + 4;  // per lane per warp
@@ -73,9 +88,11 @@ struct GqaGeom {
 
 // MULTI: multi-token decode (q_len > 1, per-row causal limits); the single-token
 // instantiation keeps the plain end-of-sequence mask and its register budget.
-template <int HEAD_DIM, bool MULTI>
+// KV8: the pools hold FP8 E4M3 codes.
+template <int HEAD_DIM, bool MULTI, bool KV8>
 __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid_constant__ GqaParams p) {
-  using Geo = GqaGeom<HEAD_DIM>;
+  using Geo = GqaGeom<HEAD_DIM, KV8>;
+  static_assert(!KV8 || HEAD_DIM == 128, "FP8 pages use one 128-byte row per token and head");
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stage_mem = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * p.stage_bytes);
@@ -142,8 +159,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           const int row_v = ((page * 2 + 1) * p.Hkv + hg * p.hpc) * bs;
 #pragma unroll
           for (int bx = 0; bx < Geo::kBoxes; ++bx) {
-            tma_load_2d(dst + bx * box_bytes, &p.tmap[si], bx * 64, row_k, &full[stage]);
-            tma_load_2d(dst + (Geo::kBoxes + bx) * box_bytes, &p.tmap[si], bx * 64, row_v, &full[stage]);
+            tma_load_2d(dst + bx * box_bytes, &p.tmap[si], bx * Geo::kBoxElems, row_k, &full[stage]);
+            tma_load_2d(dst + (Geo::kBoxes + bx) * box_bytes, &p.tmap[si], bx * Geo::kBoxElems, row_v,
+                        &full[stage]);
           }
         } else {
           mbar_arrive(&full[stage]);
@@ -211,13 +229,27 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       const size_t q1 = (((size_t)b * ql + j1) * p.Hq + (size_t)kvh * G + (r1 - j1 * G)) * HEAD_DIM;
       const uint32_t* qb0 = reinterpret_cast<const uint32_t*>(p.q + (row0 ? q0 : 0));
       const uint32_t* qb1 = reinterpret_cast<const uint32_t*>(p.q + (row1 ? q1 : 0));
+      if constexpr (KV8) {
+        // f16 query, dims 16kt + 4c .. 4c+3 in the k slots 2c, 2c+1 (a0/a1) and 2c+8, 2c+9 (a2/a3)
 #pragma unroll
-      for (int kt = 0; kt < Geo::kKTiles; ++kt) {
-        const int col = kt * 16 + c4 * 2;
-        qa[kt][0] = row0 ? __ldg(qb0 + col / 2) : 0u;
-        qa[kt][1] = row1 ? __ldg(qb1 + col / 2) : 0u;
-        qa[kt][2] = row0 ? __ldg(qb0 + (col + 8) / 2) : 0u;
-        qa[kt][3] = row1 ? __ldg(qb1 + (col + 8) / 2) : 0u;
+        for (int kt = 0; kt < Geo::kKTiles; ++kt) {
+          const int col = kt * 16 + c4 * 4;
+          const uint2 x0 = row0 ? __ldg(reinterpret_cast<const uint2*>(qb0 + col / 2)) : make_uint2(0u, 0u);
+          const uint2 x1 = row1 ? __ldg(reinterpret_cast<const uint2*>(qb1 + col / 2)) : make_uint2(0u, 0u);
+          qa[kt][0] = bf16x2_to_f16x2(x0.x);
+          qa[kt][1] = bf16x2_to_f16x2(x1.x);
+          qa[kt][2] = bf16x2_to_f16x2(x0.y);
+          qa[kt][3] = bf16x2_to_f16x2(x1.y);
+        }
+      } else {
+#pragma unroll
+        for (int kt = 0; kt < Geo::kKTiles; ++kt) {
+          const int col = kt * 16 + c4 * 2;
+          qa[kt][0] = row0 ? __ldg(qb0 + col / 2) : 0u;
+          qa[kt][1] = row1 ? __ldg(qb1 + col / 2) : 0u;
+          qa[kt][2] = row0 ? __ldg(qb0 + (col + 8) / 2) : 0u;
+          qa[kt][3] = row1 ? __ldg(qb1 + (col + 8) / 2) : 0u;
+        }
       }
       if (MULTI) {  // up to the row's own draft position
         lim0 = seq_len - (ql - 1 - j0);
@@ -247,14 +279,41 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
         for (int t0 = 0; t0 < valid; t0 += 16) {
           // ---- S = Q K^T for 16 tokens (two 8-token n-tiles)
           float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-          const uint32_t krow = (uint32_t)(hh * bs + t0 + (lane & 7) + ((lane >> 4) << 3));
+          if constexpr (KV8) {
+            // lane (g, c) needs codes 4c..4c+3 of k-tile kt of tokens g and 8 + g: one ldmatrix
+            // (8 x 16-byte rows per matrix) gives exactly that word for four (token half, k-tile)
+            // pairs -- matrices: tokens 0-7 / 8-15 of k-tiles kt and kt + 1
+            const uint32_t lrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
+            float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // odd k-tiles
 #pragma unroll
-          for (int kt = 0; kt < Geo::kKTiles; ++kt) {
-            const uint32_t chunk = (uint32_t)((kt & 3) * 2 + ((lane >> 3) & 1));
-            uint32_t b00, b01, b10, b11;
-            ldsm_x4(kbase + (kt >> 2) * box_bytes + sw128(krow, chunk), b00, b01, b10, b11);
-            mma_bf16_16816(s[0], qa[kt], b00, b01);
-            mma_bf16_16816(s[1], qa[kt], b10, b11);
+            for (int kt = 0; kt < Geo::kKTiles; kt += 2) {
+              uint32_t w0, w1, w2, w3;  // (tokens 0-7, kt), (8-15, kt), (0-7, kt+1), (8-15, kt+1)
+              ldsm_x4(kbase + sw128(lrow, (uint32_t)(kt + (lane >> 4))), w0, w1, w2, w3);
+              uint32_t k0[2], k1[2], k2[2], k3[2];
+              e4m3x4_to_f16x2x2(w0, k0[0], k0[1]);
+              e4m3x4_to_f16x2x2(w1, k1[0], k1[1]);
+              e4m3x4_to_f16x2x2(w2, k2[0], k2[1]);
+              e4m3x4_to_f16x2x2(w3, k3[0], k3[1]);
+              mma_f16_16816(s[0], qa[kt], k0[0], k0[1]);
+              mma_f16_16816(s[1], qa[kt], k1[0], k1[1]);
+              mma_f16_16816(s2[0], qa[kt + 1], k2[0], k2[1]);
+              mma_f16_16816(s2[1], qa[kt + 1], k3[0], k3[1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              s[0][i] += s2[0][i];
+              s[1][i] += s2[1][i];
+            }
+          } else {
+            const uint32_t krow = (uint32_t)(hh * bs + t0 + (lane & 7) + ((lane >> 4) << 3));
+#pragma unroll
+            for (int kt = 0; kt < Geo::kKTiles; ++kt) {
+              const uint32_t chunk = (uint32_t)((kt & 3) * 2 + ((lane >> 3) & 1));
+              uint32_t b00, b01, b10, b11;
+              ldsm_x4(kbase + (kt >> 2) * box_bytes + sw128(krow, chunk), b00, b01, b10, b11);
+              mma_bf16_16816(s[0], qa[kt], b00, b01);
+              mma_bf16_16816(s[1], qa[kt], b10, b11);
+            }
           }
           // ---- online softmax (log2 domain), rows g4 and g4 + 8
           const int vrem = valid - t0;
@@ -291,23 +350,60 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           }
           l0 = l0 * al0 + (s[0][0] + s[0][1] + s[1][0] + s[1][1]);
           l1 = l1 * al1 + (s[0][2] + s[0][3] + s[1][2] + s[1][3]);
+          // the integral maximum rarely moves, so the rescale is usually a multiply by 1: skip it then
+          if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-          for (int i = 0; i < Geo::kNTiles; ++i) {
-            o[i][0] *= al0;
-            o[i][1] *= al0;
-            o[i][2] *= al1;
-            o[i][3] *= al1;
+            for (int i = 0; i < Geo::kNTiles; ++i) {
+              o[i][0] *= al0;
+              o[i][1] *= al0;
+              o[i][2] *= al1;
+              o[i][3] *= al1;
+            }
           }
           uint32_t pa[4];
-          pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-          pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-          pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-          pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+          if constexpr (KV8) {
+            pa[0] = pack_f16x2(s[0][0], s[0][1]);
+            pa[1] = pack_f16x2(s[0][2], s[0][3]);
+            pa[2] = pack_f16x2(s[1][0], s[1][1]);
+            pa[3] = pack_f16x2(s[1][2], s[1][3]);
+          } else {
+            pa[0] = pack_bf16x2(s[0][0], s[0][1]);
+            pa[1] = pack_bf16x2(s[0][2], s[0][3]);
+            pa[2] = pack_bf16x2(s[1][0], s[1][1]);
+            pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+          }
           // ---- O += P V; V fragments of tokens past the end are zeroed
-          const uint32_t vrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
           const bool tail = vrem < 16;
           const uint32_t keep0 = (c4 * 2 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 1 < vrem ? 0xFFFF0000u : 0u);
           const uint32_t keep1 = (c4 * 2 + 8 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 9 < vrem ? 0xFFFF0000u : 0u);
+          if constexpr (KV8) {
+            // codes of dims 16g..16g+15 for tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1)
+            const uint32_t vr = (uint32_t)(hh * bs + t0 + 2 * c4);
+            const uint4 ta = lds128(vbase + sw128(vr, (uint32_t)g4));
+            const uint4 tb = lds128(vbase + sw128(vr + 1u, (uint32_t)g4));
+            const uint4 tc = lds128(vbase + sw128(vr + 8u, (uint32_t)g4));
+            const uint4 td = lds128(vbase + sw128(vr + 9u, (uint32_t)g4));
+            const uint32_t xa[4] = {ta.x, ta.y, ta.z, ta.w}, xb[4] = {tb.x, tb.y, tb.z, tb.w};
+            const uint32_t xc[4] = {tc.x, tc.y, tc.z, tc.w}, xd[4] = {td.x, td.y, td.z, td.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              // byte k of word w is dim 16g + 4w + k, i.e. n-tile 4w + k: pair the two tokens' codes
+              uint32_t b0[4], b1[4];
+              e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x5140), b0[0], b0[1]);
+              e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x7362), b0[2], b0[3]);
+              e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x5140), b1[0], b1[1]);
+              e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x7362), b1[2], b1[3]);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                if (tail) {
+                  b0[k] &= keep0;
+                  b1[k] &= keep1;
+                }
+                mma_f16_16816(o[4 * w + k], pa, b0[k], b1[k]);
+              }
+            }
+          } else {
+          const uint32_t vrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
 #pragma unroll
           for (int np = 0; np < Geo::kNTiles / 2; ++np) {
             const uint32_t chunk = (uint32_t)((np & 3) * 2 + (lane >> 4));
@@ -321,6 +417,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
             }
             mma_bf16_16816(o[2 * np], pa, v0, v1);
             mma_bf16_16816(o[2 * np + 1], pa, v2, v3);
+          }
           }
         }
       }
@@ -381,7 +478,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       // base-2 log-sum-exp of each row; empty state (all pages skipped) -> -inf
       const float lse0 = l0 > 0.f ? m0 + __log2f(l0) : -INFINITY;
       const float lse1 = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
-      const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const float inv0 = l0 > 0.f ? p.v_scale / l0 : 0.f, inv1 = l1 > 0.f ? p.v_scale / l1 : 0.f;
       // destination rows: the outputs, or this CTA's slot (rows in head-group order)
       float* Obase = p.O[si];
       float* Lbase = p.LSE[si];
@@ -393,17 +490,41 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       float* dO1 = complete ? Obase + out_row(hh * R + r1) * HEAD_DIM : sl + (size_t)(hh * R + r1) * HEAD_DIM;
       float* dL0 = complete ? Lbase + out_row(hh * R + r0) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r0;
       float* dL1 = complete ? Lbase + out_row(hh * R + r1) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r1;
-      if (row0) {
+      if constexpr (KV8) {
+        // n-tile i, column 2c (+1) holds dim 32c + i (+16): two runs of 16 consecutive dims
+        if (row0) {
 #pragma unroll
-        for (int i = 0; i < Geo::kNTiles; ++i)
-          *reinterpret_cast<float2*>(dO0 + i * 8 + c4 * 2) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
-        if (c4 == 0) *dL0 = complete ? lse0 * kLn2 : lse0;
-      }
-      if (row1) {
+          for (int i = 0; i < Geo::kNTiles; i += 4) {
+            *reinterpret_cast<float4*>(dO0 + 32 * c4 + i) =
+                make_float4(o[i][0] * inv0, o[i + 1][0] * inv0, o[i + 2][0] * inv0, o[i + 3][0] * inv0);
+            *reinterpret_cast<float4*>(dO0 + 32 * c4 + 16 + i) =
+                make_float4(o[i][1] * inv0, o[i + 1][1] * inv0, o[i + 2][1] * inv0, o[i + 3][1] * inv0);
+          }
+          if (c4 == 0) *dL0 = complete ? lse0 * kLn2 : lse0;
+        }
+        if (row1) {
 #pragma unroll
-        for (int i = 0; i < Geo::kNTiles; ++i)
-          *reinterpret_cast<float2*>(dO1 + i * 8 + c4 * 2) = make_float2(o[i][2] * inv1, o[i][3] * inv1);
-        if (c4 == 0) *dL1 = complete ? lse1 * kLn2 : lse1;
+          for (int i = 0; i < Geo::kNTiles; i += 4) {
+            *reinterpret_cast<float4*>(dO1 + 32 * c4 + i) =
+                make_float4(o[i][2] * inv1, o[i + 1][2] * inv1, o[i + 2][2] * inv1, o[i + 3][2] * inv1);
+            *reinterpret_cast<float4*>(dO1 + 32 * c4 + 16 + i) =
+                make_float4(o[i][3] * inv1, o[i + 1][3] * inv1, o[i + 2][3] * inv1, o[i + 3][3] * inv1);
+          }
+          if (c4 == 0) *dL1 = complete ? lse1 * kLn2 : lse1;
+        }
+      } else {
+        if (row0) {
+#pragma unroll
+          for (int i = 0; i < Geo::kNTiles; ++i)
+            *reinterpret_cast<float2*>(dO0 + i * 8 + c4 * 2) = make_float2(o[i][0] * inv0, o[i][1] * inv0);
+          if (c4 == 0) *dL0 = complete ? lse0 * kLn2 : lse0;
+        }
+        if (row1) {
+#pragma unroll
+          for (int i = 0; i < Geo::kNTiles; ++i)
+            *reinterpret_cast<float2*>(dO1 + i * 8 + c4 * 2) = make_float2(o[i][2] * inv1, o[i][3] * inv1);
+          if (c4 == 0) *dL1 = complete ? lse1 * kLn2 : lse1;
+        }
       }
     }
     if (!complete) {
@@ -460,9 +581,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
 // three or more stages fit.
 int gqa_row_tiles(int G, int q_len) { return (G * q_len + 15) / 16; }
 
-int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles) {
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles, int elem_bytes) {
   int cap = min(kGqaConsumerWarps / row_tiles, 256 / bs);
-  cap = min(cap, 65536 / (bs * head_dim * 4));
+  cap = min(cap, 65536 / (bs * head_dim * 2 * elem_bytes));
   int best = 1;
   for (int h = 1; h <= cap; ++h)
     if (Hkv % h == 0) best = h;
@@ -475,7 +596,7 @@ static int gqa_stage_count(uint32_t stage_bytes, size_t fixed_bytes) {
   return st > 8 ? 8 : st;
 }
 
-template <int HEAD_DIM, bool MULTI>
+template <int HEAD_DIM, bool MULTI, bool KV8>
 static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                                   const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
   WorkspaceLayout L;
@@ -494,16 +615,19 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.q_len = d.q_len;
   p.R = p.G * p.q_len;
   p.rt = gqa_row_tiles(p.G, p.q_len);
-  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs, HEAD_DIM, p.rt);
+  const int eb = KV8 ? 1 : 2;  // bytes per cached element
+  p.hpc = gqa_heads_per_cta(p.Hkv, p.bs, HEAD_DIM, p.rt, eb);
   p.n_hg = p.Hkv / p.hpc;
   p.wph = kGqaConsumerWarps / (p.hpc * p.rt);
-  p.stage_bytes = (uint32_t)(2 * p.hpc * p.bs * HEAD_DIM * 2);
+  p.stage_bytes = (uint32_t)(2 * p.hpc * p.bs * HEAD_DIM * eb);
   const size_t combine_bytes =
-      p.wph > 1 ? (size_t)kGqaConsumerWarps * GqaGeom<HEAD_DIM>::kCombineFloats * 32 * sizeof(float) : 0;
+      p.wph > 1 ? (size_t)kGqaConsumerWarps * GqaGeom<HEAD_DIM, KV8>::kCombineFloats * 32 * sizeof(float) : 0;
   const size_t fixed = 16 * 8 + 8 * 4 + kScratchInts * 4 + 8 * 4 + combine_bytes;
   p.stages = gqa_stage_count(p.stage_bytes, fixed);
   if (p.stages < 2) return DCP_ERR_UNSUPPORTED;
-  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  // FP8: scores carry k_scale, outputs v_scale
+  p.scale_log2 = (float)((double)d.softmax_scale * (KV8 ? (double)d.k_scale : 1.0) * 1.4426950408889634);
+  p.v_scale = KV8 ? d.v_scale : 1.f;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.seq_lens = seq_lens;
   p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
@@ -519,13 +643,13 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
     if (set.pool_pages[si] > 0) {
       const uint64_t rows = (uint64_t)set.pool_pages[si] * 2 * p.Hkv * p.bs;
       if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32
-      if (encode_tiled_2d(&p.tmap[si], set.pool[si], HEAD_DIM, rows, HEAD_DIM * 2, 64, (uint32_t)(p.hpc * p.bs)) !=
-          CUDA_SUCCESS)
+      if (encode_tiled_2d(&p.tmap[si], set.pool[si], HEAD_DIM, rows, HEAD_DIM * eb, GqaGeom<HEAD_DIM, KV8>::kBoxElems,
+                          (uint32_t)(p.hpc * p.bs), eb) != CUDA_SUCCESS)
         return DCP_ERR_CUDA;
     }
   }
   const size_t smem = (size_t)p.stages * p.stage_bytes + fixed;
-  auto kern = gqa_decode_kernel<HEAD_DIM, MULTI>;
+  auto kern = gqa_decode_kernel<HEAD_DIM, MULTI, KV8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return DCP_ERR_CUDA;
   dim3 grid(L.nctas, p.n_hg);
@@ -536,12 +660,17 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
 dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
   const bool multi = d.q_len > 1;
+  if (d.kv_dtype == DCP_KV_FP8_E4M3) {
+    if (d.head_dim_qk != 128) return DCP_ERR_UNSUPPORTED;
+    return multi ? launch_gqa_impl<128, true, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                 : launch_gqa_impl<128, false, true>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+  }
   if (d.head_dim_qk == 128)
-    return multi ? launch_gqa_impl<128, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
-                 : launch_gqa_impl<128, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+    return multi ? launch_gqa_impl<128, true, false>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                 : launch_gqa_impl<128, false, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
   if (d.head_dim_qk == 64)
-    return multi ? launch_gqa_impl<64, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
-                 : launch_gqa_impl<64, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+    return multi ? launch_gqa_impl<64, true, false>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                 : launch_gqa_impl<64, false, false>(d, D, set, q, seq_lens, ws, ws_bytes, st);
   return DCP_ERR_UNSUPPORTED;
 }
 

@@ -44,7 +44,7 @@ int device_sm_count();
 
 // cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes = 2);
 
 dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st);
@@ -54,10 +54,13 @@ dcp_status launch_lse_merge(const float* const* O_parts, const float* const* LSE
                             float* O, float* LSE_out, cudaStream_t st);
 dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, const int64_t* cu_seqlens,
                            const int32_t* token_begin, const int32_t* const* tables, void* const* pools,
-                           const int32_t* pool_pages, int32_t* device_error, cudaStream_t st);
+                           const int32_t* pool_pages, int32_t* device_error, bool few_rows, cudaStream_t st);
 
 // GQA geometry helpers (shared by the workspace sizing and the launcher).
 int gqa_row_tiles(int G, int q_len);
-int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles);
+int gqa_heads_per_cta(int Hkv, int bs, int head_dim, int row_tiles, int elem_bytes);
+
+// Bytes per cached KV element.
+inline int kv_elem_bytes(const dcp_attn_desc& d) { return d.kv_dtype == DCP_KV_FP8_E4M3 ? 1 : 2; }
 
 }  // namespace dcp

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libdcp.so")
 
 DCP_OK, DCP_ERR_INVALID_ARG, DCP_ERR_UNSUPPORTED, DCP_ERR_CAPACITY, DCP_ERR_CUDA, DCP_ERR_DEVICE = range(6)
 DCP_LAYOUT_GQA, DCP_LAYOUT_MLA = 0, 1
+DCP_KV_BF16, DCP_KV_FP8_E4M3 = 0, 1
 
 EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_build_block_table",
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
@@ -38,7 +39,7 @@ class dcp_attn_desc(C.Structure):
     _fields_ = [("layout", C.c_int32), ("batch", C.c_int32), ("num_q_heads", C.c_int32),
                 ("num_kv_heads", C.c_int32), ("head_dim_qk", C.c_int32), ("head_dim_v", C.c_int32),
                 ("block_size", C.c_int32), ("max_local_blocks", C.c_int32), ("softmax_scale", C.c_float),
-                ("q_len", C.c_int32)]
+                ("q_len", C.c_int32), ("kv_dtype", C.c_int32), ("k_scale", C.c_float), ("v_scale", C.c_float)]
 
 
 def _load() -> C.CDLL:
@@ -108,9 +109,10 @@ def _i32(a) -> np.ndarray:
 
 
 def make_desc(layout: int, batch: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
-              block_size: int, max_local_blocks: int, softmax_scale: float, q_len: int = 1) -> dcp_attn_desc:
+              block_size: int, max_local_blocks: int, softmax_scale: float, q_len: int = 1,
+              kv_dtype: int = 0, k_scale: float = 1.0, v_scale: float = 1.0) -> dcp_attn_desc:
     return dcp_attn_desc(layout, batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v, block_size,
-                         max_local_blocks, softmax_scale, q_len)
+                         max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale, v_scale)
 
 
 # --------------------------------------------------------------------------- host calls

@@ -172,5 +172,18 @@ def test_q_len_validation_and_workspace_growth():
 
 def test_descriptor_layout_matches_header():
     import ctypes
-    assert ctypes.sizeof(dcp.dcp_attn_desc) == 10 * 4
+    assert ctypes.sizeof(dcp.dcp_attn_desc) == 13 * 4
     assert dcp.dcp_attn_desc.q_len.offset == 36
+    assert dcp.dcp_attn_desc.v_scale.offset == 48
+
+
+def test_fp8_rejected_for_mla_and_head_dim_64():
+    # FP8 pools: GQA with head_dim 128 only; a page is one byte per value
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == 0
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == 0
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == \
+        2 * 2 * 16 * 128
+    for ks, vs in ((0.0, 1.0), (1.0, float("inf")), (-1.0, 1.0), (float("nan"), 1.0)):
+        assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1,
+                                                   dcp.DCP_KV_FP8_E4M3, ks, vs)) == 0
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1, 7)) == 0

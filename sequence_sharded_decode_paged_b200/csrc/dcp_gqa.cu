@@ -86,6 +86,78 @@ struct GqaGeom {
   static constexpr int kCombineFloats = kNTiles * 4 + 4;  // per lane per warp
 };
 
+// ---- FP8 building blocks: one 16-token chunk of one KV head (128 dims) ----
+// S (16 q rows x 16 tokens, f32) = Q K^T from E4M3 K rows at `kbase`, rows krow0 ..
+// krow0 + 15 of the swizzled tile.  Lane (g, c) needs codes 4c..4c+3 of k-tile kt of
+// tokens g and 8 + g: one ldmatrix (8 x 16-byte rows per matrix) gives that word for
+// four (token half, k-tile) pairs -- tokens 0-7 / 8-15 of k-tiles kt and kt + 1.  Two
+// accumulator sets (even / odd k-tiles) keep four independent product chains.
+template <int KT>
+__device__ __forceinline__ void kv8_scores(uint32_t kbase, uint32_t krow0, int lane, const uint32_t (&qa)[KT][4],
+                                           float (&s)[2][4]) {
+  const uint32_t lrow = krow0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+  float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int kt = 0; kt < KT; kt += 2) {
+    uint32_t w0, w1, w2, w3;  // (tokens 0-7, kt), (8-15, kt), (0-7, kt+1), (8-15, kt+1)
+    ldsm_x4(kbase + sw128(lrow, (uint32_t)(kt + (lane >> 4))), w0, w1, w2, w3);
+    uint32_t k0[2], k1[2], k2[2], k3[2];
+    e4m3x4_to_f16x2x2(w0, k0[0], k0[1]);
+    e4m3x4_to_f16x2x2(w1, k1[0], k1[1]);
+    e4m3x4_to_f16x2x2(w2, k2[0], k2[1]);
+    e4m3x4_to_f16x2x2(w3, k3[0], k3[1]);
+    mma_f16_16816(s[0], qa[kt], k0[0], k0[1]);
+    mma_f16_16816(s[1], qa[kt], k1[0], k1[1]);
+    mma_f16_16816(s2[0], qa[kt + 1], k2[0], k2[1]);
+    mma_f16_16816(s2[1], qa[kt + 1], k3[0], k3[1]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s[0][i] += s2[0][i];
+    s[1][i] += s2[1][i];
+  }
+}
+
+// O (16 q rows x 128 dims) += P V from E4M3 V rows at `vbase` (rows vrow0 .. vrow0 + 15).
+// Lane (g, c) reads codes of dims 16g..16g+15 of tokens 2c, 2c+1 (b0) and 2c+8, 2c+9
+// (b1) and pairs them by byte permutes, so n-tile nt, column n stands for dim 16n + nt.
+// Tokens masked by keep0 / keep1 (tail chunks) get zero values.
+template <int NT>
+__device__ __forceinline__ void kv8_pv(uint32_t vbase, uint32_t vrow0, int g4, int c4, const uint32_t (&pa)[4],
+                                       float (&o)[NT][4], bool tail, uint32_t keep0, uint32_t keep1) {
+  const uint32_t vr = vrow0 + 2u * c4;
+  const uint4 ta = lds128(vbase + sw128(vr, (uint32_t)g4));
+  const uint4 tb = lds128(vbase + sw128(vr + 1u, (uint32_t)g4));
+  const uint4 tc = lds128(vbase + sw128(vr + 8u, (uint32_t)g4));
+  const uint4 td = lds128(vbase + sw128(vr + 9u, (uint32_t)g4));
+  const uint32_t xa[4] = {ta.x, ta.y, ta.z, ta.w}, xb[4] = {tb.x, tb.y, tb.z, tb.w};
+  const uint32_t xc[4] = {tc.x, tc.y, tc.z, tc.w}, xd[4] = {td.x, td.y, td.z, td.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    // byte k of word w is dim 16g + 4w + k, i.e. n-tile 4w + k: pair the two tokens' codes
+    uint32_t b0[4], b1[4];
+    e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x5140), b0[0], b0[1]);
+    e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x7362), b0[2], b0[3]);
+    e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x5140), b1[0], b1[1]);
+    e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x7362), b1[2], b1[3]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (tail) {
+        b0[k] &= keep0;
+        b1[k] &= keep1;
+      }
+      mma_f16_16816(o[4 * w + k], pa, b0[k], b1[k]);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t keep_lo(int c4, int vrem) {  // tokens 2c, 2c+1 of a chunk
+  return (c4 * 2 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 1 < vrem ? 0xFFFF0000u : 0u);
+}
+__device__ __forceinline__ uint32_t keep_hi(int c4, int vrem) {  // tokens 2c+8, 2c+9
+  return (c4 * 2 + 8 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 9 < vrem ? 0xFFFF0000u : 0u);
+}
+
 // MULTI: multi-token decode (q_len > 1, per-row causal limits); the single-token
 // instantiation keeps the plain end-of-sequence mask and its register budget.
 // KV8: the pools hold FP8 E4M3 codes.
@@ -264,7 +336,103 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     // fp32 order); the PV product uses the same weights rounded to bf16.
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-    for (int j = a; j < e; ++j) {
+    int j = a;
+    if constexpr (KV8 && !MULTI) {
+      // FP8, one warp per head, one chunk per page: two pages per step -- four independent
+      // product chains and one softmax update per 32 tokens, to hide the latencies that
+      // leave a half-size FP8 chunk short of work
+      if (wph == 1 && bs == 16) {
+        for (; j + 1 < e; j += 2) {
+          const int st0 = stage;
+          const uint32_t ph0 = phase;
+          const int st1 = stage + 1 == p.stages ? 0 : stage + 1;
+          const uint32_t ph1 = stage + 1 == p.stages ? phase ^ 1u : phase;
+          stage = st1 + 1 == p.stages ? 0 : st1 + 1;
+          phase = st1 + 1 == p.stages ? ph1 ^ 1u : ph1;
+          if (!dead && !mbar_wait(&full[st0], ph0)) {
+            atomicOr(p.status, kDevTimeout);
+            dead = true;
+          }
+          if (!dead && !mbar_wait(&full[st1], ph1)) {
+            atomicOr(p.status, kDevTimeout);
+            dead = true;
+          }
+          if (!dead && active) {
+            const bool ok0 = stage_ok[st0] != 0, ok1 = stage_ok[st1] != 0;
+            const int v0 = min(16, seq_len - (j * D + shard) * 16);
+            const int v1 = min(16, seq_len - ((j + 1) * D + shard) * 16);
+            const uint32_t kb0 = smem_u32(stage_mem + (size_t)st0 * p.stage_bytes);
+            const uint32_t kb1 = smem_u32(stage_mem + (size_t)st1 * p.stage_bytes);
+            float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            if (ok0) kv8_scores(kb0, (uint32_t)(hh * 16), lane, qa, sa);
+            if (ok1) kv8_scores(kb1, (uint32_t)(hh * 16), lane, qa, sb);
+            const int va = ok0 ? v0 : 0, vb = ok1 ? v1 : 0;  // a page that was not loaded adds nothing
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int tok = nt * 8 + c4 * 2 + (i & 1);
+                sa[nt][i] = tok < va ? sa[nt][i] * p.scale_log2 : -INFINITY;
+                sb[nt][i] = tok < vb ? sb[nt][i] * p.scale_log2 : -INFINITY;
+              }
+            float mx0 = fmaxf(fmaxf(fmaxf(sa[0][0], sa[0][1]), fmaxf(sa[1][0], sa[1][1])),
+                              fmaxf(fmaxf(sb[0][0], sb[0][1]), fmaxf(sb[1][0], sb[1][1])));
+            float mx1 = fmaxf(fmaxf(fmaxf(sa[0][2], sa[0][3]), fmaxf(sa[1][2], sa[1][3])),
+                              fmaxf(fmaxf(sb[0][2], sb[0][3]), fmaxf(sb[1][2], sb[1][3])));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+            const float mn0 = mx0 > m0 ? ceilf(mx0) : m0, mn1 = mx1 > m1 ? ceilf(mx1) : m1;
+            const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
+            m0 = mn0;
+            m1 = mn1;
+            const float sub0 = mn0 == -INFINITY ? 0.f : mn0, sub1 = mn1 == -INFINITY ? 0.f : mn1;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              sa[nt][0] = ex2_approx(sa[nt][0] - sub0);
+              sa[nt][1] = ex2_approx(sa[nt][1] - sub0);
+              sa[nt][2] = ex2_approx(sa[nt][2] - sub1);
+              sa[nt][3] = ex2_approx(sa[nt][3] - sub1);
+              sb[nt][0] = ex2_approx(sb[nt][0] - sub0);
+              sb[nt][1] = ex2_approx(sb[nt][1] - sub0);
+              sb[nt][2] = ex2_approx(sb[nt][2] - sub1);
+              sb[nt][3] = ex2_approx(sb[nt][3] - sub1);
+            }
+            l0 = l0 * al0 + ((sa[0][0] + sa[0][1] + sa[1][0] + sa[1][1]) + (sb[0][0] + sb[0][1] + sb[1][0] + sb[1][1]));
+            l1 = l1 * al1 + ((sa[0][2] + sa[0][3] + sa[1][2] + sa[1][3]) + (sb[0][2] + sb[0][3] + sb[1][2] + sb[1][3]));
+            if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+              for (int i = 0; i < Geo::kNTiles; ++i) {
+                o[i][0] *= al0;
+                o[i][1] *= al0;
+                o[i][2] *= al1;
+                o[i][3] *= al1;
+              }
+            }
+            if (ok0) {
+              const uint32_t pa[4] = {pack_f16x2(sa[0][0], sa[0][1]), pack_f16x2(sa[0][2], sa[0][3]),
+                                      pack_f16x2(sa[1][0], sa[1][1]), pack_f16x2(sa[1][2], sa[1][3])};
+              kv8_pv(kb0 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v0 < 16, keep_lo(c4, v0),
+                     keep_hi(c4, v0));
+            }
+            if (ok1) {
+              const uint32_t pa[4] = {pack_f16x2(sb[0][0], sb[0][1]), pack_f16x2(sb[0][2], sb[0][3]),
+                                      pack_f16x2(sb[1][0], sb[1][1]), pack_f16x2(sb[1][2], sb[1][3])};
+              kv8_pv(kb1 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v1 < 16, keep_lo(c4, v1),
+                     keep_hi(c4, v1));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&empty[st0]);
+            mbar_arrive(&empty[st1]);
+          }
+        }
+      }
+    }
+    for (; j < e; ++j) {
       // a wait that times out marks this warp dead: it stops waiting and computing
       // but keeps the block-wide barrier sequence, so nothing else can hang on it
       if (!dead && !mbar_wait(&full[stage], phase)) {
@@ -280,30 +448,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           // ---- S = Q K^T for 16 tokens (two 8-token n-tiles)
           float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
           if constexpr (KV8) {
-            // lane (g, c) needs codes 4c..4c+3 of k-tile kt of tokens g and 8 + g: one ldmatrix
-            // (8 x 16-byte rows per matrix) gives exactly that word for four (token half, k-tile)
-            // pairs -- matrices: tokens 0-7 / 8-15 of k-tiles kt and kt + 1
-            const uint32_t lrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
-            float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};  // odd k-tiles
-#pragma unroll
-            for (int kt = 0; kt < Geo::kKTiles; kt += 2) {
-              uint32_t w0, w1, w2, w3;  // (tokens 0-7, kt), (8-15, kt), (0-7, kt+1), (8-15, kt+1)
-              ldsm_x4(kbase + sw128(lrow, (uint32_t)(kt + (lane >> 4))), w0, w1, w2, w3);
-              uint32_t k0[2], k1[2], k2[2], k3[2];
-              e4m3x4_to_f16x2x2(w0, k0[0], k0[1]);
-              e4m3x4_to_f16x2x2(w1, k1[0], k1[1]);
-              e4m3x4_to_f16x2x2(w2, k2[0], k2[1]);
-              e4m3x4_to_f16x2x2(w3, k3[0], k3[1]);
-              mma_f16_16816(s[0], qa[kt], k0[0], k0[1]);
-              mma_f16_16816(s[1], qa[kt], k1[0], k1[1]);
-              mma_f16_16816(s2[0], qa[kt + 1], k2[0], k2[1]);
-              mma_f16_16816(s2[1], qa[kt + 1], k3[0], k3[1]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              s[0][i] += s2[0][i];
-              s[1][i] += s2[1][i];
-            }
+            kv8_scores(kbase, (uint32_t)(hh * bs + t0), lane, qa, s);
           } else {
             const uint32_t krow = (uint32_t)(hh * bs + t0 + (lane & 7) + ((lane >> 4) << 3));
 #pragma unroll
@@ -319,13 +464,20 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           const int vrem = valid - t0;
           const int vr0 = MULTI ? lim0 - (gblk * bs + t0) : vrem;
           const int vr1 = MULTI ? lim1 - (gblk * bs + t0) : vrem;
+          if (MULTI || vrem < 16) {  // a chunk with masked tokens
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int tok = nt * 8 + c4 * 2 + (i & 1);
-              s[nt][i] = tok < (i < 2 ? vr0 : vr1) ? s[nt][i] * p.scale_log2 : -INFINITY;
-            }
+              for (int i = 0; i < 4; ++i) {
+                const int tok = nt * 8 + c4 * 2 + (i & 1);
+                s[nt][i] = tok < (i < 2 ? vr0 : vr1) ? s[nt][i] * p.scale_log2 : -INFINITY;
+              }
+          } else {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) s[nt][i] *= p.scale_log2;
+          }
           float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
           float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
           mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
@@ -343,10 +495,10 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           const float sub1 = (MULTI && mn1 == -INFINITY) ? 0.f : mn1;
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            s[nt][0] = exp2f(s[nt][0] - sub0);
-            s[nt][1] = exp2f(s[nt][1] - sub0);
-            s[nt][2] = exp2f(s[nt][2] - sub1);
-            s[nt][3] = exp2f(s[nt][3] - sub1);
+            s[nt][0] = ex2_approx(s[nt][0] - sub0);
+            s[nt][1] = ex2_approx(s[nt][1] - sub0);
+            s[nt][2] = ex2_approx(s[nt][2] - sub1);
+            s[nt][3] = ex2_approx(s[nt][3] - sub1);
           }
           l0 = l0 * al0 + (s[0][0] + s[0][1] + s[1][0] + s[1][1]);
           l1 = l1 * al1 + (s[0][2] + s[0][3] + s[1][2] + s[1][3]);
@@ -374,34 +526,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           }
           // ---- O += P V; V fragments of tokens past the end are zeroed
           const bool tail = vrem < 16;
-          const uint32_t keep0 = (c4 * 2 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 1 < vrem ? 0xFFFF0000u : 0u);
-          const uint32_t keep1 = (c4 * 2 + 8 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 9 < vrem ? 0xFFFF0000u : 0u);
+          const uint32_t keep0 = keep_lo(c4, vrem), keep1 = keep_hi(c4, vrem);
           if constexpr (KV8) {
-            // codes of dims 16g..16g+15 for tokens 2c, 2c+1 (b0) and 2c+8, 2c+9 (b1)
-            const uint32_t vr = (uint32_t)(hh * bs + t0 + 2 * c4);
-            const uint4 ta = lds128(vbase + sw128(vr, (uint32_t)g4));
-            const uint4 tb = lds128(vbase + sw128(vr + 1u, (uint32_t)g4));
-            const uint4 tc = lds128(vbase + sw128(vr + 8u, (uint32_t)g4));
-            const uint4 td = lds128(vbase + sw128(vr + 9u, (uint32_t)g4));
-            const uint32_t xa[4] = {ta.x, ta.y, ta.z, ta.w}, xb[4] = {tb.x, tb.y, tb.z, tb.w};
-            const uint32_t xc[4] = {tc.x, tc.y, tc.z, tc.w}, xd[4] = {td.x, td.y, td.z, td.w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              // byte k of word w is dim 16g + 4w + k, i.e. n-tile 4w + k: pair the two tokens' codes
-              uint32_t b0[4], b1[4];
-              e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x5140), b0[0], b0[1]);
-              e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x7362), b0[2], b0[3]);
-              e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x5140), b1[0], b1[1]);
-              e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x7362), b1[2], b1[3]);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                if (tail) {
-                  b0[k] &= keep0;
-                  b1[k] &= keep1;
-                }
-                mma_f16_16816(o[4 * w + k], pa, b0[k], b1[k]);
-              }
-            }
+            kv8_pv(vbase, (uint32_t)(hh * bs + t0), g4, c4, pa, o, tail, keep0, keep1);
           } else {
           const uint32_t vrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
 #pragma unroll

@@ -267,8 +267,9 @@ DCP_API dcp_status dcp_workspace_init(void *workspace, size_t workspace_bytes, v
  * With q_len > 1 each (request, query token j, head) row follows the same
  * formulas over the visible tokens t < seq_len - (q_len - 1 - j).
  *   workspace   device, >= dcp_decode_workspace_bytes(desc, D) bytes, initialised.
- * Page ids outside [0, pool_pages) are not read (their tokens count as zero
- * keys and values) and set the workspace status (see dcp_read_device_error).
+ * Page ids outside [0, pool_pages) are not read: their tokens are left out
+ * of the softmax, and the workspace status records the error (see
+ * dcp_read_device_error).
  */
 DCP_API dcp_status dcp_decode_partial(const dcp_attn_desc *desc, const void *q, const void *kv_pool, int32_t pool_pages,
                               const int32_t *table, const int32_t *seq_lens, int32_t shard, int32_t D, float *O_i,

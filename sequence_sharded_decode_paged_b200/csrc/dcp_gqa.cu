@@ -151,6 +151,44 @@ __device__ __forceinline__ void kv8_pv(uint32_t vbase, uint32_t vrow0, int g4, i
   }
 }
 
+// ---- bf16 building blocks: one 16-token chunk of one KV head ----
+// S = Q K^T with K fragments by ldmatrix from the 128-byte swizzled boxes (64 dims each).
+template <int KT>
+__device__ __forceinline__ void bf16_scores(uint32_t kbase, uint32_t box_bytes, uint32_t krow0, int lane,
+                                            const uint32_t (&qa)[KT][4], float (&s)[2][4]) {
+  const uint32_t krow = krow0 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) {
+    const uint32_t chunk = (uint32_t)((kt & 3) * 2 + ((lane >> 3) & 1));
+    uint32_t b00, b01, b10, b11;
+    ldsm_x4(kbase + (kt >> 2) * box_bytes + sw128(krow, chunk), b00, b01, b10, b11);
+    mma_bf16_16816(s[0], qa[kt], b00, b01);
+    mma_bf16_16816(s[1], qa[kt], b10, b11);
+  }
+}
+
+// O += P V with V fragments by ldmatrix.trans; tokens masked by keep0 / keep1 get zero values.
+template <int NT>
+__device__ __forceinline__ void bf16_pv(uint32_t vbase, uint32_t box_bytes, uint32_t vrow0, int lane,
+                                        const uint32_t (&pa)[4], float (&o)[NT][4], bool tail, uint32_t keep0,
+                                        uint32_t keep1) {
+  const uint32_t vrow = vrow0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+  for (int np = 0; np < NT / 2; ++np) {
+    const uint32_t chunk = (uint32_t)((np & 3) * 2 + (lane >> 4));
+    uint32_t v0, v1, v2, v3;
+    ldsm_x4_t(vbase + (np >> 2) * box_bytes + sw128(vrow, chunk), v0, v1, v2, v3);
+    if (tail) {
+      v0 &= keep0;
+      v1 &= keep1;
+      v2 &= keep0;
+      v3 &= keep1;
+    }
+    mma_bf16_16816(o[2 * np], pa, v0, v1);
+    mma_bf16_16816(o[2 * np + 1], pa, v2, v3);
+  }
+}
+
 __device__ __forceinline__ uint32_t keep_lo(int c4, int vrem) {  // tokens 2c, 2c+1 of a chunk
   return (c4 * 2 < vrem ? 0xFFFFu : 0u) | (c4 * 2 + 1 < vrem ? 0xFFFF0000u : 0u);
 }
@@ -337,10 +375,12 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
     int j = a;
-    if constexpr (KV8 && !MULTI) {
-      // FP8, one warp per head, one chunk per page: two pages per step -- four independent
-      // product chains and one softmax update per 32 tokens, to hide the latencies that
-      // leave a half-size FP8 chunk short of work
+    if constexpr (KV8 || MULTI) {
+      // One warp per (head, row tile) and one chunk per page: two pages per step -- four
+      // independent product chains and one softmax update per 32 tokens.  This hides the
+      // latencies that leave a warp short of work when its chunk carries few bytes (FP8) or
+      // its CTA streams few heads (several row tiles per head); single-token bf16 is HBM-bound
+      // without it.
       if (wph == 1 && bs == 16) {
         for (; j + 1 < e; j += 2) {
           const int st0 = stage;
@@ -365,16 +405,24 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
             const uint32_t kb1 = smem_u32(stage_mem + (size_t)st1 * p.stage_bytes);
             float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
             float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            if (ok0) kv8_scores(kb0, (uint32_t)(hh * 16), lane, qa, sa);
-            if (ok1) kv8_scores(kb1, (uint32_t)(hh * 16), lane, qa, sb);
-            const int va = ok0 ? v0 : 0, vb = ok1 ? v1 : 0;  // a page that was not loaded adds nothing
+            if constexpr (KV8) {
+              if (ok0) kv8_scores(kb0, (uint32_t)(hh * 16), lane, qa, sa);
+              if (ok1) kv8_scores(kb1, (uint32_t)(hh * 16), lane, qa, sb);
+            } else {
+              if (ok0) bf16_scores(kb0, box_bytes, (uint32_t)(hh * 16), lane, qa, sa);
+              if (ok1) bf16_scores(kb1, box_bytes, (uint32_t)(hh * 16), lane, qa, sb);
+            }
+            // visible tokens of each page for rows g4 / g4 + 8 (a page that was not loaded adds nothing)
+            const int t0a = (j * D + shard) * 16, t0b = ((j + 1) * D + shard) * 16;
+            const int va0 = !ok0 ? 0 : (MULTI ? lim0 - t0a : v0), va1 = !ok0 ? 0 : (MULTI ? lim1 - t0a : v0);
+            const int vb0 = !ok1 ? 0 : (MULTI ? lim0 - t0b : v1), vb1 = !ok1 ? 0 : (MULTI ? lim1 - t0b : v1);
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const int tok = nt * 8 + c4 * 2 + (i & 1);
-                sa[nt][i] = tok < va ? sa[nt][i] * p.scale_log2 : -INFINITY;
-                sb[nt][i] = tok < vb ? sb[nt][i] * p.scale_log2 : -INFINITY;
+                sa[nt][i] = tok < (i < 2 ? va0 : va1) ? sa[nt][i] * p.scale_log2 : -INFINITY;
+                sb[nt][i] = tok < (i < 2 ? vb0 : vb1) ? sb[nt][i] * p.scale_log2 : -INFINITY;
               }
             float mx0 = fmaxf(fmaxf(fmaxf(sa[0][0], sa[0][1]), fmaxf(sa[1][0], sa[1][1])),
                               fmaxf(fmaxf(sb[0][0], sb[0][1]), fmaxf(sb[1][0], sb[1][1])));
@@ -411,17 +459,33 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
                 o[i][3] *= al1;
               }
             }
+            // values of tokens past the sequence end are zeroed (stale slots); causal masking
+            // within the sequence is carried by P = 0
             if (ok0) {
-              const uint32_t pa[4] = {pack_f16x2(sa[0][0], sa[0][1]), pack_f16x2(sa[0][2], sa[0][3]),
-                                      pack_f16x2(sa[1][0], sa[1][1]), pack_f16x2(sa[1][2], sa[1][3])};
-              kv8_pv(kb0 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v0 < 16, keep_lo(c4, v0),
-                     keep_hi(c4, v0));
+              if constexpr (KV8) {
+                const uint32_t pa[4] = {pack_f16x2(sa[0][0], sa[0][1]), pack_f16x2(sa[0][2], sa[0][3]),
+                                        pack_f16x2(sa[1][0], sa[1][1]), pack_f16x2(sa[1][2], sa[1][3])};
+                kv8_pv(kb0 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v0 < 16, keep_lo(c4, v0),
+                       keep_hi(c4, v0));
+              } else {
+                const uint32_t pa[4] = {pack_bf16x2(sa[0][0], sa[0][1]), pack_bf16x2(sa[0][2], sa[0][3]),
+                                        pack_bf16x2(sa[1][0], sa[1][1]), pack_bf16x2(sa[1][2], sa[1][3])};
+                bf16_pv(kb0 + Geo::kBoxes * box_bytes, box_bytes, (uint32_t)(hh * 16), lane, pa, o, v0 < 16,
+                        keep_lo(c4, v0), keep_hi(c4, v0));
+              }
             }
             if (ok1) {
-              const uint32_t pa[4] = {pack_f16x2(sb[0][0], sb[0][1]), pack_f16x2(sb[0][2], sb[0][3]),
-                                      pack_f16x2(sb[1][0], sb[1][1]), pack_f16x2(sb[1][2], sb[1][3])};
-              kv8_pv(kb1 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v1 < 16, keep_lo(c4, v1),
-                     keep_hi(c4, v1));
+              if constexpr (KV8) {
+                const uint32_t pa[4] = {pack_f16x2(sb[0][0], sb[0][1]), pack_f16x2(sb[0][2], sb[0][3]),
+                                        pack_f16x2(sb[1][0], sb[1][1]), pack_f16x2(sb[1][2], sb[1][3])};
+                kv8_pv(kb1 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v1 < 16, keep_lo(c4, v1),
+                       keep_hi(c4, v1));
+              } else {
+                const uint32_t pa[4] = {pack_bf16x2(sb[0][0], sb[0][1]), pack_bf16x2(sb[0][2], sb[0][3]),
+                                        pack_bf16x2(sb[1][0], sb[1][1]), pack_bf16x2(sb[1][2], sb[1][3])};
+                bf16_pv(kb1 + Geo::kBoxes * box_bytes, box_bytes, (uint32_t)(hh * 16), lane, pa, o, v1 < 16,
+                        keep_lo(c4, v1), keep_hi(c4, v1));
+              }
             }
           }
           __syncwarp();
@@ -450,15 +514,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           if constexpr (KV8) {
             kv8_scores(kbase, (uint32_t)(hh * bs + t0), lane, qa, s);
           } else {
-            const uint32_t krow = (uint32_t)(hh * bs + t0 + (lane & 7) + ((lane >> 4) << 3));
-#pragma unroll
-            for (int kt = 0; kt < Geo::kKTiles; ++kt) {
-              const uint32_t chunk = (uint32_t)((kt & 3) * 2 + ((lane >> 3) & 1));
-              uint32_t b00, b01, b10, b11;
-              ldsm_x4(kbase + (kt >> 2) * box_bytes + sw128(krow, chunk), b00, b01, b10, b11);
-              mma_bf16_16816(s[0], qa[kt], b00, b01);
-              mma_bf16_16816(s[1], qa[kt], b10, b11);
-            }
+            bf16_scores(kbase, box_bytes, (uint32_t)(hh * bs + t0), lane, qa, s);
           }
           // ---- online softmax (log2 domain), rows g4 and g4 + 8
           const int vrem = valid - t0;
@@ -530,21 +586,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           if constexpr (KV8) {
             kv8_pv(vbase, (uint32_t)(hh * bs + t0), g4, c4, pa, o, tail, keep0, keep1);
           } else {
-          const uint32_t vrow = (uint32_t)(hh * bs + t0 + (lane & 7) + (((lane >> 3) & 1) << 3));
-#pragma unroll
-          for (int np = 0; np < Geo::kNTiles / 2; ++np) {
-            const uint32_t chunk = (uint32_t)((np & 3) * 2 + (lane >> 4));
-            uint32_t v0, v1, v2, v3;
-            ldsm_x4_t(vbase + (np >> 2) * box_bytes + sw128(vrow, chunk), v0, v1, v2, v3);
-            if (tail) {
-              v0 &= keep0;
-              v1 &= keep1;
-              v2 &= keep0;
-              v3 &= keep1;
-            }
-            mma_bf16_16816(o[2 * np], pa, v0, v1);
-            mma_bf16_16816(o[2 * np + 1], pa, v2, v3);
-          }
+            bf16_pv(vbase, box_bytes, (uint32_t)(hh * bs + t0), lane, pa, o, tail, keep0, keep1);
           }
         }
       }

@@ -146,12 +146,12 @@ def test_append_writes_the_same_codes_as_placement():
 
 
 
-@pytest.mark.parametrize("D", [1, 2, 3])
-def test_two_pages_per_step_path(D):
-    # eight KV heads at block 16 (one warp per head, one chunk per page): pages go two at a time,
-    # odd page counts leave a single page, partial last pages and one-token requests included
+@pytest.mark.parametrize("D,q_len", [(1, 1), (2, 1), (3, 1), (3, 2), (2, 4)])
+def test_two_pages_per_step_path(D, q_len):
+    # eight KV heads at block 16 (one warp per head and row tile, one chunk per page): pages go two
+    # at a time, odd page counts leave a single page, partial last pages and one-token requests included
     w = synth.custom(synth.GQA, [1, 16, 17, 31, 32, 33, 48, 500, 1111], 64, 8, 128, 128, 16, seed=17 + D,
-                     kv_amp=0.5)
+                     kv_amp=0.5, q_len=q_len)
     cache, q = _cache(w, D, 0.01, 0.01)
     cache.step(q)
     torch.cuda.synchronize()

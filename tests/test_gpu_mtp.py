@@ -53,6 +53,19 @@ def test_gqa_70b_heads(q_len):
     _check(w, 4, cache)
 
 
+@pytest.mark.parametrize("q_len", [2, 3, 4])
+def test_gqa_two_pages_per_step(q_len):
+    # 8 KV heads, block 16: one warp per (head, row tile), pages taken two at a time; the draft
+    # straddles page boundaries and odd page counts leave a single page
+    w = synth.custom(synth.GQA, [1, 2, 16, 17, 18, 33, 47, 300, 1001], 64, 8, 128, 128, 16, seed=70 + q_len,
+                     q_len=q_len, kv_amp=0.5)
+    for D in (1, 3):
+        cache, q = build_cache(w, D)
+        cache.step(q)
+        torch.cuda.synchronize()
+        _check(w, D, cache)
+
+
 def test_gqa_sixteen_heads_per_kv_head():
     # G = 16, q_len 4: 64 rows per KV head, four row tiles
     w = synth.custom(synth.GQA, [4, 70, 513], 32, 2, 128, 128, 32, seed=5, q_len=4)

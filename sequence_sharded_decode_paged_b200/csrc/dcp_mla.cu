@@ -23,7 +23,9 @@
 //                     two 64-column TMEM buffers (head h in lane h%16 + 32*(h/16)).
 //      O^T += V^T P^T: M=128 (value dims, four tiles) N=64 (heads) K=64 tokens;
 //                     V^T is read straight from the latent tile as an MN-major
-//                     operand, P^T from a 64 x 64 bf16 tile the softmax writes.
+//                     operand, P^T from a 64 x 64 bf16 tile the softmax writes
+//                     into the page's own rope box (dead after QK^T), so the
+//                     softmax of a page never waits for the previous PV product.
 //    S of page i+1 is issued before O of page i, so the tensor pipe works while
 //    the softmax runs.
 //  * Warps 2-5: softmax (four threads per head row of S), fp32, base-2; the
@@ -59,9 +61,10 @@ constexpr uint32_t kBlockBytes = 8192;                // 64 rows x 64 bf16, 128-
 constexpr uint32_t kTileBytes = 9 * kBlockBytes;      // 64 rows x 576 bf16
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffKV = kTileBytes;               // two stages
-constexpr uint32_t kOffP = 3 * kTileBytes;            // P^T tile: 64 heads x 64 tokens bf16
-constexpr uint32_t kOffMisc = kOffP + kBlockBytes;
-constexpr uint32_t kMlaSmem = kOffMisc + 3072;  // 232,448 bytes: the sm_100 per-block maximum
+// P^T (64 heads x 64 tokens bf16, 8 KB) of a page lives in its stage's rope box (dims 512-575 of
+// the latent tile), which only QK^T reads: no separate buffer.
+constexpr uint32_t kOffMisc = 3 * kTileBytes;
+constexpr uint32_t kMlaSmem = kOffMisc + 3072;  // 224,256 bytes
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                         // O^T: 4 tiles x 64 columns
 constexpr uint32_t kColS = 256;                       // S: 2 buffers x 64 columns
@@ -212,19 +215,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           const bool ok = page_ok(p, si, b, j, &page);
           if (!ok) atomicOr(p.status, kDevBadPage);
           uint8_t* dst = smem + kOffKV + st * kTileBytes;
-          // box groups in the order they are freed: rope box, value boxes 0-3, value boxes 4-7
-          for (int g = 0; g < 3 && !dead; ++g) {
+          // box groups in the order they are freed: value boxes 0-3, value boxes 4-7, rope box
+          // (the rope box holds the page's P^T tile until its PV product is done)
+          for (int gi = 0; gi < 3 && !dead; ++gi) {
+            const int g = gi == 2 ? 0 : gi + 1;
             wait_or_die(&misc->kv_empty[st][g], kv_ph ^ 1u, dead, p.status);
             if (dead) break;
             if (ok) {
+              if (gi == 0) mbar_arrive_expect_tx(&misc->kv_full[st], kTileBytes);
               if (g == 0) {
-                mbar_arrive_expect_tx(&misc->kv_full[st], kTileBytes);
                 tma_load_2d(dst + 8 * kBlockBytes, &p.kvmap[si], 8 * 64, page * kMlaBs, &misc->kv_full[st]);
               } else {
                 for (int cb = 4 * (g - 1); cb < 4 * g; ++cb)
                   tma_load_2d(dst + cb * kBlockBytes, &p.kvmap[si], cb * 64, page * kMlaBs, &misc->kv_full[st]);
               }
-            } else if (g == 2) {
+            } else if (gi == 2) {
               mbar_arrive(&misc->kv_full[st]);
             }
           }
@@ -258,7 +263,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(64, 64, false, false);
       const uint32_t idO = idesc_bf16_f32(128, 64, true, false);
-      const uint32_t qa = smem_u32(smem + kOffQ), pa = smem_u32(smem + kOffP);
+      const uint32_t qa = smem_u32(smem + kOffQ);
       struct PageRec {
         bool ok, seg_first, seg_last;
       };
@@ -311,7 +316,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           const uint32_t ost = (uint32_t)(jo & 1);
           if (r.ok && !dead) {
             const uint64_t ad = sw128_desc(smem_u32(smem + kOffKV + ost * kTileBytes), kBlockBytes, 1024);
-            const uint64_t bd = sw128_desc(pa, 16, 1024);
+            // P^T of this page sits in its stage's rope box (free once QK^T of the page is done)
+            const uint64_t bd = sw128_desc(smem_u32(smem + kOffKV + ost * kTileBytes + 8 * kBlockBytes), 16, 1024);
 #pragma unroll
             for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
@@ -325,6 +331,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             umma_commit(&misc->kv_empty[ost][1]);
           }
           umma_commit(&misc->kv_empty[ost][2]);  // value boxes 4-7 are free
+          umma_commit(&misc->kv_empty[ost][0]);  // the rope box (P^T) is free
           umma_commit(&misc->o_done);
           ++jo;
           progressed = true;
@@ -349,7 +356,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               }
             }
             umma_commit(&misc->s_full[st]);
-            umma_commit(&misc->kv_empty[st][0]);           // the rope box is read by QK^T only
             if (r.seg_last) umma_commit(&misc->q_empty);  // Q is free once these S products are done
             ++js;
             progressed = true;
@@ -483,7 +489,27 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           l0 = l0 * a0 + (((s[0] + s[1]) + (s[4] + s[5])) + ((s[8] + s[9]) + (s[12] + s[13])));
           l1 = l1 * a1 + (((s[2] + s[3]) + (s[6] + s[7])) + ((s[10] + s[11]) + (s[14] + s[15])));
         }
-        if (j > a) {  // O^T of the previous page is complete: P and O^T may be touched
+        if (ok && !dead) {
+          uint8_t* kv = smem + kOffKV + st * kTileBytes;
+          if (valid < kMlaBs) {  // zero the value rows of tokens past the end (dims 0..511)
+            const int nchunks = (kMlaBs - valid) * 64;
+            for (int i = ts; i < nchunks; i += kSoftmaxThreads) {
+              const int row = valid + (i >> 6), cb = (i >> 3) & 7, ch = i & 7;
+              *reinterpret_cast<uint4*>(kv + cb * kBlockBytes + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
+            }
+          }
+          // P^T tile (K-major, 128-byte swizzle) in this stage's rope box, which QK^T of the page
+          // has finished reading (s_full): 4-byte pieces, the quad fills each 16-byte chunk.  Each
+          // page has its own P^T, so this needs no wait for the previous page's PV product.
+          uint8_t* pt = kv + 8 * kBlockBytes + 4 * quad;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t ch = (uint32_t)(4 * hf + k);
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr0, ch)) = pack_bf16x2(s[4 * k + 0], s[4 * k + 1]);
+            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr1, ch)) = pack_bf16x2(s[4 * k + 2], s[4 * k + 3]);
+          }
+        }
+        if (j > a) {  // O^T of the previous page is complete: O^T may be rescaled
           wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
           od_ph ^= 1u;
           tc_fence_after();
@@ -508,24 +534,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
                 tmem_st32(ta, v);
               }
             tmem_st_wait();
-          }
-        }
-        if (ok && !dead) {
-          uint8_t* kv = smem + kOffKV + st * kTileBytes;
-          if (valid < kMlaBs) {  // zero the value rows of tokens past the end (dims 0..511)
-            const int nchunks = (kMlaBs - valid) * 64;
-            for (int i = ts; i < nchunks; i += kSoftmaxThreads) {
-              const int row = valid + (i >> 6), cb = (i >> 3) & 7, ch = i & 7;
-              *reinterpret_cast<uint4*>(kv + cb * kBlockBytes + row * 128 + ch * 16) = make_uint4(0u, 0u, 0u, 0u);
-            }
-          }
-          // P^T tile (K-major, 128-byte swizzle): 4-byte pieces, the quad fills each 16-byte chunk
-          uint8_t* pt = smem + kOffP + 4 * quad;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t ch = (uint32_t)(4 * hf + k);
-            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr0, ch)) = pack_bf16x2(s[4 * k + 0], s[4 * k + 1]);
-            *reinterpret_cast<uint32_t*>(pt + sw128((uint32_t)hr1, ch)) = pack_bf16x2(s[4 * k + 2], s[4 * k + 3]);
           }
         }
         fence_proxy_async_smem();

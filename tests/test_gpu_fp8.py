@@ -157,3 +157,33 @@ def test_two_pages_per_step_path(D, q_len):
     torch.cuda.synchronize()
     _check(w, D, cache, 0.01, 0.01)
     assert cache.device_error() == 0
+
+
+def test_70b_class_layer_sampled():
+    """Full-size GQA layer with an FP8 cache (2.6 GB of codes) in the benchmark's launch configuration
+    (D = 4, scales 2^-7): a sample of requests against the oracle over the dequantised values, every
+    row finite."""
+    import synth.device as sdev
+    w = synth.workload("gqa_70b")
+    D, scale = 4, 2.0 ** -7
+    cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size, D,
+                              w.seq_lens, w.softmax_scale, 0, "cuda", kv_dtype=FP8, k_scale=scale, v_scale=scale)
+    kv = sdev.kv_source(w, "cuda", cache.cu_seqlens)
+    cache.place(kv)
+    del kv
+    q = sdev.query(w, "cuda")
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    assert torch.isfinite(cache.O).all() and torch.isfinite(cache.LSE).all()
+    lens = np.array(w.seq_lens)
+    sample = sorted({int(lens.argmin()), int(lens.argmax())})
+    O, L = cache.O.cpu().numpy(), cache.LSE.cpu().numpy()
+    for b in sample:
+        vals = oracle.dequantize_kv_gqa(oracle.quantize_kv_gqa(w.kv_source(b), scale, scale), scale, scale)
+        Ob, Lb, _, _ = oracle.sharded_values(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v,
+                                             w.query(b), vals, w.softmax_scale, w.block_size, D)
+        assert_o_close(O[b], Ob, O_TOL, f"O[{b}]")
+        assert_lse_close(L[b], Lb, LSE_TOL, f"LSE[{b}]")
+    del cache
+    torch.cuda.empty_cache()

@@ -115,3 +115,40 @@ def test_d_invariance(layout):
         np.testing.assert_allclose(O, outs[0][0], rtol=0, atol=D_INVARIANCE_TOL)
         np.testing.assert_allclose(L, outs[0][1], rtol=0, atol=D_INVARIANCE_TOL)
 
+
+
+def _oracle_mtp_heads(w, b, D, heads):
+    """Merged multi-token result of request b for a head range (oracle, float64)."""
+    hb, he = heads
+    parts = [oracle.attend_mtp(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.queries(b),
+                               w.kv_source(b), w.softmax_scale, w.q_len, w.block_size, D, s, heads)
+             for s in range(D)]
+    Op = np.stack([p[0][:, hb:he] for p in parts])
+    Lp = np.stack([p[1][:, hb:he] for p in parts])
+    rows = w.q_len * (he - hb)
+    O, L = oracle.merge(Op.reshape(D, rows, -1), Lp.reshape(D, rows))
+    return O.reshape(w.q_len, he - hb, -1), L.reshape(w.q_len, he - hb)
+
+
+@pytest.mark.parametrize("name,q_len,heads", [("gqa_70b", 4, (0, 64)), ("mla_b32", 2, (0, 4))])
+def test_full_size_workload_sampled(name, q_len, heads):
+    """Full-size workloads with draft tokens, in the benchmark's launch configuration: sampled
+    requests (and, for MLA, a head range) against the oracle, every row finite."""
+    w = synth.workload(name)
+    w.q_len = q_len
+    D = max(w.shards)
+    cache, q = build_cache(w, D, device_kv=True)
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    assert torch.isfinite(cache.O).all() and torch.isfinite(cache.LSE).all()
+    lens = np.array(w.seq_lens)
+    sample = sorted({int(lens.argmin()), int(np.argsort(lens)[len(lens) // 2])})
+    O, L = cache.O.cpu().numpy(), cache.LSE.cpu().numpy()
+    hb, he = heads
+    for b in sample:
+        Ob, Lb = _oracle_mtp_heads(w, b, D, heads)
+        assert_o_close(O[b][:, hb:he], Ob, O_TOL, f"O[{b}]")
+        assert_lse_close(L[b][:, hb:he], Lb, LSE_TOL, f"LSE[{b}]")
+    del cache
+    torch.cuda.empty_cache()

@@ -28,7 +28,8 @@
 //                     softmax of a page never waits for the previous PV product.
 //    S of page i+1 is issued before O of page i, so the tensor pipe works while
 //    the softmax runs.
-//  * Warps 2-5: softmax (four threads per head row of S), fp32, base-2; the
+//  * Warps 2-9: softmax (two warps per TMEM sub-partition of 16 head rows, each
+//    on half the page's tokens, four threads per head row), fp32, base-2; the
 //    reference maximum is an integer and is only raised (O^T rescaled in TMEM
 //    by an exact power of two) when a page's maximum exceeds it by more than 8
 //    (a factor of 256); the result is unchanged because the final
@@ -379,7 +380,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       wait_or_die(&misc->mma_done, 0, d2, p.status);
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 2-5)
+    // ------------------------------------------------------------ softmax + epilogue (warps 2-9)
     // Warps 2-9: warp w reads TMEM sub-partition q = w % 4, which holds head rows
     // 16q..16q+15 of S (lanes 32q..32q+15), and token half hf = (w - 2) / 4 of
     // the page.  With the 16x256b load thread t holds heads hr0 = 16q + t/4 and

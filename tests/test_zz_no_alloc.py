@@ -57,6 +57,25 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
         _close(O, L, ref_O, ref_L)
 
 
+@pytest.mark.parametrize("q_len,kv_dtype", [(3, dcp.DCP_KV_BF16), (1, dcp.DCP_KV_FP8_E4M3), (3, dcp.DCP_KV_FP8_E4M3)])
+def test_noalloc_with_draft_tokens_and_fp8_cache(q_len, kv_dtype):
+    # the same kernel variants as the workspace entry point: draft rows, FP8 pools, paired pages
+    from sequence_sharded_decode_paged_b200.cache import ShardedPagedCache
+    w = synth.custom(synth.GQA, [4000, 17, 9000, 1], 64, 8, 128, 128, 16, seed=43, q_len=q_len, kv_amp=0.5)
+    cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size, 3,
+                              w.seq_lens, w.softmax_scale, 0, "cuda", pool_fill=0xFFFF, q_len=q_len,
+                              kv_dtype=kv_dtype, k_scale=2.0 ** -7, v_scale=2.0 ** -7)
+    from gpu_cases import host_kv, host_q
+    cache.place(torch.from_numpy(host_kv(w).view(np.int16)).cuda())
+    q = torch.from_numpy(host_q(w).view(np.int16)).cuda()
+    cache.partials(q)
+    torch.cuda.synchronize()
+    ref_O, ref_L = cache.O_parts.clone(), cache.LSE_parts.clone()
+    for _ in range(2):
+        O, L = _run_noalloc(cache, q)
+        _close(O, L, ref_O, ref_L)
+
+
 def test_noalloc_rejects_problems_larger_than_its_scratch():
     # 16 query heads per KV head and 8 KV heads per CTA: the split partials need more than 16 MiB.
     w = synth.custom(synth.GQA, [64], 128, 8, 128, 128, 16, seed=3)

@@ -152,3 +152,26 @@ def test_full_size_workload_sampled(name, q_len, heads):
         assert_lse_close(L[b][:, hb:he], Lb, LSE_TOL, f"LSE[{b}]")
     del cache
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("layout,kv_dtype", [(synth.GQA, 0), (synth.GQA, 1), (synth.MLA, 0)])
+def test_per_shard_calls_agree_with_one_launch(layout, kv_dtype):
+    """D single-shard dcp_decode_partial calls and one dcp_decode_partial_all launch agree to rounding
+    (different CTA splits), with draft tokens and, for GQA, either cache type."""
+    from sequence_sharded_decode_paged_b200.cache import ShardedPagedCache
+    from gpu_cases import host_kv, host_q
+    shape = (64, 8, 128, 128, 16) if layout == synth.GQA else (64, 1, 576, 512, 64)
+    w = synth.custom(layout, [300, 17, 1000, 64], *shape, seed=29, q_len=2, kv_amp=0.5)
+    cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size, 3,
+                              w.seq_lens, w.softmax_scale, 5, "cuda", pool_fill=0xFFFF, q_len=2, kv_dtype=kv_dtype,
+                              k_scale=2.0 ** -7, v_scale=2.0 ** -7)
+    cache.place(torch.from_numpy(host_kv(w).view(np.int16)).cuda())
+    q = torch.from_numpy(host_q(w).view(np.int16)).cuda()
+    cache.partials(q, per_shard=False)
+    a = (cache.O_parts.clone(), cache.LSE_parts.clone())
+    cache.partials(q, per_shard=True)
+    torch.cuda.synchronize()
+    assert (cache.O_parts - a[0]).abs().max().item() <= 1e-4
+    inf = torch.isinf(a[1])
+    assert torch.equal(torch.isinf(cache.LSE_parts), inf)
+    assert (cache.LSE_parts[~inf] - a[1][~inf]).abs().max().item() <= 1e-4

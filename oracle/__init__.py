@@ -50,6 +50,20 @@ def _load():
             lib.oracle_token_local_block.argtypes = [C.c_int64, C.c_int, C.c_int]
             lib.oracle_block_tables.restype = C.c_int
             lib.oracle_block_tables.argtypes = [p, C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_int, p, p, p]
+            lib.oracle_token_shard_rule.restype = C.c_int
+            lib.oracle_token_shard_rule.argtypes = [C.c_int64, C.c_int, C.c_int, C.c_int, C.c_int64]
+            lib.oracle_token_local_block_rule.restype = C.c_int64
+            lib.oracle_token_local_block_rule.argtypes = [C.c_int64, C.c_int, C.c_int, C.c_int, C.c_int64]
+            lib.oracle_block_tables_rule.restype = C.c_int
+            lib.oracle_block_tables_rule.argtypes = [p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_uint64, C.c_int, p, p,
+                                                     p]
+            lib.oracle_place_request_rule.restype = None
+            lib.oracle_place_request_rule.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                      C.c_int, C.c_int, p, C.c_int64, p, p]
+            lib.oracle_attend_rule_f64.restype = None
+            lib.oracle_attend_rule_f64.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, p, C.c_int64, p,
+                                                   C.c_double, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int64, C.c_int,
+                                                   C.c_int, p, p]
             lib.oracle_grow_tables.restype = C.c_int
             lib.oracle_grow_tables.argtypes = [p, p, C.c_int, C.c_int, C.c_int, C.c_int, p, p, p, p]
             lib.oracle_place_request.restype = None
@@ -71,7 +85,7 @@ def _load():
             lib.oracle_dequantize_e4m3.argtypes = [p, C.c_int64, C.c_double, p]
             lib.oracle_place_request_u8.restype = None
             lib.oracle_place_request_u8.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
-                                                    p, C.c_int64, p, p]
+                                                    C.c_int, p, C.c_int64, p, p]
             lib.oracle_merge.restype = None
             lib.oracle_merge.argtypes = [p, p, C.c_int, C.c_int64, C.c_int, p, p]
             lib.oracle_merge_ml.restype = None
@@ -99,8 +113,20 @@ def token_local_block(t: int, block_size: int, D: int) -> int:
     return _load().oracle_token_local_block(t, block_size, D)
 
 
+INTERLEAVED, CONTIGUOUS = 0, 1  # shard rules
+
+
+def token_shard_rule(t: int, block_size: int, D: int, rule: int, seq_len: int) -> int:
+    return _load().oracle_token_shard_rule(t, block_size, D, rule, seq_len)
+
+
+def token_local_block_rule(t: int, block_size: int, D: int, rule: int, seq_len: int) -> int:
+    return _load().oracle_token_local_block_rule(t, block_size, D, rule, seq_len)
+
+
 def block_tables(seq_lens: Sequence[int], block_size: int, D: int, perm_seed: int = 0,
-                 max_local_blocks: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+                 max_local_blocks: Optional[int] = None, rule: int = INTERLEAVED
+                 ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Returns ``(tables[D][B][max_local_blocks], local_len[D][B], num_pages[D])`` (int32)."""
     sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
     B = sl.shape[0]
@@ -110,8 +136,8 @@ def block_tables(seq_lens: Sequence[int], block_size: int, D: int, perm_seed: in
     tables = np.empty((D, B, max_local_blocks), dtype=np.int32)
     local_len = np.empty((D, B), dtype=np.int32)
     num_pages = np.empty((D,), dtype=np.int32)
-    rc = _load().oracle_block_tables(_ptr(sl), B, block_size, D, perm_seed, max_local_blocks, _ptr(tables),
-                                     _ptr(local_len), _ptr(num_pages))
+    rc = _load().oracle_block_tables_rule(_ptr(sl), B, block_size, D, rule, perm_seed, max_local_blocks,
+                                          _ptr(tables), _ptr(local_len), _ptr(num_pages))
     if rc != 0:
         raise ValueError(f"oracle_block_tables failed ({rc})")
     return tables, local_len, num_pages
@@ -130,7 +156,8 @@ def grow_tables(old_lens: Sequence[int], new_lens: Sequence[int], block_size: in
 
 
 def place(layout: int, Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray,
-          sources: List[np.ndarray], num_pages: np.ndarray, fill: int = 0xFFFF) -> List[np.ndarray]:
+          sources: List[np.ndarray], num_pages: np.ndarray, fill: int = 0xFFFF, rule: int = INTERLEAVED
+          ) -> List[np.ndarray]:
     """Reference cache placement: returns D pools (uint16 bf16 bits), unused slots set to ``fill``."""
     B = len(sources)
     mlb = tables.shape[2]
@@ -140,8 +167,8 @@ def place(layout: int, Hkv: int, d: int, block_size: int, D: int, tables: np.nda
     t = np.ascontiguousarray(tables, dtype=np.int32)
     for b, src in enumerate(sources):
         src = np.ascontiguousarray(src, dtype=np.uint16)
-        _load().oracle_place_request(layout, Hkv, d, block_size, D, B, b, mlb, _ptr(t), src.shape[0], _ptr(src),
-                                     C.cast(arr, C.c_void_p))
+        _load().oracle_place_request_rule(layout, Hkv, d, block_size, D, rule, B, b, mlb, _ptr(t), src.shape[0],
+                                          _ptr(src), C.cast(arr, C.c_void_p))
     return pools
 
 
@@ -149,14 +176,19 @@ def place(layout: int, Hkv: int, d: int, block_size: int, D: int, tables: np.nda
 # attention and merge
 # ---------------------------------------------------------------------------
 def attend(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
-           block_size: int = 1, D: int = 1, shard: int = -1, heads: Optional[Tuple[int, int]] = None
-           ) -> Tuple[np.ndarray, np.ndarray]:
+           block_size: int = 1, D: int = 1, shard: int = -1, heads: Optional[Tuple[int, int]] = None,
+           rule: int = INTERLEAVED, rule_len: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Attention of one request (q bf16 bits [Hq][d_qk], src unsharded rows) -> (O[Hq][d_v], LSE[Hq]) f64.
 
-    ``shard < 0``: all tokens; otherwise only the tokens whose logical block
-    ``t // block_size`` is congruent to ``shard`` modulo ``D``.  Heads outside
-    ``heads = (begin, end)`` are left as NaN.
+    ``shard < 0``: all tokens; otherwise only the tokens shard ``shard`` stores: under the interleaved
+    rule those whose logical block ``t // block_size`` is congruent to ``shard`` modulo ``D``, under the
+    contiguous rule those in its chunk of a request of ``rule_len`` tokens (default: ``len(src)``).
+    Heads outside ``heads = (begin, end)`` are left as NaN.
     """
+    if rule != INTERLEAVED:
+        bits = np.ascontiguousarray(src, dtype=np.uint16)
+        wide = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)  # exact
+        return attend_values(layout, Hq, Hkv, d_qk, d_v, q, wide, scale, block_size, D, shard, heads, rule, rule_len)
     q = np.ascontiguousarray(q, dtype=np.uint16)
     src = np.ascontiguousarray(src, dtype=np.uint16)
     hb, he = heads if heads is not None else (0, Hq)
@@ -169,15 +201,17 @@ def attend(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, s
 
 def attend_values(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray,
                   scale: float, block_size: int = 1, D: int = 1, shard: int = -1,
-                  heads: Optional[Tuple[int, int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+                  heads: Optional[Tuple[int, int]] = None, rule: int = INTERLEAVED,
+                  rule_len: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
     """``attend`` with the key/value source given as float64 values (same row layout)."""
     q = np.ascontiguousarray(q, dtype=np.uint16)
     src = np.ascontiguousarray(src, dtype=np.float64)
     hb, he = heads if heads is not None else (0, Hq)
     O = np.full((Hq, d_v), np.nan)
     LSE = np.full((Hq,), np.nan)
-    _load().oracle_attend_f64(layout, Hq, Hkv, d_qk, d_v, _ptr(q), src.shape[0], _ptr(src), scale, block_size, D,
-                              shard, hb, he, _ptr(O), _ptr(LSE))
+    n = src.shape[0]
+    _load().oracle_attend_rule_f64(layout, Hq, Hkv, d_qk, d_v, _ptr(q), n, _ptr(src), scale, block_size, D, shard,
+                                   rule, n if rule_len is None else rule_len, hb, he, _ptr(O), _ptr(LSE))
     return O, LSE
 
 
@@ -231,7 +265,7 @@ def dequantize_kv_gqa(codes: np.ndarray, k_scale: float, v_scale: float) -> np.n
 
 
 def place_u8(Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray, codes: List[np.ndarray],
-             num_pages: np.ndarray, fill: int = 0xFF) -> List[np.ndarray]:
+             num_pages: np.ndarray, fill: int = 0xFF, rule: int = INTERLEAVED) -> List[np.ndarray]:
     """Reference placement of quantised GQA rows: D byte pools, unused bytes set to ``fill``."""
     B = len(codes)
     mlb = tables.shape[2]
@@ -241,15 +275,16 @@ def place_u8(Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray, code
     t = np.ascontiguousarray(tables, dtype=np.int32)
     for b, c in enumerate(codes):
         c = np.ascontiguousarray(c, dtype=np.uint8)
-        _load().oracle_place_request_u8(Hkv, d, block_size, D, B, b, mlb, _ptr(t), c.shape[0], _ptr(c),
+        _load().oracle_place_request_u8(Hkv, d, block_size, D, rule, B, b, mlb, _ptr(t), c.shape[0], _ptr(c),
                                         C.cast(arr, C.c_void_p))
     return pools
 
 
 def sharded_values(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray,
-                   scale: float, block_size: int, D: int):
+                   scale: float, block_size: int, D: int, rule: int = INTERLEAVED):
     """``sharded`` over a float64-valued source (e.g. a dequantised FP8 cache)."""
-    parts = [attend_values(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s) for s in range(D)]
+    parts = [attend_values(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s, None, rule)
+             for s in range(D)]
     Op = np.stack([p[0] for p in parts])
     Lp = np.stack([p[1] for p in parts])
     O, LSE = merge(Op, Lp)
@@ -279,9 +314,9 @@ def merge_ml(U_parts: np.ndarray, m_parts: np.ndarray, l_parts: np.ndarray) -> n
 
 
 def sharded(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
-            block_size: int, D: int, heads: Optional[Tuple[int, int]] = None):
+            block_size: int, D: int, heads: Optional[Tuple[int, int]] = None, rule: int = INTERLEAVED):
     """Per-shard partials followed by the merge: returns (O, LSE, O_parts[D], LSE_parts[D])."""
-    parts = [attend(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s, heads) for s in range(D)]
+    parts = [attend(layout, Hq, Hkv, d_qk, d_v, q, src, scale, block_size, D, s, heads, rule) for s in range(D)]
     Op = np.stack([p[0] for p in parts])
     Lp = np.stack([p[1] for p in parts])
     hb, he = heads if heads is not None else (0, Hq)
@@ -303,7 +338,7 @@ def visible_tokens(seq_len: int, q_len: int, j: int) -> int:
 
 def attend_mtp(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
                q_len: int, block_size: int = 1, D: int = 1, shard: int = -1,
-               heads: Optional[Tuple[int, int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+               heads: Optional[Tuple[int, int]] = None, rule: int = INTERLEAVED) -> Tuple[np.ndarray, np.ndarray]:
     """Attention of the ``q_len`` query tokens of one request: ``q`` bf16 bits [q_len][Hq][d_qk] ->
     (O[q_len][Hq][d_v], LSE[q_len][Hq]).  Token j is ``attend`` over the first
     ``visible_tokens(len(src), q_len, j)`` source rows (restricted to ``shard`` as in ``attend``)."""
@@ -312,15 +347,17 @@ def attend_mtp(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarra
     O = np.empty((q_len, Hq, d_v))
     LSE = np.empty((q_len, Hq))
     for j in range(q_len):
+        # the shard of a token follows from the whole request (L tokens), not from the visible prefix
         O[j], LSE[j] = attend(layout, Hq, Hkv, d_qk, d_v, q[j], src[:visible_tokens(L, q_len, j)], scale,
-                              block_size, D, shard, heads)
+                              block_size, D, shard, heads, rule, L)
     return O, LSE
 
 
 def sharded_mtp(layout: int, Hq: int, Hkv: int, d_qk: int, d_v: int, q: np.ndarray, src: np.ndarray, scale: float,
-                q_len: int, block_size: int, D: int):
+                q_len: int, block_size: int, D: int, rule: int = INTERLEAVED):
     """Per-shard multi-token partials and their merge: (O[q_len][Hq][d_v], LSE[q_len][Hq], O_parts[D], LSE_parts[D])."""
-    parts = [attend_mtp(layout, Hq, Hkv, d_qk, d_v, q, src, scale, q_len, block_size, D, s) for s in range(D)]
+    parts = [attend_mtp(layout, Hq, Hkv, d_qk, d_v, q, src, scale, q_len, block_size, D, s, None, rule)
+             for s in range(D)]
     Op = np.stack([p[0] for p in parts])
     Lp = np.stack([p[1] for p in parts])
     O, LSE = merge(Op.reshape(D, q_len * Hq, d_v), Lp.reshape(D, q_len * Hq))

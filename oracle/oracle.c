@@ -64,6 +64,32 @@ int64_t oracle_token_local_block(int64_t t, int block_size, int D) {
     return (t / block_size) / D;
 }
 
+/*
+ * Contiguous-chunk rule (the [P1] "A2 方法细节" illustration "GPU0 holds 0-50K,
+ * GPU1 50K-100K, ..." for a 200K sequence on 4 GPUs): the nblk = ceil(len/bs)
+ * logical blocks of a request are cut into D consecutive chunks, shard s
+ * holding blocks floor(s*nblk/D) .. floor((s+1)*nblk/D) - 1; its local block
+ * index counts from the start of its chunk.  The chunking depends on the
+ * request's total length `seq_len`.  rule 0 is the interleaved rule above,
+ * rule 1 this one.
+ */
+static int64_t or_chunk_begin(int64_t nblk, int D, int s) { return ((int64_t)s * nblk) / D; }
+
+int oracle_token_shard_rule(int64_t t, int block_size, int D, int rule, int64_t seq_len) {
+    if (rule == 0) return oracle_token_shard(t, block_size, D);
+    int64_t g = t / block_size, nblk = (seq_len + block_size - 1) / block_size;
+    for (int s = 0; s < D; ++s)
+        if (g < or_chunk_begin(nblk, D, s + 1)) return s;
+    return D - 1;
+}
+
+int64_t oracle_token_local_block_rule(int64_t t, int block_size, int D, int rule, int64_t seq_len) {
+    if (rule == 0) return oracle_token_local_block(t, block_size, D);
+    int64_t nblk = (seq_len + block_size - 1) / block_size;
+    int s = oracle_token_shard_rule(t, block_size, D, rule, seq_len);
+    return t / block_size - or_chunk_begin(nblk, D, s);
+}
+
 /* SplitMix64 (Steele, Lea & Flood 2014), used only for the optional page permutation. */
 static uint64_t or_mix(uint64_t z) {
     z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;
@@ -89,8 +115,8 @@ static uint64_t or_mix(uint64_t z) {
  * Returns 0 on success, -1 on bad arguments, -2 if max_local_blocks is too
  * small for some request.
  */
-int oracle_block_tables(const int32_t *seq_lens, int B, int block_size, int D, uint64_t perm_seed,
-                        int max_local_blocks, int32_t *tables, int32_t *local_len, int32_t *num_pages) {
+int oracle_block_tables_rule(const int32_t *seq_lens, int B, int block_size, int D, int rule, uint64_t perm_seed,
+                             int max_local_blocks, int32_t *tables, int32_t *local_len, int32_t *num_pages) {
     if (B < 0 || block_size <= 0 || D <= 0 || max_local_blocks < 0) return -1;
     for (int b = 0; b < B; ++b)
         if (seq_lens[b] < 0) return -1;
@@ -100,8 +126,8 @@ int oracle_block_tables(const int32_t *seq_lens, int B, int block_size, int D, u
     int rc = 0;
     for (int b = 0; b < B && rc == 0; ++b) {
         for (int64_t t = 0; t < seq_lens[b]; ++t) {
-            int s = oracle_token_shard(t, block_size, D);
-            int64_t j = oracle_token_local_block(t, block_size, D);
+            int s = oracle_token_shard_rule(t, block_size, D, rule, seq_lens[b]);
+            int64_t j = oracle_token_local_block_rule(t, block_size, D, rule, seq_lens[b]);
             if (j >= max_local_blocks) { rc = -2; break; }
             int32_t *entry = &tables[((int64_t)s * B + b) * max_local_blocks + j];
             if (*entry < 0) *entry = (int32_t)next_page[s]++;
@@ -133,6 +159,13 @@ int oracle_block_tables(const int32_t *seq_lens, int B, int block_size, int D, u
     }
     free(next_page);
     return rc;
+}
+
+/* The tables under the interleaved rule. */
+int oracle_block_tables(const int32_t *seq_lens, int B, int block_size, int D, uint64_t perm_seed,
+                        int max_local_blocks, int32_t *tables, int32_t *local_len, int32_t *num_pages) {
+    return oracle_block_tables_rule(seq_lens, B, block_size, D, 0, perm_seed, max_local_blocks, tables, local_len,
+                                    num_pages);
 }
 
 /*
@@ -177,12 +210,12 @@ int oracle_grow_tables(const int32_t *old_lens, const int32_t *new_lens, int B, 
  *   MLA pool page layout: [bs][d_qk]               (source row [d_qk])
  * pools[s] points at shard s's pool (bytes, bf16 elements).
  */
-void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int B, int b,
-                          int max_local_blocks, const int32_t *tables, int64_t n_tok, const uint16_t *src,
-                          uint16_t **pools) {
+void oracle_place_request_rule(int layout, int Hkv, int d, int block_size, int D, int rule, int B, int b,
+                               int max_local_blocks, const int32_t *tables, int64_t n_tok, const uint16_t *src,
+                               uint16_t **pools) {
     for (int64_t t = 0; t < n_tok; ++t) {
-        int s = oracle_token_shard(t, block_size, D);
-        int64_t j = oracle_token_local_block(t, block_size, D);
+        int s = oracle_token_shard_rule(t, block_size, D, rule, n_tok);
+        int64_t j = oracle_token_local_block_rule(t, block_size, D, rule, n_tok);
         int64_t page = tables[((int64_t)s * B + b) * max_local_blocks + j];
         int64_t slot = t % block_size;
         if (layout == OR_GQA) {
@@ -198,6 +231,12 @@ void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int
     }
 }
 
+void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int B, int b,
+                          int max_local_blocks, const int32_t *tables, int64_t n_tok, const uint16_t *src,
+                          uint16_t **pools) {
+    oracle_place_request_rule(layout, Hkv, d, block_size, D, 0, B, b, max_local_blocks, tables, n_tok, src, pools);
+}
+
 /* ------------------------------------------------------------------ */
 /* Attention of one request over a token subset                        */
 /* ------------------------------------------------------------------ */
@@ -205,8 +244,9 @@ void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int
 /*
  * Softmax attention of the single decode query of one request against the
  * tokens t in [0, n_tok) that satisfy the filter: all tokens when shard < 0,
- * else the tokens whose logical block floor(t/bs) satisfies block % D ==
- * shard (P3 §2.2).  Direct definition, two passes, no blocking:
+ * else the tokens that shard `shard` stores under `rule` (interleaved: logical
+ * block floor(t/bs) % D == shard, P3 §2.2; contiguous: the chunk of a request
+ * of rule_len tokens, see above).  Direct definition, two passes, no blocking:
  *   s_t   = scale * sum_k q[h][k] * K_t[k]
  *   M     = max_t s_t,  Z = sum_t exp(s_t - M)
  *   O[h]  = sum_t exp(s_t - M) V_t / Z,   LSE[h] = M + ln Z
@@ -216,9 +256,9 @@ void oracle_place_request(int layout, int Hkv, int d, int block_size, int D, int
  * Heads are computed for h in [h_begin, h_end); outputs are indexed by the
  * absolute head: O[h][d_v], LSE[h].
  */
-void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
-                       const double *src, double scale, int block_size, int D, int shard, int h_begin, int h_end,
-                       double *O, double *LSE) {
+void oracle_attend_rule_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
+                            const double *src, double scale, int block_size, int D, int shard, int rule,
+                            int64_t rule_len, int h_begin, int h_end, double *O, double *LSE) {
     double *s = (double *)malloc((size_t)(n_tok > 0 ? n_tok : 1) * sizeof(double));
     double *qd = (double *)malloc((size_t)d_qk * sizeof(double));
     int group = (layout == OR_GQA) ? Hq / Hkv : Hq;
@@ -228,7 +268,7 @@ void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uin
         double M = -INFINITY;
         int64_t count = 0;
         for (int64_t t = 0; t < n_tok; ++t) {
-            if (shard >= 0 && oracle_token_shard(t, block_size, D) != shard) continue;
+            if (shard >= 0 && oracle_token_shard_rule(t, block_size, D, rule, rule_len) != shard) continue;
             const double *krow = (layout == OR_GQA) ? src + ((t * 2 + 0) * Hkv + kvh) * (int64_t)d_qk
                                                     : src + t * (int64_t)d_qk;
             double acc = 0.0;
@@ -245,7 +285,7 @@ void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uin
         }
         double Z = 0.0;
         for (int64_t t = 0; t < n_tok; ++t) {
-            if (shard >= 0 && oracle_token_shard(t, block_size, D) != shard) continue;
+            if (shard >= 0 && oracle_token_shard_rule(t, block_size, D, rule, rule_len) != shard) continue;
             const double *vrow = (layout == OR_GQA) ? src + ((t * 2 + 1) * Hkv + kvh) * (int64_t)d_qk
                                                     : src + t * (int64_t)d_qk;
             double w = exp(s[t] - M);
@@ -257,6 +297,14 @@ void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uin
     }
     free(qd);
     free(s);
+}
+
+/* Interleaved-rule attention over a float64-valued source. */
+void oracle_attend_f64(int layout, int Hq, int Hkv, int d_qk, int d_v, const uint16_t *q, int64_t n_tok,
+                       const double *src, double scale, int block_size, int D, int shard, int h_begin, int h_end,
+                       double *O, double *LSE) {
+    oracle_attend_rule_f64(layout, Hq, Hkv, d_qk, d_v, q, n_tok, src, scale, block_size, D, shard, 0, n_tok, h_begin,
+                           h_end, O, LSE);
 }
 
 /* The same attention with the key/value source given as bf16 bit patterns
@@ -335,13 +383,13 @@ void oracle_dequantize_e4m3(const uint8_t *codes, int64_t n, double scale, doubl
 /*
  * Placement of one request's quantised GQA rows (codes [n_tok][2][Hkv][d],
  * one byte per element) into byte pools whose pages are [2][Hkv][bs][d]:
- * the same token walk as oracle_place_request, one byte per element.
+ * the same token walk as oracle_place_request_rule, one byte per element.
  */
-void oracle_place_request_u8(int Hkv, int d, int block_size, int D, int B, int b, int max_local_blocks,
+void oracle_place_request_u8(int Hkv, int d, int block_size, int D, int rule, int B, int b, int max_local_blocks,
                              const int32_t *tables, int64_t n_tok, const uint8_t *src, uint8_t **pools) {
     for (int64_t t = 0; t < n_tok; ++t) {
-        int s = oracle_token_shard(t, block_size, D);
-        int64_t j = oracle_token_local_block(t, block_size, D);
+        int s = oracle_token_shard_rule(t, block_size, D, rule, n_tok);
+        int64_t j = oracle_token_local_block_rule(t, block_size, D, rule, n_tok);
         int64_t page = tables[((int64_t)s * B + b) * max_local_blocks + j];
         int64_t slot = t % block_size;
         for (int kv = 0; kv < 2; ++kv)

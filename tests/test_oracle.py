@@ -545,3 +545,96 @@ def test_fp8_placement_roundtrip():
             np.testing.assert_array_equal(pg[:, :, t % 16], codes[b][t])
     used = sum(int(w.seq_lens[b]) for b in range(w.batch)) * 2 * 2 * 128
     assert sum(int((p != 0x7F).sum()) for p in pools) <= used
+
+
+# ---------------------------------------------------------------------------
+# contiguous-chunk shard rule ([P1] A2 illustration: "GPU0 holds 0-50K, GPU1 50K-100K, ...")
+# ---------------------------------------------------------------------------
+CONTIG = oracle.CONTIGUOUS
+
+
+def test_contiguous_rule_page_example():
+    # 200,000 tokens on 4 shards (block 16: 12,500 blocks): shard s holds tokens [50,000 s, 50,000 (s+1))
+    L = 200_000
+    for t, s, j in [(0, 0, 0), (49_999, 0, 3124), (50_000, 1, 0), (99_999, 1, 3124), (150_000, 3, 0),
+                    (199_999, 3, 3124)]:
+        assert oracle.token_shard_rule(t, 16, 4, CONTIG, L) == s
+        assert oracle.token_local_block_rule(t, 16, 4, CONTIG, L) == j
+    _, local_len, pages = oracle.block_tables([L], 16, 4, rule=CONTIG)
+    assert list(local_len[:, 0]) == [50_000] * 4 and list(pages) == [3125] * 4
+
+
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("bs", [1, 16, 64])
+def test_contiguous_tables_are_a_bijection_of_contiguous_ranges(D, bs):
+    rng = np.random.default_rng(D * 31 + bs)
+    seq_lens = list(rng.integers(0, 700, size=7)) + [1, bs, bs + 1, 3 * bs]
+    tables, local_len, num_pages = oracle.block_tables(seq_lens, bs, D, perm_seed=9, rule=CONTIG)
+    seen = [set() for _ in range(D)]
+    for b, n in enumerate(seq_lens):
+        assert int(local_len[:, b].sum()) == n
+        nblk = -(-n // bs)
+        owner = [oracle.token_shard_rule(t, bs, D, CONTIG, n) for t in range(n)]
+        assert owner == sorted(owner)  # each shard holds one run of consecutive tokens, in shard order
+        sizes = [sum(1 for g in range(nblk) if oracle.token_shard_rule(g * bs, bs, D, CONTIG, n) == s) for s in range(D)]
+        assert max(sizes) - min(sizes) <= 1  # chunks differ by at most one block
+        for t in range(n):
+            s, j = owner[t], oracle.token_local_block_rule(t, bs, D, CONTIG, n)
+            assert j == t // bs - sum(sizes[:s])
+            page = tables[s, b, j]
+            assert 0 <= page < num_pages[s]
+            key = (int(page), t % bs)
+            assert key not in seen[s]
+            seen[s].add(key)
+    for s in range(D):
+        assert {p for p, _ in seen[s]} == set(range(int(num_pages[s])))
+
+
+def test_contiguous_with_one_shard_is_interleaved():
+    seq_lens = [300, 5, 1000]
+    a = oracle.block_tables(seq_lens, 16, 1)
+    b = oracle.block_tables(seq_lens, 16, 1, rule=CONTIG)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("D", [2, 3, 4, 8])
+def test_contiguous_sharded_merge_equals_direct(D):
+    for layout, Hq, Hkv, dqk, dv in [(GQA, 8, 2, 64, 64), (MLA, 4, 1, 576, 512)]:
+        for L in [5, 40, 257]:  # fewer blocks than shards, and several blocks per shard
+            w = synth.custom(layout, [L], Hq, Hkv, dqk, dv, 16, seed=L + D)
+            q, src = w.query(0), w.kv_source(0)
+            O, LSE = oracle.attend(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale)
+            Om, Lm, _, Lp = oracle.sharded(layout, Hq, Hkv, dqk, dv, q, src, w.softmax_scale, 16, D, rule=CONTIG)
+            np.testing.assert_allclose(Om, O, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(Lm, LSE, rtol=0, atol=1e-12)
+
+
+def test_contiguous_multi_token_merge_equals_direct():
+    w = synth.custom(GQA, [70], 8, 2, 64, 64, 16, seed=71, q_len=3)
+    q, src = w.queries(0), w.kv_source(0)
+    O, LSE = oracle.attend_mtp(GQA, 8, 2, 64, 64, q, src, w.softmax_scale, 3)
+    Om, Lm, _, _ = oracle.sharded_mtp(GQA, 8, 2, 64, 64, q, src, w.softmax_scale, 3, 16, 3, rule=CONTIG)
+    np.testing.assert_allclose(Om, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lm, LSE, rtol=0, atol=1e-12)
+    # the drafts (the last tokens) all fall in the last shard: on the other shards every draft sees the
+    # whole shard, so its partial is plain attention over that shard
+    _, _, Op, Lp = oracle.sharded_mtp(GQA, 8, 2, 64, 64, q, src, w.softmax_scale, 3, 16, 3, rule=CONTIG)
+    for s in range(2):
+        for j in range(3):
+            Os, Ls = oracle.attend(GQA, 8, 2, 64, 64, q[j], src, w.softmax_scale, 16, 3, s, rule=CONTIG)
+            np.testing.assert_array_equal(Op[s][j], Os)
+            np.testing.assert_array_equal(Lp[s][j], Ls)
+
+
+def test_contiguous_placement_roundtrip():
+    w = synth.custom(GQA, [37, 16, 1, 100], 4, 2, 64, 64, 16, seed=9)
+    D = 3
+    tables, _, num_pages = oracle.block_tables(w.seq_lens, 16, D, perm_seed=5, rule=CONTIG)
+    srcs = [w.kv_source(b) for b in range(w.batch)]
+    pools = oracle.place(GQA, 2, 64, 16, D, tables, srcs, num_pages, fill=0xFFFF, rule=CONTIG)
+    for b, n in enumerate(w.seq_lens):
+        for t in range(n):
+            s, j = oracle.token_shard_rule(t, 16, D, CONTIG, n), oracle.token_local_block_rule(t, 16, D, CONTIG, n)
+            pg = pools[s][tables[s, b, j] * 2 * 2 * 16 * 64:(tables[s, b, j] + 1) * 2 * 2 * 16 * 64].reshape(2, 2, 16, 64)
+            np.testing.assert_array_equal(pg[:, :, t % 16], srcs[b][t])

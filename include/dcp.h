@@ -92,6 +92,23 @@ typedef enum dcp_layout {
  *                    products; query elements outside f16's normal range
  *                    (|q| > 65504 or |q| < 2^-14) lose precision there.
  */
+/*
+ * How a request's logical blocks are dealt to the D shards.
+ *   DCP_SHARD_INTERLEAVED  block g -> shard g % D as local block g / D ([P3] §2.2/§3.2; the
+ *                          rule the pages' implementation uses).
+ *   DCP_SHARD_CONTIGUOUS   the nblk = ceil(len / block_size) blocks are cut into D consecutive
+ *                          chunks: shard s holds blocks floor(s*nblk/D) .. floor((s+1)*nblk/D) - 1,
+ *                          local block g - floor(s*nblk/D) ([P1] "A2 方法细节" illustrates
+ *                          sequence sharding as "GPU0 holds 0-50K, GPU1 50K-100K, ...").  A
+ *                          token's shard depends on the request's total length, so contiguous
+ *                          tables cannot grow: dcp_grow_block_table and dcp_append_kv are
+ *                          interleaved only.
+ */
+typedef enum dcp_shard_rule {
+    DCP_SHARD_INTERLEAVED = 0,
+    DCP_SHARD_CONTIGUOUS = 1
+} dcp_shard_rule;
+
 typedef enum dcp_kv_dtype {
     DCP_KV_BF16 = 0,
     DCP_KV_FP8_E4M3 = 1
@@ -118,6 +135,7 @@ typedef enum dcp_kv_dtype {
  *                    shard gets O = 0, LSE = -inf there.
  *   kv_dtype         dcp_kv_dtype of the pools.
  *   k_scale, v_scale per-tensor scales of an FP8 cache (positive, finite); ignored for bf16.
+ *   shard_rule       dcp_shard_rule the tables were built with (pools, tables and seq_lens must agree).
  */
 typedef struct dcp_attn_desc {
     int32_t layout;
@@ -133,6 +151,7 @@ typedef struct dcp_attn_desc {
     int32_t kv_dtype;
     float k_scale;
     float v_scale;
+    int32_t shard_rule;
 } dcp_attn_desc;
 
 /* Library version, major * 10000 + minor * 100 + patch. */
@@ -174,6 +193,19 @@ DCP_API dcp_status dcp_build_block_table(const int32_t *seq_lens, int32_t batch,
                                  uint64_t perm_seed, int32_t max_local_blocks, int32_t *tables,
                                  int32_t *local_len);
 
+/*
+ * The same two calls under a chosen dcp_shard_rule (the calls above use
+ * DCP_SHARD_INTERLEAVED).  Under DCP_SHARD_CONTIGUOUS, tables[s][b][j] holds
+ * the page of global block floor(s*nblk_b/D) + j, pages are still numbered in
+ * (request, local block) order, and local_len counts the chunk's tokens.
+ * Errors: as above, and DCP_ERR_INVALID_ARG for an unknown rule.
+ */
+DCP_API dcp_status dcp_block_table_extent_rule(const int32_t *seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                               int32_t shard_rule, int32_t *max_local_blocks, int32_t *num_pages);
+DCP_API dcp_status dcp_build_block_table_rule(const int32_t *seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                              int32_t shard_rule, uint64_t perm_seed, int32_t max_local_blocks,
+                                              int32_t *tables, int32_t *local_len);
+
 /* Bytes of one KV page for `desc` (GQA: 2*Hkv*block_size*head_dim*e; MLA: block_size*576*2; e = 2 for
  * bf16, 1 for FP8); 0 if invalid. */
 DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
@@ -184,9 +216,9 @@ DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
  *   kv_src      device bf16, requests concatenated in order:
  *               GQA rows [token][2 (K,V)][Hkv][head_dim]; MLA rows [token][576].
  *   cu_seqlens  device int64[batch+1], prefix sums of seq_lens (row offsets in kv_src).
- *   seq_lens    device int32[batch].
+ *   seq_lens    device int32[batch] (the contiguous rule reads them to find each token's shard).
  *   tables      host array of D device pointers, each int32[batch][max_local_blocks]
- *               (as built by dcp_build_block_table).
+ *               (as built by dcp_build_block_table / _rule with desc->shard_rule).
  *   kv_pools    host array of D device pointers; pool s holds pool_pages[s] pages:
  *               GQA page [2 (K,V)][Hkv][block_size][head_dim] of the pool's
  *               kv_dtype (bf16, or FP8 codes quantised on the way in);
@@ -232,6 +264,7 @@ DCP_API dcp_status dcp_grow_block_table(const int32_t *old_seq_lens, const int32
  *   cu_rows     device int64[batch+1];  first_pos  device int32[batch].
  *   tables, kv_pools, pool_pages, device_error: as in dcp_place_kv (tables
  *               already grown to cover the new tokens).
+ * Interleaved shard rule only (DCP_ERR_UNSUPPORTED otherwise).
  */
 DCP_API dcp_status dcp_append_kv(const dcp_attn_desc *desc, int32_t D, const void *kv_new, const int64_t *cu_rows,
                                  const int32_t *first_pos, const int32_t *const *tables, void *const *kv_pools,
@@ -252,7 +285,8 @@ DCP_API dcp_status dcp_workspace_init(void *workspace, size_t workspace_bytes, v
 /*
  * Partial attention of ONE shard.  [P1 "A2 方法细节", Compute step]
  * For every request b and query head h, over the tokens of b that shard
- * `shard` stores (logical blocks g with g % D == shard):
+ * `shard` stores (logical blocks g with g % D == shard, or its chunk under
+ * the contiguous rule):
  *   s_t = softmax_scale * q[b][h] . k_t,  m = max s_t,  l = sum exp(s_t - m),
  *   O_i[b][h] = sum exp(s_t - m) v_t / l,  LSE_i[b][h] = m + ln l.
  * GQA: k_t, v_t are KV head h / (Hq/Hkv) of token t.  MLA: k_t is the whole
@@ -262,7 +296,7 @@ DCP_API dcp_status dcp_workspace_init(void *workspace, size_t workspace_bytes, v
  *   kv_pool     device, this shard's pool (layout as in dcp_place_kv), pool_pages pages.
  *   table       device int32 [batch][max_local_blocks], this shard's block table.
  *   seq_lens    device int32 [batch], GLOBAL lengths; the local token count is
- *               derived from (seq_len, block_size, shard, D).
+ *               derived from (seq_len, block_size, shard, D, desc->shard_rule).
  *   O_i         device fp32 [batch][q_len][Hq][head_dim_v];  LSE_i  device fp32 [batch][q_len][Hq].
  * With q_len > 1 each (request, query token j, head) row follows the same
  * formulas over the visible tokens t < seq_len - (q_len - 1 - j).

@@ -21,20 +21,20 @@ class ShardedPagedCache:
     def __init__(self, layout: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
                  block_size: int, D: int, seq_lens: Sequence[int], softmax_scale: float, perm_seed: int = 0,
                  device="cuda", pool_fill: Optional[int] = None, q_len: int = 1, kv_dtype: int = 0,
-                 k_scale: float = 1.0, v_scale: float = 1.0):
+                 k_scale: float = 1.0, v_scale: float = 1.0, shard_rule: int = 0):
         self.D = D
         self.q_len = q_len
         self.device = torch.device(device)
         self.seq_lens = [int(x) for x in seq_lens]
         self.batch = len(self.seq_lens)
-        mlb, num_pages = dcp.dcp_block_table_extent(self.seq_lens, block_size, D)
+        mlb, num_pages = dcp.dcp_block_table_extent(self.seq_lens, block_size, D, shard_rule)
         self.max_local_blocks = max(1, mlb)
         self.num_pages = num_pages
         self.tables_host, self.local_len = dcp.dcp_build_block_table(self.seq_lens, block_size, D, perm_seed,
-                                                                     self.max_local_blocks)
+                                                                     self.max_local_blocks, shard_rule)
         self.desc = dcp.make_desc(layout, self.batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v,
                                   block_size, self.max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale,
-                                  v_scale)
+                                  v_scale, shard_rule)
         self.page_bytes = dcp.dcp_kv_page_bytes(self.desc)
         if self.page_bytes == 0:
             raise ValueError("unsupported attention shape")

@@ -18,9 +18,23 @@
 
 namespace dcp {
 
-static int nloc_blocks(int64_t len, int bs, int D, int s) {
+// Contiguous rule: shard s holds the blocks [chunk_begin(s), chunk_begin(s + 1)).
+static int64_t chunk_begin(int64_t nblk, int D, int s) { return (int64_t)s * nblk / D; }
+
+static int nloc_blocks(int64_t len, int bs, int D, int s, int rule = DCP_SHARD_INTERLEAVED) {
   const int64_t nblk = (len + bs - 1) / bs;
+  if (rule == DCP_SHARD_CONTIGUOUS) return (int)(chunk_begin(nblk, D, s + 1) - chunk_begin(nblk, D, s));
   return nblk > s ? (int)((nblk - 1 - s) / D + 1) : 0;
+}
+
+// Tokens of a request that shard s stores: its blocks, less the unused tail of the request's last
+// block when that block is the shard's.
+static int64_t nloc_tokens(int64_t len, int bs, int D, int s, int rule) {
+  const int64_t nblk = (len + bs - 1) / bs;
+  const int n = nloc_blocks(len, bs, D, s, rule);
+  if (n == 0) return 0;
+  const bool has_last = rule == DCP_SHARD_CONTIGUOUS ? chunk_begin(nblk, D, s + 1) == nblk : (nblk - 1) % D == s;
+  return (int64_t)n * bs - (has_last ? nblk * bs - len : 0);
 }
 
 int device_sm_count() {
@@ -74,6 +88,7 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
       d.q_len < 1)
     return false;
   if (d.kv_dtype != DCP_KV_BF16 && d.kv_dtype != DCP_KV_FP8_E4M3) return false;
+  if (d.shard_rule != DCP_SHARD_INTERLEAVED && d.shard_rule != DCP_SHARD_CONTIGUOUS) return false;
   if (d.kv_dtype == DCP_KV_FP8_E4M3 &&
       !(d.k_scale > 0.f && d.k_scale < INFINITY && d.v_scale > 0.f && d.v_scale < INFINITY))
     return false;
@@ -146,17 +161,17 @@ const char* dcp_status_string(dcp_status s) {
   return "unknown status";
 }
 
-dcp_status dcp_block_table_extent(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
-                                  int32_t* max_local_blocks, int32_t* num_pages) {
+dcp_status dcp_block_table_extent_rule(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                       int32_t shard_rule, int32_t* max_local_blocks, int32_t* num_pages) {
   if (seq_lens == nullptr || max_local_blocks == nullptr || num_pages == nullptr || batch < 0 || block_size <= 0 ||
-      D < 1 || D > kMaxShardsHost)
+      D < 1 || D > kMaxShardsHost || (shard_rule != DCP_SHARD_INTERLEAVED && shard_rule != DCP_SHARD_CONTIGUOUS))
     return DCP_ERR_INVALID_ARG;
   int64_t mx = 0;
   std::vector<int64_t> pages(D, 0);
   for (int b = 0; b < batch; ++b) {
     if (seq_lens[b] < 0) return DCP_ERR_INVALID_ARG;
     for (int s = 0; s < D; ++s) {
-      const int n = nloc_blocks(seq_lens[b], block_size, D, s);
+      const int n = nloc_blocks(seq_lens[b], block_size, D, s, shard_rule);
       pages[s] += n;
       if (n > mx) mx = n;
     }
@@ -169,30 +184,32 @@ dcp_status dcp_block_table_extent(const int32_t* seq_lens, int32_t batch, int32_
   return DCP_OK;
 }
 
-dcp_status dcp_build_block_table(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
-                                 uint64_t perm_seed, int32_t max_local_blocks, int32_t* tables, int32_t* local_len) {
+dcp_status dcp_block_table_extent(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                  int32_t* max_local_blocks, int32_t* num_pages) {
+  return dcp_block_table_extent_rule(seq_lens, batch, block_size, D, DCP_SHARD_INTERLEAVED, max_local_blocks,
+                                     num_pages);
+}
+
+dcp_status dcp_build_block_table_rule(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                      int32_t shard_rule, uint64_t perm_seed, int32_t max_local_blocks,
+                                      int32_t* tables, int32_t* local_len) {
   if (seq_lens == nullptr || tables == nullptr || batch < 0 || block_size <= 0 || D < 1 || D > kMaxShardsHost ||
-      max_local_blocks < 0)
+      max_local_blocks < 0 || (shard_rule != DCP_SHARD_INTERLEAVED && shard_rule != DCP_SHARD_CONTIGUOUS))
     return DCP_ERR_INVALID_ARG;
   for (int b = 0; b < batch; ++b)
     if (seq_lens[b] < 0) return DCP_ERR_INVALID_ARG;
   for (int b = 0; b < batch; ++b)
     for (int s = 0; s < D; ++s)
-      if (nloc_blocks(seq_lens[b], block_size, D, s) > max_local_blocks) return DCP_ERR_CAPACITY;
+      if (nloc_blocks(seq_lens[b], block_size, D, s, shard_rule) > max_local_blocks) return DCP_ERR_CAPACITY;
   for (int s = 0; s < D; ++s) {
     int32_t next = 0;
     for (int b = 0; b < batch; ++b) {
       const int64_t len = seq_lens[b];
-      const int64_t nblk = (len + block_size - 1) / block_size;
-      const int n = nloc_blocks(len, block_size, D, s);
+      const int n = nloc_blocks(len, block_size, D, s, shard_rule);
       int32_t* row = tables + ((size_t)s * batch + b) * max_local_blocks;
       for (int j = 0; j < max_local_blocks; ++j) row[j] = j < n ? next + j : -1;
       next += n;
-      if (local_len != nullptr) {
-        int64_t toks = (int64_t)n * block_size;
-        if (n > 0 && (nblk - 1) % D == s) toks -= nblk * block_size - len;  // partial last block
-        local_len[(size_t)s * batch + b] = (int32_t)toks;
-      }
+      if (local_len != nullptr) local_len[(size_t)s * batch + b] = (int32_t)nloc_tokens(len, block_size, D, s, shard_rule);
     }
     if (perm_seed != 0 && next > 1) {
       std::vector<int32_t> pi(next);
@@ -215,6 +232,12 @@ dcp_status dcp_build_block_table(const int32_t* seq_lens, int32_t batch, int32_t
     }
   }
   return DCP_OK;
+}
+
+dcp_status dcp_build_block_table(const int32_t* seq_lens, int32_t batch, int32_t block_size, int32_t D,
+                                 uint64_t perm_seed, int32_t max_local_blocks, int32_t* tables, int32_t* local_len) {
+  return dcp_build_block_table_rule(seq_lens, batch, block_size, D, DCP_SHARD_INTERLEAVED, perm_seed,
+                                    max_local_blocks, tables, local_len);
 }
 
 size_t dcp_kv_page_bytes(const dcp_attn_desc* desc) {
@@ -241,8 +264,8 @@ dcp_status dcp_place_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_src
     if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
   }
   if ((reinterpret_cast<uintptr_t>(kv_src) & 15u) != 0) return DCP_ERR_INVALID_ARG;
-  return launch_place_kv(*desc, D, kv_src, cu_seqlens, nullptr, tables, kv_pools, pool_pages, device_error, false,
-                         static_cast<cudaStream_t>(stream));
+  return launch_place_kv(*desc, D, kv_src, cu_seqlens, nullptr, seq_lens, tables, kv_pools, pool_pages, device_error,
+                         false, static_cast<cudaStream_t>(stream));
 }
 
 dcp_status dcp_grow_block_table(const int32_t* old_seq_lens, const int32_t* new_seq_lens, int32_t batch,
@@ -288,14 +311,16 @@ dcp_status dcp_append_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_ne
     return DCP_ERR_INVALID_ARG;
   dcp_status why;
   if (!desc_supported(*desc, D, &why)) return why;
+  // under the contiguous rule a token's shard depends on the request's final length
+  if (desc->shard_rule != DCP_SHARD_INTERLEAVED) return DCP_ERR_UNSUPPORTED;
   for (int s = 0; s < D; ++s) {
     if (tables[s] == nullptr || pool_pages[s] < 0 || (pool_pages[s] > 0 && kv_pools[s] == nullptr))
       return DCP_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(kv_pools[s]) & 15u) != 0) return DCP_ERR_INVALID_ARG;
   }
   if ((reinterpret_cast<uintptr_t>(kv_new) & 15u) != 0) return DCP_ERR_INVALID_ARG;
-  return launch_place_kv(*desc, D, kv_new, cu_rows, first_pos, tables, kv_pools, pool_pages, device_error, true,
-                         static_cast<cudaStream_t>(stream));
+  return launch_place_kv(*desc, D, kv_new, cu_rows, first_pos, nullptr, tables, kv_pools, pool_pages, device_error,
+                         true, static_cast<cudaStream_t>(stream));
 }
 
 size_t dcp_decode_workspace_bytes(const dcp_attn_desc* desc, int32_t D) {

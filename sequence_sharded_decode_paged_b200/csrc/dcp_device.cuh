@@ -227,9 +227,21 @@ struct SegmentInfo {
   int n;       // pages of the segment
 };
 
-__device__ __forceinline__ int local_pages(int seq_len, int bs, int D, int shard) {
+// Shard rules (the descriptor's shard_rule): 0 = interleaved, block g -> shard g % D as local
+// block g / D; 1 = contiguous chunks, shard s holds the blocks [chunk_begin(s), chunk_begin(s+1))
+// with chunk_begin(s) = floor(s * nblk / D), local block g - chunk_begin(s).
+__device__ __forceinline__ int chunk_begin(int nblk, int D, int s) { return (int)(((long long)s * nblk) / D); }
+
+__device__ __forceinline__ int local_pages(int seq_len, int bs, int D, int shard, int rule) {
   const int nblk = (seq_len + bs - 1) / bs;
+  if (rule != 0) return chunk_begin(nblk, D, shard + 1) - chunk_begin(nblk, D, shard);
   return nblk > shard ? (nblk - 1 - shard) / D + 1 : 0;
+}
+
+// Logical block of local page j of `shard` in a request of seq_len tokens.
+__device__ __forceinline__ int global_block(int j, int seq_len, int bs, int D, int shard, int rule) {
+  if (rule != 0) return chunk_begin((seq_len + bs - 1) / bs, D, shard) + j;
+  return j * D + shard;
 }
 
 // First CTA that works on a segment, and the last one.  An empty segment
@@ -254,7 +266,7 @@ struct CtaPlan {
 // Block-wide planner.  Every thread of the block must call it.  `scratch`
 // holds at least (blockDim.x / 32 + 4) ints of shared memory.
 __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens, int B, int n_si,
-                                            const int* shard_of_si, int bs, int D, int cta, int nctas,
+                                            const int* shard_of_si, int bs, int D, int rule, int cta, int nctas,
                                             int* scratch) {
   const int S = n_si * B;
   const int nt = blockDim.x;
@@ -265,7 +277,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
   int local = 0;
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
-    local += local_pages(seq_lens[b], bs, D, shard_of_si[si]);
+    local += local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
   }
   // block exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
@@ -300,7 +312,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
   // first segment whose last CTA is >= cta (monotone in sid)
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
-    const int n = local_pages(seq_lens[b], bs, D, shard_of_si[si]);
+    const int n = local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
     if (seg_last_cta(pre, n, T, P) >= cta) {
       atomicMin(&scratch[nw + 1], sid);
       break;
@@ -318,7 +330,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
     int p2 = scratch[warp] + incl - local;
     for (int sid = s_begin; sid < plan.sid0; ++sid) {
       const int si = sid / B, b = sid - si * B;
-      p2 += local_pages(seq_lens[b], bs, D, shard_of_si[si]);
+      p2 += local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
     }
     scratch[nw + 2] = p2;
   }

@@ -64,6 +64,7 @@ struct GqaParams {
   float v_scale;  // multiplies O (FP8 cache); 1 for bf16
   int n_si, B, Hq, Hkv, G, bs, D, mlb;
   int q_len, R, rt;  // query tokens per request, rows per KV head (q_len * G), 16-row tiles per head
+  int rule;          // shard rule (interleaved / contiguous)
   int hpc, n_hg, stages, wph;
   uint32_t stage_bytes;
   int slot_floats;
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       if (p.pool_pages[si] > 0) prefetch_tmap(&p.tmap[si]);
   __syncthreads();
 
-  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, bs, D, cta, nctas, scratch);
+  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, bs, D, p.rule, cta, nctas, scratch);
   const int T = plan.T, P = plan.P;
   const int lo = cta * P, hi = min(lo + P, T);
   const int S = p.n_si * B;
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     int pre = plan.pre0;
     for (int sid = plan.sid0; sid < S && !aborted; ++sid) {
       const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
-      const int n = local_pages(p.seq_lens[b], bs, D, shard);
+      const int n = local_pages(p.seq_lens[b], bs, D, shard, p.rule);
       if (seg_first_cta(pre, n, T, P) > cta) break;
       const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
       const int32_t* trow = p.table[si] + (size_t)b * p.mlb;
@@ -310,7 +311,10 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   for (int sid = plan.sid0; sid < S; ++sid) {
     const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
     const int seq_len = p.seq_lens[b];
-    const int n = local_pages(seq_len, bs, D, shard);
+    const int n = local_pages(seq_len, bs, D, shard, p.rule);
+    // logical block of local page j: g0 + j * gs (interleaved: shard + j * D; contiguous: chunk start + j)
+    const int gs = p.rule != 0 ? 1 : D;
+    const int g0 = global_block(0, seq_len, bs, D, shard, p.rule);
     const int c0 = seg_first_cta(pre, n, T, P);
     if (c0 > cta) break;
     const int c1 = seg_last_cta(pre, n, T, P);
@@ -399,8 +403,8 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           }
           if (!dead && active) {
             const bool ok0 = stage_ok[st0] != 0, ok1 = stage_ok[st1] != 0;
-            const int v0 = min(16, seq_len - (j * D + shard) * 16);
-            const int v1 = min(16, seq_len - ((j + 1) * D + shard) * 16);
+            const int t0a = (g0 + j * gs) * 16, t0b = (g0 + (j + 1) * gs) * 16;
+            const int v0 = min(16, seq_len - t0a), v1 = min(16, seq_len - t0b);
             const uint32_t kb0 = smem_u32(stage_mem + (size_t)st0 * p.stage_bytes);
             const uint32_t kb1 = smem_u32(stage_mem + (size_t)st1 * p.stage_bytes);
             float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -413,7 +417,6 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
               if (ok1) bf16_scores(kb1, box_bytes, (uint32_t)(hh * 16), lane, qa, sb);
             }
             // visible tokens of each page for rows g4 / g4 + 8 (a page that was not loaded adds nothing)
-            const int t0a = (j * D + shard) * 16, t0b = ((j + 1) * D + shard) * 16;
             const int va0 = !ok0 ? 0 : (MULTI ? lim0 - t0a : v0), va1 = !ok0 ? 0 : (MULTI ? lim1 - t0a : v0);
             const int vb0 = !ok1 ? 0 : (MULTI ? lim0 - t0b : v1), vb1 = !ok1 ? 0 : (MULTI ? lim1 - t0b : v1);
 #pragma unroll
@@ -504,7 +507,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
         dead = true;
       }
       if (!dead && active && ((j - a) % wph) == sub && stage_ok[stage]) {
-        const int gblk = j * D + shard;
+        const int gblk = g0 + j * gs;
         const int valid = min(bs, seq_len - gblk * bs);
         const uint32_t kbase = smem_u32(stage_mem + (size_t)stage * p.stage_bytes);
         const uint32_t vbase = kbase + Geo::kBoxes * box_bytes;
@@ -782,6 +785,7 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.D = D;
   p.mlb = d.max_local_blocks;
   p.q_len = d.q_len;
+  p.rule = d.shard_rule;
   p.R = p.G * p.q_len;
   p.rt = gqa_row_tiles(p.G, p.q_len);
   const int eb = KV8 ? 1 : 2;  // bytes per cached element

@@ -53,8 +53,9 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
 dcp_status launch_lse_merge(const float* const* O_parts, const float* const* LSE_parts, int D, int rows, int d_v,
                             float* O, float* LSE_out, cudaStream_t st);
 dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, const int64_t* cu_seqlens,
-                           const int32_t* token_begin, const int32_t* const* tables, void* const* pools,
-                           const int32_t* pool_pages, int32_t* device_error, bool few_rows, cudaStream_t st);
+                           const int32_t* token_begin, const int32_t* seq_lens, const int32_t* const* tables,
+                           void* const* pools, const int32_t* pool_pages, int32_t* device_error, bool few_rows,
+                           cudaStream_t st);
 
 // GQA geometry helpers (shared by the workspace sizing and the launcher).
 int gqa_row_tiles(int G, int q_len);

@@ -106,6 +106,7 @@ struct MlaParams {
   float* slots;
   float scale_log2;
   int n_si, B, D, mlb, slot_floats, q_len;
+  int rule;  // shard rule (interleaved / contiguous)
 };
 
 namespace {
@@ -185,7 +186,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
   tc_fence_after();
   const uint32_t tbase = misc->tmem_base;
 
-  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, kMlaBs, D, cta, nctas, misc->scratch);
+  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, kMlaBs, D, p.rule, cta, nctas, misc->scratch);
   const int T = plan.T, P = plan.P;
   const int lo = cta * P, hi = min(lo + P, T);
   const int S = p.n_si * B;
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       int pre = plan.pre0;
       for (int sid = plan.sid0; sid < S; ++sid) {
         const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
-        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard);
+        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard, p.rule);
         if (seg_first_cta(pre, n, T, P) > cta) break;
         const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
         pre += n;
@@ -290,7 +291,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           }
           if (w_sid >= S) { w_live = false; break; }
           const int si2 = w_sid / B, b2 = w_sid - si2 * B;
-          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2]);
+          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2], p.rule);
           if (seg_first_cta(w_pre, n2, T, P) > cta) { w_live = false; break; }
           w_si = si2;
           w_b = b2;
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     for (int sid = plan.sid0; sid < S; ++sid) {
       const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
       const int seq_len = p.seq_lens[b];
-      const int n = local_pages(seq_len, kMlaBs, D, shard);
+      const int n = local_pages(seq_len, kMlaBs, D, shard, p.rule);
       const int c0 = seg_first_cta(pre, n, T, P);
       if (c0 > cta) break;
       const int c1 = seg_last_cta(pre, n, T, P);
@@ -422,8 +423,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       for (int j = a; j < e; ++j) {
         int page;
         const bool ok = page_ok(p, si, b, j, &page);
-        const int valid = min(kMlaBs, seq_len - (j * D + shard) * kMlaBs);
-        const int vis = lim - (j * D + shard) * kMlaBs;  // visible tokens of this page (may be <= 0)
+        const int tok0 = global_block(j, seq_len, kMlaBs, D, shard, p.rule) * kMlaBs;  // first token of the page
+        const int valid = min(kMlaBs, seq_len - tok0);
+        const int vis = lim - tok0;  // visible tokens of this page (may be <= 0)
         const uint32_t sb = gpage & 1u;
         wait_or_die_warp(&misc->s_full[sb], (gpage >> 1) & 1u, dead, p.status);
         tc_fence_after();
@@ -672,6 +674,7 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   p.slot_floats = L.slot_floats;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.q_len = d.q_len;
+  p.rule = d.shard_rule;
   p.seq_lens = seq_lens;
   p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
   p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);

@@ -5,6 +5,9 @@
 // block g / D and lives in the physical page that the shard's block table
 // names.  This is the cache write that precedes decoding; it is a pure copy.
 //
+// Under the contiguous shard rule a token's shard and local block follow from
+// its request's length (seq_lens): shard s holds the blocks
+// [floor(s * nblk / D), floor((s + 1) * nblk / D)).
 // Bulk placement (place_kv_kernel): one warp per source row (token); the warp
 // finds its request by binary search over cu_seqlens, then copies the row with
 // 16-byte loads and stores.
@@ -32,6 +35,8 @@ struct PlaceParams {
   int32_t* err;
   int layout, B, Hkv, d, bs, D, mlb;
   int eb;            // bytes per pool element: 2 (bf16) or 1 (FP8 code)
+  int rule;          // shard rule: 0 interleaved, 1 contiguous chunks (needs seq_lens)
+  const int32_t* seq_lens;
   float inv_k, inv_v;  // FP8: multipliers applied before rounding to E4M3
 };
 
@@ -51,8 +56,17 @@ __device__ __forceinline__ bool row_slot(const PlaceParams& p, long r, bool repo
     return false;
   }
   const long g = t / p.bs;
-  const int s = (int)(g % p.D);
-  const long j = g / p.D;
+  int s;
+  long j;
+  if (p.rule == 0) {
+    s = (int)(g % p.D);
+    j = g / p.D;
+  } else {  // the chunk of the request's blocks that holds g
+    const int nblk = (p.seq_lens[b] + p.bs - 1) / p.bs;
+    s = 0;
+    while (s < p.D - 1 && g >= chunk_begin(nblk, p.D, s + 1)) ++s;
+    j = g - chunk_begin(nblk, p.D, s);
+  }
   const int slot = (int)(t % p.bs);
   const int page = (j < p.mlb) ? p.table[s][(size_t)b * p.mlb + j] : -1;
   if (page < 0 || page >= p.pool_pages[s]) {
@@ -121,8 +135,9 @@ __global__ void __launch_bounds__(256) place_kv_kernel(const __grid_constant__ P
 }
 
 dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, const int64_t* cu_seqlens,
-                           const int32_t* token_begin, const int32_t* const* tables, void* const* pools,
-                           const int32_t* pool_pages, int32_t* device_error, bool few_rows, cudaStream_t st) {
+                           const int32_t* token_begin, const int32_t* seq_lens, const int32_t* const* tables,
+                           void* const* pools, const int32_t* pool_pages, int32_t* device_error, bool few_rows,
+                           cudaStream_t st) {
   PlaceParams p;
   memset(&p, 0, sizeof(p));
   for (int s = 0; s < D; ++s) {
@@ -142,6 +157,9 @@ dcp_status launch_place_kv(const dcp_attn_desc& d, int D, const void* kv_src, co
   p.D = D;
   p.mlb = d.max_local_blocks;
   p.eb = kv_elem_bytes(d);
+  p.rule = d.shard_rule;
+  p.seq_lens = seq_lens;
+  if (p.rule != 0 && seq_lens == nullptr) return DCP_ERR_INVALID_ARG;
   p.inv_k = p.eb == 1 ? 1.0f / d.k_scale : 1.f;
   p.inv_v = p.eb == 1 ? 1.0f / d.v_scale : 1.f;
   if (few_rows) {

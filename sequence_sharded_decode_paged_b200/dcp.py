@@ -22,8 +22,10 @@ LIB_PATH = os.path.join(_HERE, "libdcp.so")
 DCP_OK, DCP_ERR_INVALID_ARG, DCP_ERR_UNSUPPORTED, DCP_ERR_CAPACITY, DCP_ERR_CUDA, DCP_ERR_DEVICE = range(6)
 DCP_LAYOUT_GQA, DCP_LAYOUT_MLA = 0, 1
 DCP_KV_BF16, DCP_KV_FP8_E4M3 = 0, 1
+DCP_SHARD_INTERLEAVED, DCP_SHARD_CONTIGUOUS = 0, 1
 
 EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_build_block_table",
+            "dcp_block_table_extent_rule", "dcp_build_block_table_rule",
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
             "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_grow_block_table", "dcp_append_kv"]
@@ -39,7 +41,8 @@ class dcp_attn_desc(C.Structure):
     _fields_ = [("layout", C.c_int32), ("batch", C.c_int32), ("num_q_heads", C.c_int32),
                 ("num_kv_heads", C.c_int32), ("head_dim_qk", C.c_int32), ("head_dim_v", C.c_int32),
                 ("block_size", C.c_int32), ("max_local_blocks", C.c_int32), ("softmax_scale", C.c_float),
-                ("q_len", C.c_int32), ("kv_dtype", C.c_int32), ("k_scale", C.c_float), ("v_scale", C.c_float)]
+                ("q_len", C.c_int32), ("kv_dtype", C.c_int32), ("k_scale", C.c_float), ("v_scale", C.c_float),
+                ("shard_rule", C.c_int32)]
 
 
 def _load() -> C.CDLL:
@@ -53,6 +56,8 @@ def _load() -> C.CDLL:
         "dcp_status_string": (C.c_char_p, [C.c_int]),
         "dcp_block_table_extent": (C.c_int, [p, i32, i32, i32, p, p]),
         "dcp_build_block_table": (C.c_int, [p, i32, i32, i32, u64, i32, p, p]),
+        "dcp_block_table_extent_rule": (C.c_int, [p, i32, i32, i32, i32, p, p]),
+        "dcp_build_block_table_rule": (C.c_int, [p, i32, i32, i32, i32, u64, i32, p, p]),
         "dcp_kv_page_bytes": (sz, [p]),
         "dcp_place_kv": (C.c_int, [p, i32, p, p, p, p, p, p, p, p]),
         "dcp_decode_workspace_bytes": (sz, [p, i32]),
@@ -110,9 +115,9 @@ def _i32(a) -> np.ndarray:
 
 def make_desc(layout: int, batch: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
               block_size: int, max_local_blocks: int, softmax_scale: float, q_len: int = 1,
-              kv_dtype: int = 0, k_scale: float = 1.0, v_scale: float = 1.0) -> dcp_attn_desc:
+              kv_dtype: int = 0, k_scale: float = 1.0, v_scale: float = 1.0, shard_rule: int = 0) -> dcp_attn_desc:
     return dcp_attn_desc(layout, batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v, block_size,
-                         max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale, v_scale)
+                         max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale, v_scale, shard_rule)
 
 
 # --------------------------------------------------------------------------- host calls
@@ -120,26 +125,35 @@ def dcp_version() -> int:
     return _lib.dcp_version()
 
 
-def dcp_block_table_extent(seq_lens: Sequence[int], block_size: int, D: int):
+def dcp_block_table_extent(seq_lens: Sequence[int], block_size: int, D: int, shard_rule: int = 0):
     sl = _i32(seq_lens)
     mlb = C.c_int32(0)
     pages = np.zeros(D, dtype=np.int32)
-    _check("dcp_block_table_extent", _lib.dcp_block_table_extent(
-        sl.ctypes.data, sl.shape[0], block_size, D, C.addressof(mlb), pages.ctypes.data))
+    if shard_rule == DCP_SHARD_INTERLEAVED:
+        rc = _lib.dcp_block_table_extent(sl.ctypes.data, sl.shape[0], block_size, D, C.addressof(mlb),
+                                         pages.ctypes.data)
+    else:
+        rc = _lib.dcp_block_table_extent_rule(sl.ctypes.data, sl.shape[0], block_size, D, shard_rule,
+                                              C.addressof(mlb), pages.ctypes.data)
+    _check("dcp_block_table_extent", rc)
     return int(mlb.value), pages
 
 
 def dcp_build_block_table(seq_lens: Sequence[int], block_size: int, D: int, perm_seed: int = 0,
-                          max_local_blocks: Optional[int] = None):
+                          max_local_blocks: Optional[int] = None, shard_rule: int = 0):
     """Returns ``(tables int32[D][B][max_local_blocks], local_len int32[D][B])``."""
     sl = _i32(seq_lens)
     if max_local_blocks is None:
-        max_local_blocks = max(1, dcp_block_table_extent(sl, block_size, D)[0])
+        max_local_blocks = max(1, dcp_block_table_extent(sl, block_size, D, shard_rule)[0])
     tables = np.empty((D, sl.shape[0], max_local_blocks), dtype=np.int32)
     local_len = np.empty((D, sl.shape[0]), dtype=np.int32)
-    _check("dcp_build_block_table", _lib.dcp_build_block_table(
-        sl.ctypes.data, sl.shape[0], block_size, D, perm_seed, max_local_blocks, tables.ctypes.data,
-        local_len.ctypes.data))
+    if shard_rule == DCP_SHARD_INTERLEAVED:
+        rc = _lib.dcp_build_block_table(sl.ctypes.data, sl.shape[0], block_size, D, perm_seed, max_local_blocks,
+                                        tables.ctypes.data, local_len.ctypes.data)
+    else:
+        rc = _lib.dcp_build_block_table_rule(sl.ctypes.data, sl.shape[0], block_size, D, shard_rule, perm_seed,
+                                             max_local_blocks, tables.ctypes.data, local_len.ctypes.data)
+    _check("dcp_build_block_table", rc)
     return tables, local_len
 
 

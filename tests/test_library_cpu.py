@@ -172,7 +172,7 @@ def test_q_len_validation_and_workspace_growth():
 
 def test_descriptor_layout_matches_header():
     import ctypes
-    assert ctypes.sizeof(dcp.dcp_attn_desc) == 13 * 4
+    assert ctypes.sizeof(dcp.dcp_attn_desc) == 14 * 4
     assert dcp.dcp_attn_desc.q_len.offset == 36
     assert dcp.dcp_attn_desc.v_scale.offset == 48
 
@@ -187,3 +187,34 @@ def test_fp8_rejected_for_mla_and_head_dim_64():
         assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1,
                                                    dcp.DCP_KV_FP8_E4M3, ks, vs)) == 0
     assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1, 7)) == 0
+
+
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 8, 16])
+@pytest.mark.parametrize("bs", [16, 64])
+@pytest.mark.parametrize("perm", [0, 99])
+def test_contiguous_tables_bit_exact_vs_oracle(D, bs, perm):
+    rng = np.random.default_rng(D * 2000 + bs + perm)
+    seq_lens = list(rng.integers(0, 3000, size=9)) + [0, 1, bs, bs + 1, D * bs, D * bs + 1, (D - 1) * bs + 1]
+    C = dcp.DCP_SHARD_CONTIGUOUS
+    t_lib, l_lib = dcp.dcp_build_block_table(seq_lens, bs, D, perm, shard_rule=C)
+    mlb, pages = dcp.dcp_block_table_extent(seq_lens, bs, D, C)
+    t_or, l_or, p_or = oracle.block_tables(seq_lens, bs, D, perm_seed=perm, max_local_blocks=t_lib.shape[2],
+                                           rule=oracle.CONTIGUOUS)
+    np.testing.assert_array_equal(t_lib, t_or)
+    np.testing.assert_array_equal(l_lib, l_or)
+    np.testing.assert_array_equal(pages, p_or)
+    assert mlb == int((t_or >= 0).sum(axis=2).max())
+
+
+def test_contiguous_rule_argument_checks():
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_build_block_table([100], 16, 2, 0, shard_rule=2)
+    assert e.value.status == dcp.DCP_ERR_INVALID_ARG
+    bad = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 4, 0.125, shard_rule=5)
+    assert dcp.dcp_decode_workspace_bytes(bad, 2) == 0
+    ok = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 4, 0.125, shard_rule=dcp.DCP_SHARD_CONTIGUOUS)
+    assert dcp.dcp_decode_workspace_bytes(ok, 2) > 0
+    # contiguous tables cannot grow: appending is refused before anything runs
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_append_kv(ok, 2, 16, 16, 16, [16, 16], [16, 16], [1, 1])
+    assert e.value.status == dcp.DCP_ERR_UNSUPPORTED

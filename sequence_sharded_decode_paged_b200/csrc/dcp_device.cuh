@@ -232,10 +232,12 @@ struct SegmentInfo {
 // with chunk_begin(s) = floor(s * nblk / D), local block g - chunk_begin(s).
 __device__ __forceinline__ int chunk_begin(int nblk, int D, int s) { return (int)(((long long)s * nblk) / D); }
 
-__device__ __forceinline__ int local_pages(int seq_len, int bs, int D, int shard, int rule) {
+// Local pages of `shard` in a request of seq_len tokens (kernels are instantiated per rule).
+template <int RULE>
+__device__ __forceinline__ int local_pages_r(int seq_len, int bs, int D, int shard) {
   const int nblk = (seq_len + bs - 1) / bs;
-  if (rule != 0) return chunk_begin(nblk, D, shard + 1) - chunk_begin(nblk, D, shard);
-  return nblk > shard ? (nblk - 1 - shard) / D + 1 : 0;
+  if constexpr (RULE != 0) return chunk_begin(nblk, D, shard + 1) - chunk_begin(nblk, D, shard);
+  else return nblk > shard ? (nblk - 1 - shard) / D + 1 : 0;
 }
 
 // Logical block of local page j of `shard` in a request of seq_len tokens.
@@ -263,11 +265,12 @@ struct CtaPlan {
   int pre0;     // its first page in the concatenation
 };
 
-// Block-wide planner.  Every thread of the block must call it.  `scratch`
+// Block-wide planner for shard rule RULE.  Every thread of the block must call it.  `scratch`
 // holds at least (blockDim.x / 32 + 4) ints of shared memory.
-__device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens, int B, int n_si,
-                                            const int* shard_of_si, int bs, int D, int rule, int cta, int nctas,
-                                            int* scratch) {
+template <int RULE>
+__device__ __forceinline__ CtaPlan plan_cta_r(const int32_t* __restrict__ seq_lens, int B, int n_si,
+                                              const int* shard_of_si, int bs, int D, int cta, int nctas,
+                                              int* scratch) {
   const int S = n_si * B;
   const int nt = blockDim.x;
   const int tid = threadIdx.x;
@@ -277,7 +280,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
   int local = 0;
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
-    local += local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
+    local += local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
   }
   // block exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
@@ -312,7 +315,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
   // first segment whose last CTA is >= cta (monotone in sid)
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
-    const int n = local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
+    const int n = local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
     if (seg_last_cta(pre, n, T, P) >= cta) {
       atomicMin(&scratch[nw + 1], sid);
       break;
@@ -330,7 +333,7 @@ __device__ __forceinline__ CtaPlan plan_cta(const int32_t* __restrict__ seq_lens
     int p2 = scratch[warp] + incl - local;
     for (int sid = s_begin; sid < plan.sid0; ++sid) {
       const int si = sid / B, b = sid - si * B;
-      p2 += local_pages(seq_lens[b], bs, D, shard_of_si[si], rule);
+      p2 += local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
     }
     scratch[nw + 2] = p2;
   }

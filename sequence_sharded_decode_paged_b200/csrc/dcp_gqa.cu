@@ -64,7 +64,6 @@ struct GqaParams {
   float v_scale;  // multiplies O (FP8 cache); 1 for bf16
   int n_si, B, Hq, Hkv, G, bs, D, mlb;
   int q_len, R, rt;  // query tokens per request, rows per KV head (q_len * G), 16-row tiles per head
-  int rule;          // shard rule (interleaved / contiguous)
   int hpc, n_hg, stages, wph;
   uint32_t stage_bytes;
   int slot_floats;
@@ -199,8 +198,8 @@ __device__ __forceinline__ uint32_t keep_hi(int c4, int vrem) {  // tokens 2c+8,
 
 // MULTI: multi-token decode (q_len > 1, per-row causal limits); the single-token
 // instantiation keeps the plain end-of-sequence mask and its register budget.
-// KV8: the pools hold FP8 E4M3 codes.
-template <int HEAD_DIM, bool MULTI, bool KV8>
+// KV8: the pools hold FP8 E4M3 codes.  RULE: the shard rule (0 interleaved, 1 contiguous chunks).
+template <int HEAD_DIM, bool MULTI, bool KV8, int RULE>
 __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid_constant__ GqaParams p) {
   using Geo = GqaGeom<HEAD_DIM, KV8>;
   static_assert(!KV8 || HEAD_DIM == 128, "FP8 pages use one 128-byte row per token and head");
@@ -234,7 +233,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       if (p.pool_pages[si] > 0) prefetch_tmap(&p.tmap[si]);
   __syncthreads();
 
-  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, bs, D, p.rule, cta, nctas, scratch);
+  const CtaPlan plan = plan_cta_r<RULE>(p.seq_lens, B, p.n_si, p.shard_of_si, bs, D, cta, nctas, scratch);
   const int T = plan.T, P = plan.P;
   const int lo = cta * P, hi = min(lo + P, T);
   const int S = p.n_si * B;
@@ -249,7 +248,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     int pre = plan.pre0;
     for (int sid = plan.sid0; sid < S && !aborted; ++sid) {
       const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
-      const int n = local_pages(p.seq_lens[b], bs, D, shard, p.rule);
+      const int n = local_pages_r<RULE>(p.seq_lens[b], bs, D, shard);
       if (seg_first_cta(pre, n, T, P) > cta) break;
       const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
       const int32_t* trow = p.table[si] + (size_t)b * p.mlb;
@@ -311,10 +310,10 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   for (int sid = plan.sid0; sid < S; ++sid) {
     const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
     const int seq_len = p.seq_lens[b];
-    const int n = local_pages(seq_len, bs, D, shard, p.rule);
-    // logical block of local page j: g0 + j * gs (interleaved: shard + j * D; contiguous: chunk start + j)
-    const int gs = p.rule != 0 ? 1 : D;
-    const int g0 = global_block(0, seq_len, bs, D, shard, p.rule);
+    const int n = local_pages_r<RULE>(seq_len, bs, D, shard);
+    // logical block of local page j: g0 + j * gstride (interleaved: shard + j * D; contiguous: chunk start + j)
+    const int g0 = global_block(0, seq_len, bs, D, shard, RULE);
+    const int gstride = RULE != 0 ? 1 : D;
     const int c0 = seg_first_cta(pre, n, T, P);
     if (c0 > cta) break;
     const int c1 = seg_last_cta(pre, n, T, P);
@@ -403,7 +402,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           }
           if (!dead && active) {
             const bool ok0 = stage_ok[st0] != 0, ok1 = stage_ok[st1] != 0;
-            const int t0a = (g0 + j * gs) * 16, t0b = (g0 + (j + 1) * gs) * 16;
+            const int t0a = (g0 + j * gstride) * 16, t0b = (g0 + (j + 1) * gstride) * 16;
             const int v0 = min(16, seq_len - t0a), v1 = min(16, seq_len - t0b);
             const uint32_t kb0 = smem_u32(stage_mem + (size_t)st0 * p.stage_bytes);
             const uint32_t kb1 = smem_u32(stage_mem + (size_t)st1 * p.stage_bytes);
@@ -507,7 +506,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
         dead = true;
       }
       if (!dead && active && ((j - a) % wph) == sub && stage_ok[stage]) {
-        const int gblk = g0 + j * gs;
+        const int gblk = g0 + j * gstride;
         const int valid = min(bs, seq_len - gblk * bs);
         const uint32_t kbase = smem_u32(stage_mem + (size_t)stage * p.stage_bytes);
         const uint32_t vbase = kbase + Geo::kBoxes * box_bytes;
@@ -785,7 +784,6 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.D = D;
   p.mlb = d.max_local_blocks;
   p.q_len = d.q_len;
-  p.rule = d.shard_rule;
   p.R = p.G * p.q_len;
   p.rt = gqa_row_tiles(p.G, p.q_len);
   const int eb = KV8 ? 1 : 2;  // bytes per cached element
@@ -822,7 +820,8 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
     }
   }
   const size_t smem = (size_t)p.stages * p.stage_bytes + fixed;
-  auto kern = gqa_decode_kernel<HEAD_DIM, MULTI, KV8>;
+  auto kern = d.shard_rule == DCP_SHARD_INTERLEAVED ? gqa_decode_kernel<HEAD_DIM, MULTI, KV8, 0>
+                                                    : gqa_decode_kernel<HEAD_DIM, MULTI, KV8, 1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return DCP_ERR_CUDA;
   dim3 grid(L.nctas, p.n_hg);

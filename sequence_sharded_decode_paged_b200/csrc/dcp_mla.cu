@@ -106,7 +106,6 @@ struct MlaParams {
   float* slots;
   float scale_log2;
   int n_si, B, D, mlb, slot_floats, q_len;
-  int rule;  // shard rule (interleaved / contiguous)
 };
 
 namespace {
@@ -145,6 +144,8 @@ __device__ __forceinline__ bool page_ok(const MlaParams& p, int si, int b, int j
 
 }  // namespace
 
+// RULE: the shard rule (0 interleaved, 1 contiguous chunks), fixed at compile time.
+template <int RULE>
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid_constant__ MlaParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
   tc_fence_after();
   const uint32_t tbase = misc->tmem_base;
 
-  const CtaPlan plan = plan_cta(p.seq_lens, B, p.n_si, p.shard_of_si, kMlaBs, D, p.rule, cta, nctas, misc->scratch);
+  const CtaPlan plan = plan_cta_r<RULE>(p.seq_lens, B, p.n_si, p.shard_of_si, kMlaBs, D, cta, nctas, misc->scratch);
   const int T = plan.T, P = plan.P;
   const int lo = cta * P, hi = min(lo + P, T);
   const int S = p.n_si * B;
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       int pre = plan.pre0;
       for (int sid = plan.sid0; sid < S; ++sid) {
         const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
-        const int n = local_pages(p.seq_lens[b], kMlaBs, D, shard, p.rule);
+        const int n = local_pages_r<RULE>(p.seq_lens[b], kMlaBs, D, shard);
         if (seg_first_cta(pre, n, T, P) > cta) break;
         const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
         pre += n;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           }
           if (w_sid >= S) { w_live = false; break; }
           const int si2 = w_sid / B, b2 = w_sid - si2 * B;
-          const int n2 = local_pages(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2], p.rule);
+          const int n2 = local_pages_r<RULE>(p.seq_lens[b2], kMlaBs, D, p.shard_of_si[si2]);
           if (seg_first_cta(w_pre, n2, T, P) > cta) { w_live = false; break; }
           w_si = si2;
           w_b = b2;
@@ -399,13 +400,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     for (int sid = plan.sid0; sid < S; ++sid) {
       const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
       const int seq_len = p.seq_lens[b];
-      const int n = local_pages(seq_len, kMlaBs, D, shard, p.rule);
+      const int n = local_pages_r<RULE>(seq_len, kMlaBs, D, shard);
       const int c0 = seg_first_cta(pre, n, T, P);
       if (c0 > cta) break;
       const int c1 = seg_last_cta(pre, n, T, P);
       float* Oout = p.O[si] + ((size_t)b * ql + jq) * kMlaHeads * kMlaDv;
       float* Lout = p.LSE[si] + ((size_t)b * ql + jq) * kMlaHeads;
       const int lim = seq_len - (ql - 1 - jq);  // tokens this query token sees
+      // logical block of local page j: g0 + j * gstride (computed once per segment)
+      const int g0 = global_block(0, seq_len, kMlaBs, D, shard, RULE);
       if (n == 0) {
         for (int i = ts; i < kMlaHeads * kMlaDv / 4; i += kSoftmaxThreads)
           reinterpret_cast<float4*>(Oout)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -423,7 +426,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       for (int j = a; j < e; ++j) {
         int page;
         const bool ok = page_ok(p, si, b, j, &page);
-        const int tok0 = global_block(j, seq_len, kMlaBs, D, shard, p.rule) * kMlaBs;  // first token of the page
+        const int tok0 = (g0 + j * (RULE != 0 ? 1 : D)) * kMlaBs;  // first token of the page
         const int valid = min(kMlaBs, seq_len - tok0);
         const int vis = lim - tok0;  // visible tokens of this page (may be <= 0)
         const uint32_t sb = gpage & 1u;
@@ -674,7 +677,6 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   p.slot_floats = L.slot_floats;
   p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
   p.q_len = d.q_len;
-  p.rule = d.shard_rule;
   p.seq_lens = seq_lens;
   p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
   p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);
@@ -695,10 +697,10 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
         return DCP_ERR_CUDA;
     }
   }
-  if (cudaFuncSetAttribute(mla_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMlaSmem) !=
-      cudaSuccess)
+  auto kern = d.shard_rule == DCP_SHARD_INTERLEAVED ? mla_decode_kernel<0> : mla_decode_kernel<1>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMlaSmem) != cudaSuccess)
     return DCP_ERR_CUDA;
-  mla_decode_kernel<<<dim3(L.nctas, d.q_len), kMlaThreads, kMlaSmem, stream>>>(p);
+  kern<<<dim3(L.nctas, d.q_len), kMlaThreads, kMlaSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
 }
 

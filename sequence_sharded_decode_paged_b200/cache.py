@@ -1,11 +1,14 @@
-"""D interleaved paged KV shards on one GPU, driven through the C ABI.
+"""D paged KV shards on one GPU, driven through the C ABI.
 
 ``ShardedPagedCache`` owns the device buffers of one decode problem: the D
 shard pools, their block tables, the per-shard partial outputs, the merged
 output and the workspace.  torch only allocates memory here; the tables are
-built by ``dcp_build_block_table``, the cache write is ``dcp_place_kv``, and a
-decode step is ``dcp_decode_partial_all`` (or D ``dcp_decode_partial`` calls)
-followed by ``dcp_lse_merge``.
+built by ``dcp_build_block_table`` (interleaved or contiguous-chunk rule), the
+cache write is ``dcp_place_kv`` (bf16 pools, or FP8 E4M3 codes with per-tensor
+scales), and a decode step is ``dcp_decode_partial_all`` (or D
+``dcp_decode_partial`` calls) followed by ``dcp_lse_merge``.  With ``q_len > 1``
+each request decodes ``q_len`` draft tokens (causal within the draft) and the
+outputs gain a ``q_len`` axis.
 """
 from __future__ import annotations
 

@@ -147,7 +147,7 @@ using namespace dcp;
 
 extern "C" {
 
-int32_t dcp_version(void) { return 100; }
+int32_t dcp_version(void) { return 200; }  // 0.2.0: q_len, kv_dtype, scales and shard_rule in dcp_attn_desc
 
 const char* dcp_status_string(dcp_status s) {
   switch (s) {

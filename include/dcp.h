@@ -31,9 +31,10 @@
  *   - Return value: DCP_OK, or an error code.  Argument errors are detected
  *     on the host before anything is launched (nothing is written then).
  *     DCP_ERR_CUDA means a CUDA runtime call or a launch failed.
- *   - Data types: queries and KV are bf16 (raw 16-bit patterns), outputs
- *     and LSE are fp32, LSE in natural-log units of the SCALED scores,
- *     tables and lengths are int32.
+ *   - Data types: queries and KV sources are bf16 (raw 16-bit patterns);
+ *     pools hold bf16 or FP8 E4M3 codes (dcp_kv_dtype); outputs and LSE are
+ *     fp32, LSE in natural-log units of the SCALED scores; tables and
+ *     lengths are int32.
  *   - Supported shapes (anything else is DCP_ERR_UNSUPPORTED):
  *       GQA: head_dim_qk == head_dim_v in {64, 128}; Hq % Hkv == 0 and
  *            Hq / Hkv <= 16; block_size a multiple of 16 with
@@ -45,6 +46,7 @@
  *       Multi-token decode: 1 <= q_len <= 4 query tokens per request
  *       (GQA and MLA).
  *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA with head_dim 128 only.
+ *       Shard rules: interleaved (default) or contiguous chunks (dcp_shard_rule).
  */
 #ifndef DCP_H
 #define DCP_H

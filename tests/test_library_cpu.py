@@ -218,3 +218,25 @@ def test_contiguous_rule_argument_checks():
     with pytest.raises(dcp.DcpError) as e:
         dcp.dcp_append_kv(ok, 2, 16, 16, 16, [16, 16], [16, 16], [1, 1])
     assert e.value.status == dcp.DCP_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("q_len", [1, 2, 3, 4])
+@pytest.mark.parametrize("rule", [0, 1])
+def test_descriptor_option_matrix(q_len, rule):
+    # every supported combination of draft length, pool type and shard rule sizes its buffers; the shard
+    # rule never changes them, and an FP8 page is half a bf16 page
+    def desc(layout, kv_dtype, Hq=64, Hkv=8, d=128, bs=16):
+        dv = 512 if layout == dcp.DCP_LAYOUT_MLA else d
+        return dcp.make_desc(layout, 8, Hq, Hkv, d, dv, bs, 32, 0.1, q_len, kv_dtype, 0.5, 0.25, rule)
+    g16, g8 = desc(0, 0), desc(0, 1)
+    mla = desc(1, 0, 64, 1, 576, 64)
+    assert dcp.dcp_kv_page_bytes(g8) * 2 == dcp.dcp_kv_page_bytes(g16) > 0
+    assert dcp.dcp_kv_page_bytes(mla) == 64 * 576 * 2
+    for dsc in (g16, g8, mla):
+        ws = dcp.dcp_decode_workspace_bytes(dsc, 4)
+        assert ws > 0
+        other = dcp.dcp_attn_desc.from_buffer_copy(dsc)
+        other.shard_rule = 1 - rule
+        assert dcp.dcp_decode_workspace_bytes(other, 4) == ws
+    assert dcp.dcp_kv_page_bytes(desc(1, 1, 64, 1, 576, 64)) == 0  # FP8 MLA
+    assert dcp.dcp_kv_page_bytes(desc(0, 1, 16, 2, 64)) == 0      # FP8 head_dim 64

@@ -4,12 +4,19 @@
 One step = the whole hot path for one decode token of every request of the
 workload: all D shard partials (one ``dcp_decode_partial_all`` launch)
 followed by the LSE merge (``dcp_lse_merge``), through the C ABI.  Inputs are
-seeded synthetic tensors resident in HBM; L2 is flushed (a write of twice its
-size) before every timed step, outside the timed events.
+seeded synthetic tensors resident in HBM; before every timed step L2 is
+flushed by READING a buffer twice its size (outside the timed events), so the
+previous step's dirty lines are written back before the timer starts.
 
-Default: the GQA 70B-class layer (batch 64, 64 q / 8 KV heads, head_dim 128,
-block 16, lengths 8K-32K) at D = 4; the other D values of the workload are
-measured in the same run and reported under ``other_D``.
+Default: the largest single-GPU workload, the MLA agentic mix (256 requests,
+17.8 M context tokens, 20.5 GB of latent cache) at D = 8; its other D values
+are measured in the same run (``other_D``), and the GQA 70B-class layer at
+D = 4 is measured as a nested line (``extra``).
+
+``e2e`` times the same step through ``dcp_decode_step_host`` -- the C-ABI
+call that takes HOST buffers: every step copies its query, lengths and block
+tables up from pinned host memory and its merged O and LSE back, inside the
+timed region, one step after another on one stream.
 
 ``--impl reference`` times the float64 CPU oracle (the reference arm of this
 build) on a bounded sample of the same workload.  Under torchrun every rank
@@ -35,20 +42,24 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "decode-attn KV GB/s & % of HBM/tensor roofline; merge GB/s; µs/step/layer"
-DEFAULT_WORKLOAD = "gqa_70b"
+DEFAULT_WORKLOAD = "mla_mix"
+DEFAULT_EXTRA = "gqa_70b:4"
 
 
 def parse(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--shards", type=int, default=None, help="D (default: the largest of the workload's list)")
-    ap.add_argument("--other-d-steps", type=int, default=200, help="steps for the workload's other D values (0: skip)")
-    ap.add_argument("--e2e-steps", type=int, default=100)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline time budget")
+    ap.add_argument("--other-d-steps", type=int, default=50, help="steps for the workload's other D values (0: skip)")
+    ap.add_argument("--extra", default=DEFAULT_EXTRA,
+                    help="comma-separated workload:D lines measured after the headline ('' for none)")
+    ap.add_argument("--extra-steps", type=int, default=300)
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU baseline budget per leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-len", type=int, default=1,
                     help="query tokens per request (multi-token decode, causal within the draft; 1..4)")
@@ -173,18 +184,18 @@ def recorded_traffic(workload: str, D: int, layout: int):
     return ent.get("dram_bytes_per_launch")
 
 
-def load_workload(args):
+def load_workload(name, batch_limit=None, q_len=1, kv_dtype="bf16"):
     import synth
-    w = synth.workload(args.workload)
-    if args.batch_limit is not None and args.batch_limit < w.batch:
-        w.seq_lens = w.seq_lens[:args.batch_limit]
-        w.batch = args.batch_limit
-        w.name = f"{w.name}[:{args.batch_limit}]"
-    if args.q_len != 1:
-        w.q_len = args.q_len
-        w.name = f"{w.name} q_len={args.q_len}"
-    w.extra["kv_dtype"] = args.kv_dtype
-    if args.kv_dtype == "fp8":
+    w = synth.workload(name)
+    if batch_limit is not None and batch_limit < w.batch:
+        w.seq_lens = w.seq_lens[:batch_limit]
+        w.batch = batch_limit
+        w.name = f"{w.name}[:{batch_limit}]"
+    if q_len != 1:
+        w.q_len = q_len
+        w.name = f"{w.name} q_len={q_len}"
+    w.extra["kv_dtype"] = kv_dtype
+    if kv_dtype == "fp8":
         w.name = f"{w.name} fp8"
     return w
 
@@ -223,6 +234,11 @@ def algorithmic_bytes(w, D: int):
     return kv, decode, merge
 
 
+# Below this ideal time at the copy peak a merge is launch/latency-bound (a launch and its
+# first loads cost a few microseconds on their own), so its GB/s is not a bandwidth figure.
+MERGE_LATENCY_FLOOR_US = 5.0
+
+
 # ----------------------------------------------------------------------------- CPU oracle baseline
 def run_oracle_sample(w, D: int, sample) -> float:
     """Seconds the float64 oracle takes for one sample: D shard partials + their merge."""
@@ -233,24 +249,15 @@ def run_oracle_sample(w, D: int, sample) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, D: int, budget_s: float):
-    """Time the oracle on (request, KV head) samples until ``budget_s`` seconds of oracle work.
-
-    Returns (GB/s of KV processed, seconds, description)."""
-    spent, kv_bytes, n = 0.0, 0, 0
-    i = 0
-    while spent < budget_s and i < 4 * w.batch:
-        s = _sample_at(w, i)
-        spent += run_oracle_sample(w, D, s)
-        kv_bytes += s[4]
-        n += 1
-        i += 1
-    what = "(request, KV head) pairs" if w.layout == 0 else "(request, 4 of 64 heads) pairs"
-    desc = f"{n} {what} of {w.name}, D={D}: float64 shard partials + merge, single thread"
-    return kv_bytes / spent / 1e9, spent, desc
+MLA_SAMPLE_HEADS = 4
 
 
 def _sample_at(w, i: int, max_tokens: int = None):
+    """(request, q, KV source, heads, KV bytes the sample stands for).
+
+    GQA: one (request, KV head) pair -- its G query heads are the whole work on those KV bytes.
+    MLA: 4 of the 64 query heads of a request; every head reads the whole latent row, so the
+    sample stands for 4/64 of the request's KV bytes."""
     import synth
     order = sorted(range(w.batch), key=lambda b: (b * 7919) % w.batch)
     b = order[i % w.batch]
@@ -260,160 +267,351 @@ def _sample_at(w, i: int, max_tokens: int = None):
         src = w.kv_source_head(b, h, max_tokens)
         return (b, w.query(b)[h * G:(h + 1) * G], src, G, src.shape[0] * 2 * w.head_dim_qk * 2)
     src = w.kv_source(b, max_tokens)
-    return (b, w.query(b)[:4], src, 4, src.shape[0] * w.head_dim_qk * 2)
+    hq = MLA_SAMPLE_HEADS
+    return (b, w.query(b)[:hq], src, hq, src.shape[0] * w.head_dim_qk * 2 * hq // w.num_q_heads)
+
+
+def cpu_single_thread(w, D: int, budget_s: float):
+    """Time the oracle on samples in this process until ``budget_s`` seconds of oracle work."""
+    spent, kv_bytes, n, i = 0.0, 0, 0, 0
+    while spent < budget_s and i < 4 * w.batch:
+        s = _sample_at(w, i)
+        spent += run_oracle_sample(w, D, s)
+        kv_bytes += s[4]
+        n += 1
+        i += 1
+    return kv_bytes / spent / 1e9, spent, n
+
+
+def _oracle_worker(wname, batch_limit, D, indices, reps, max_tokens, start, out):
+    """One process of the all-core leg: build its few samples, wait for the others, then time the
+    oracle over them `reps` times (the oracle's time does not depend on the values)."""
+    sys.path.insert(0, ROOT)
+    w = load_workload(wname, batch_limit)
+    samples = [_sample_at(w, i, max_tokens) for i in indices]
+    start.wait()
+    t0 = time.perf_counter()
+    kv = 0
+    for r in range(reps):
+        s = samples[r % len(samples)]
+        run_oracle_sample(w, D, s)
+        kv += s[4]
+    out.put((kv, time.perf_counter() - t0))
+
+
+def cpu_all_cores(w, D: int, rate_1t_gbs: float, budget_s: float, batch_limit=None):
+    """The oracle in one process per host core (spawned: no fork after CUDA initialisation),
+    each on its own samples of at most 4,096 tokens, sized so every process has about
+    ``budget_s`` seconds of oracle work.  Returns (GB/s, cores, samples, seconds)."""
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    max_tokens = 4096
+    s0 = _sample_at(w, 0, max_tokens)
+    per_sample_s = max(1e-3, s0[4] / (rate_1t_gbs * 1e9))
+    per_worker = max(1, int(budget_s / per_sample_s))
+    ctx = mp.get_context("spawn")
+    start = ctx.Barrier(cores + 1)
+    out = ctx.Queue()
+    distinct = min(per_worker, 3)
+    procs = [ctx.Process(target=_oracle_worker,
+                         args=(w.name.split("[")[0].split(" ")[0], batch_limit, D,
+                               [c * distinct + k for k in range(distinct)], per_worker, max_tokens, start, out))
+             for c in range(cores)]
+    for p in procs:
+        p.start()
+    try:
+        start.wait(timeout=600)
+        res = [out.get(timeout=600) for _ in procs]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.terminate()
+    kv = sum(r[0] for r in res)
+    secs = max(r[1] for r in res)
+    return kv / secs / 1e9, cores, cores * per_worker, secs, max_tokens
+
+
+def cpu_baseline(w, D: int, budget_s: float, batch_limit=None):
+    what = "(request, KV head) pairs" if w.layout == 0 else f"(request, {MLA_SAMPLE_HEADS} of 64 heads) pairs"
+    gbs1, secs1, n1 = cpu_single_thread(w, D, budget_s)
+    line = {"unit": "GB/s", "kind": "oracle",
+            "single_thread": {"value": round(gbs1, 4), "cores": 1, "seconds": round(secs1, 2),
+                              "sample": f"{n1} {what} of {w.name}, D={D}, whole requests"}}
+    try:
+        gbs, cores, n, secs, mt = cpu_all_cores(w, D, gbs1, budget_s, batch_limit)
+        line.update({"value": round(gbs, 4), "cores": cores, "seconds": round(secs, 2),
+                     "sample": f"{n} {what} of {w.name} (first {mt} tokens each), D={D}: float64 shard "
+                               f"partials + merge, one process per host core ({cores})"})
+    except Exception as e:  # the all-core leg is a report; a host that cannot spawn falls back to 1 core
+        line.update({"value": round(gbs1, 4), "cores": 1, "sample": line["single_thread"]["sample"],
+                     "all_cores_error": f"{type(e).__name__}: {e}"})
+    line["host_cores"] = os.cpu_count()
+    return line
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local):
-    import numpy as np
-    import torch
+class Bench:
+    """Device-side plumbing shared by every measured line."""
 
-    import synth
-    import synth.device as sdev
-    from sequence_sharded_decode_paged_b200.cache import ShardedPagedCache
+    def __init__(self, local: int, world: int):
+        import torch
+        torch.cuda.set_device(local)
+        self.dev = torch.device("cuda", local)
+        self.world = world
+        l2 = torch.cuda.get_device_properties(local).L2_cache_size
+        # never written after this: reading it evicts L2 without adding dirty lines of its own
+        self.flush_buf = torch.ones(2 * l2 // 4, dtype=torch.int32, device=self.dev)
+        self.flush_out = torch.empty((), dtype=torch.int32, device=self.dev)
+        self.peaks, self.peaks_kind = measured_peaks()
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist_init(world, "nccl")
-    w = load_workload(args)
-    D = args.shards or max(w.shards)
-    peaks, peaks_kind = measured_peaks()
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    def flush(self):
+        import torch
+        torch.amax(self.flush_buf, dim=0, out=self.flush_out)
 
-    def build(Dx):
+    def build(self, w, D):
+        import torch
+        import synth.device as sdev
+        from sequence_sharded_decode_paged_b200.cache import ShardedPagedCache
         cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v,
-                                  w.block_size, Dx, w.seq_lens, w.softmax_scale, device=dev, q_len=w.q_len,
+                                  w.block_size, D, w.seq_lens, w.softmax_scale, device=self.dev, q_len=w.q_len,
                                   kv_dtype=1 if cache_elem_bytes(w) == 1 else 0, k_scale=FP8_SCALE,
                                   v_scale=FP8_SCALE)
-        kv = sdev.kv_source(w, dev, cache.cu_seqlens)
+        kv = sdev.kv_source(w, self.dev, cache.cu_seqlens)
         cache.place(kv)
         del kv
+        q = sdev.query(w, self.dev)
         torch.cuda.synchronize()
-        return cache
+        return cache, q
 
-    q = sdev.query(w, dev)
-
-    def timed(cache, steps, warmup):
-        for i in range(warmup):
-            flush.fill_(i & 0xFF)
+    def timed(self, cache, q, steps, warmup):
+        """(mean step ms, mean partials ms, mean merge ms, median step ms) over `steps` steps."""
+        import torch
+        for _ in range(warmup):
+            self.flush()
             cache.step(q)
         torch.cuda.synchronize()
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-        barrier(world)
+        barrier(self.world)
         torch.cuda.synchronize()
         for i in range(steps):
-            flush.fill_(i & 0xFF)
+            self.flush()
             ev[i][0].record()
             cache.partials(q)
             ev[i][1].record()
             cache.merge()
             ev[i][2].record()
         torch.cuda.synchronize()
-        barrier(world)
+        barrier(self.world)
         part = [e[0].elapsed_time(e[1]) for e in ev]
         merge = [e[1].elapsed_time(e[2]) for e in ev]
         step = [e[0].elapsed_time(e[2]) for e in ev]
         return sum(step) / steps, sum(part) / steps, sum(merge) / steps, statistics.median(step)
 
-    cache = build(D)
+    def figures(self, w, D, step_ms, part_ms, merge_ms):
+        """Roofline and throughput figures of one measured line (times already max over ranks)."""
+        kv_b, dec_b, mrg_b = algorithmic_bytes(w, D)
+        peak = self.peaks["hbm_gbs"]
+        achieved = dec_b / part_ms / 1e6
+        merge_ideal_us = mrg_b / (peak * 1e3)
+        return {
+            "kv_gbs": round(job_value(self.world, kv_b, step_ms), 1),
+            "us_per_step_per_layer": round(step_ms * 1e3, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name, D, w.layout),
+                         "kernel": "gqa_decode_kernel" if w.layout == 0 else "mla_decode_kernel",
+                         "peak_kind": f"{self.peaks_kind} HBM copy (burst)",
+                         "algorithmic_bytes_per_launch": dec_b},
+            "decode_kernel_us": round(part_ms * 1e3, 2),
+            "merge_kernel_us": round(merge_ms * 1e3, 2),
+            "merge_gbs": round(mrg_b / merge_ms / 1e6, 1),
+            "merge_frac": round(mrg_b / merge_ms / 1e6 / peak, 4),
+            "merge_bytes": mrg_b,
+            "merge_bound": ("hbm" if merge_ideal_us >= MERGE_LATENCY_FLOOR_US else
+                            f"latency (ideal {merge_ideal_us:.2f} us at the copy peak, under the "
+                            f"{MERGE_LATENCY_FLOOR_US:.0f} us launch/latency floor)"),
+            "context_tokens_per_s": round(self.world * w.total_tokens / step_ms * 1e3, 1),
+            "query_tokens_per_s": round(self.world * w.batch * w.q_len / step_ms * 1e3, 1),
+            "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
+            "tensor": tensor_figures(w, part_ms, self.peaks, self.peaks_kind),
+        }
+
+    def e2e_host_calls(self, cache, q, steps):
+        """Steps through dcp_decode_step_host (host inputs and outputs), one after another on one
+        stream; returns (ms per step, h2d bytes, d2h bytes)."""
+        import numpy as np
+        import torch
+        from sequence_sharded_decode_paged_b200 import dcp
+        d = cache.desc
+        rows = cache.batch * cache.q_len * d.num_q_heads
+        h_q = torch.empty(q.numel(), dtype=torch.int16).pin_memory()
+        h_q.copy_(q.reshape(-1).view(torch.int16).cpu())
+        h_lens = torch.tensor(cache.seq_lens, dtype=torch.int32).pin_memory()
+        h_tab = torch.from_numpy(np.ascontiguousarray(cache.tables_host, dtype=np.int32)).pin_memory()
+        h_O = [torch.empty(rows * d.head_dim_v, dtype=torch.float32).pin_memory() for _ in range(2)]
+        h_L = [torch.empty(rows, dtype=torch.float32).pin_memory() for _ in range(2)]
+        nb = dcp.dcp_host_step_staging_bytes(d, cache.D)
+        staging = torch.empty(nb, dtype=torch.uint8, device=self.dev)
+        stream = torch.cuda.current_stream()
+
+        def step(i):
+            dcp.dcp_decode_step_host(d, cache.D, h_q, h_lens, h_tab, cache.pools, cache.pool_pages, staging,
+                                     cache.workspace, h_O[i & 1], h_L[i & 1], stream=stream)
+
+        for i in range(2):
+            self.flush()
+            step(i)
+        torch.cuda.synchronize()
+        barrier(self.world)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(steps):
+            self.flush()
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(self.world)
+        ms = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+        assert np.isfinite(h_O[0].numpy()).all(), "e2e: non-finite output"
+        h2d = h_q.numel() * 2 + h_lens.numel() * 4 + h_tab.numel() * 4
+        d2h = h_O[0].numel() * 4 + h_L[0].numel() * 4
+        return ms, h2d, d2h
+
+    def e2e_pipelined(self, cache, q, steps):
+        """The overlapped host pipeline (uploads and downloads of neighbouring steps hidden behind
+        the current step's compute): a throughput figure, reported beside the per-step e2e."""
+        import numpy as np
+        import torch
+        from sequence_sharded_decode_paged_b200.cache import HostStepPipeline
+        pipe = HostStepPipeline(cache)
+        host_in = pipe.pack_inputs(q.view(torch.int16).cpu().numpy(), cache.seq_lens, cache.tables_host)
+        host_out = [pipe.host_output(), pipe.host_output()]
+        for i in range(2):
+            pipe.step(i, host_in, host_out[i & 1])
+        pipe.synchronize()
+        barrier(self.world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(pipe.s_in)
+        for i in range(steps):
+            pipe.step(i, host_in, host_out[i & 1])
+        e1.record(pipe.s_out)
+        pipe.synchronize()
+        torch.cuda.synchronize()
+        barrier(self.world)
+        assert np.isfinite(pipe.unpack_output(host_out[0])[0].numpy()).all()
+        return e0.elapsed_time(e1) / max(1, steps)
+
+    def append_us(self, w, cache, D):
+        """Cache write of one new token per request (the append that precedes each decode step),
+        20 calls captured in one CUDA graph; it rewrites each request's last slot."""
+        import torch
+        from sequence_sharded_decode_paged_b200 import dcp
+        row_elems = w.kv_bytes_per_token // 2
+        kv_row = torch.zeros((w.batch, row_elems), dtype=torch.int16, device=self.dev)
+        cu_rows = torch.arange(w.batch + 1, dtype=torch.int64, device=self.dev)
+        last_pos = (cache.seq_lens_dev - 1).clamp_min(0).contiguous()
+        side = torch.cuda.Stream(self.dev)
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
+                                  cache.pool_pages, stream=side)
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(20):
+                dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
+                                  cache.pool_pages, stream=side)
+        graph.replay()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(5):
+            graph.replay()
+        a1.record()
+        torch.cuda.synchronize()
+        ms = a0.elapsed_time(a1) / 100
+        del graph
+        return ms
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    dist_init(world, "nccl")
+    bench = Bench(local, world)
+    dev = bench.dev
+    w = load_workload(args.workload, args.batch_limit, args.q_len, args.kv_dtype)
+    D = args.shards or max(w.shards)
+    launches = 0
+
+    cache, q = bench.build(w, D)
     sampler = ClockSampler(local)
     time.sleep(0.3)
-    step_ms, part_ms, merge_ms, step_med = timed(cache, args.steps, args.warmup)
+    step_ms, part_ms, merge_ms, step_med = bench.timed(cache, q, args.steps, args.warmup)
     clocks = sampler.stop()
+    launches += 2 * args.steps
     err = cache.device_error()
     if err != 0:
         raise RuntimeError(f"device status {err} during the timed run")
 
-    # end to end through the public API: every step uploads its packed inputs (query,
-    # lengths, block tables) from pinned host memory and reads its results (O, LSE)
-    # back; neighbouring steps' copies overlap the current step's compute
-    from sequence_sharded_decode_paged_b200.cache import HostStepPipeline
-    pipe = HostStepPipeline(cache)
-    host_in = pipe.pack_inputs(q.view(torch.int16).cpu().numpy(), w.seq_lens, cache.tables_host)
-    host_out = [pipe.host_output(), pipe.host_output()]
-    for i in range(2):
-        pipe.step(i, host_in, host_out[i & 1])
-    pipe.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(pipe.s_in)
-    for i in range(args.e2e_steps):
-        pipe.step(i, host_in, host_out[i & 1])
-    e1.record(pipe.s_out)
-    pipe.synchronize()
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = e0.elapsed_time(e1) / max(1, args.e2e_steps)
-    h2d, d2h = pipe.in_bytes, pipe.out_bytes
-    assert np.isfinite(pipe.unpack_output(host_out[0])[0].numpy()).all()
+    e2e_ms, h2d, d2h = bench.e2e_host_calls(cache, q, args.e2e_steps)
+    launches_e2e = 2 * args.e2e_steps
+    pipe_ms = bench.e2e_pipelined(cache, q, args.e2e_steps)
+    if cache.device_error() != 0:
+        raise RuntimeError("device status set during the e2e runs")
+    append_ms = bench.append_us(w, cache, D)
 
-    # cache write of one new token per request (the append that precedes each decode step),
-    # timed on its own; it rewrites each request's last slot, after which the cache is not reused
-    from sequence_sharded_decode_paged_b200 import dcp
-    row_elems = w.kv_bytes_per_token // 2
-    kv_row = torch.zeros((w.batch, row_elems), dtype=torch.int16, device=dev)
-    cu_rows = torch.arange(w.batch + 1, dtype=torch.int64, device=dev)
-    last_pos = (cache.seq_lens_dev - 1).clamp_min(0).contiguous()
-    # 20 appends captured in one CUDA graph, so the events time the kernels, not the host calls
-    side = torch.cuda.Stream(dev)
-    with torch.cuda.stream(side):
-        for _ in range(3):
-            dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
-                              cache.pool_pages, stream=side)
-    side.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=side):
-        for _ in range(20):
-            dcp.dcp_append_kv(cache.desc, D, kv_row, cu_rows, last_pos, cache.tables, cache.pools,
-                              cache.pool_pages, stream=side)
-    graph.replay()
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for _ in range(5):
-        graph.replay()
-    a1.record()
-    torch.cuda.synchronize()
-    append_ms = a0.elapsed_time(a1) / 100
-    del graph
-
-    kv_b, dec_b, mrg_b = algorithmic_bytes(w, D)
-    step_ms_max = reduce_max(step_ms, world, dev)
-    append_ms_max = reduce_max(append_ms, world, dev)
-    part_ms_max = reduce_max(part_ms, world, dev)
-    merge_ms_max = reduce_max(merge_ms, world, dev)
-    e2e_ms_max = reduce_max(e2e_ms, world, dev)
+    step_ms, part_ms, merge_ms, e2e_ms, pipe_ms, append_ms = (
+        reduce_max(x, world, dev) for x in (step_ms, part_ms, merge_ms, e2e_ms, pipe_ms, append_ms))
+    fig = bench.figures(w, D, step_ms, part_ms, merge_ms)
+    kv_b, _, _ = algorithmic_bytes(w, D)
 
     other = {}
     if args.other_d_steps > 0:
         for Dx in w.shards:
             if Dx == D:
                 continue
-            del cache
+            del cache, q
             torch.cuda.empty_cache()
-            cache = build(Dx)
-            s_ms, p_ms, m_ms, _ = timed(cache, args.other_d_steps, max(3, args.warmup // 2))
+            cache, q = bench.build(w, Dx)
+            s_ms, p_ms, m_ms, _ = bench.timed(cache, q, args.other_d_steps, max(3, args.warmup))
             s_ms, p_ms, m_ms = (reduce_max(x, world, dev) for x in (s_ms, p_ms, m_ms))
-            kb, db, mb = algorithmic_bytes(w, Dx)
-            other[str(Dx)] = {"kv_gbs": round(world * kb / s_ms / 1e6, 1), "us_per_step_per_layer": round(s_ms * 1e3, 2),
-                              "decode_kernel_gbs": round(db / p_ms / 1e6, 1), "merge_gbs": round(mb / m_ms / 1e6, 1),
-                              "decode_us": round(p_ms * 1e3, 2), "merge_us": round(m_ms * 1e3, 2),
-                              "steps": args.other_d_steps}
+            f = bench.figures(w, Dx, s_ms, p_ms, m_ms)
+            other[str(Dx)] = {k: f[k] for k in ("kv_gbs", "us_per_step_per_layer", "decode_kernel_us",
+                                                 "merge_kernel_us", "merge_gbs", "merge_bound")}
+            other[str(Dx)]["roofline_frac"] = f["roofline"]["frac"]
+            other[str(Dx)]["steps"] = args.other_d_steps
+    del cache, q
+    torch.cuda.empty_cache()
+
+    extra = {}
+    for spec in [s for s in args.extra.split(",") if s.strip()]:
+        name, _, dspec = spec.partition(":")
+        wx = load_workload(name.strip())
+        Dx = int(dspec) if dspec else max(wx.shards)
+        cx, qx = bench.build(wx, Dx)
+        s_ms, p_ms, m_ms, _ = bench.timed(cx, qx, args.extra_steps, max(3, args.warmup))
+        if cx.device_error() != 0:
+            raise RuntimeError(f"device status set during the {name} run")
+        s_ms, p_ms, m_ms = (reduce_max(x, world, dev) for x in (s_ms, p_ms, m_ms))
+        f = bench.figures(wx, Dx, s_ms, p_ms, m_ms)
+        f.update({"workload": f"{wx.name}: {wx.note}", "D": Dx, "steps": args.extra_steps,
+                  "ms_per_step": round(s_ms, 4), "context_tokens": wx.total_tokens})
+        extra[f"{wx.name}/D{Dx}"] = f
+        del cx, qx
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return None
-    peak = peaks["hbm_gbs"]
-    achieved = dec_b / part_ms_max / 1e6
     line = {
         "metric": METRIC,
-        "value": round(job_value(world, kv_b, step_ms_max), 1),
+        "value": fig["kv_gbs"],
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(step_ms_max, 4),
+        "ms_per_step": round(step_ms, 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -421,45 +619,47 @@ def run_ours(args, rank, world, local):
         "data": "synthetic",
         "config": {"workload": f"{w.name}: {w.note}", "D": D, "batch": w.batch, "q_len": w.q_len,
                    "context_tokens": w.total_tokens, "kv_bytes_per_step": kv_b,
-                   "l2": "flushed before every step (write of 2x L2), outside the timed events",
+                   "l2": "flushed before every step by reading a buffer of 2x L2 (no writes), outside the "
+                         "timed events; the KV read per step is also far larger than L2",
                    "parallelism": "replicas" if world > 1 else "single GPU (D shard pools in one HBM)"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": recorded_traffic(w.name, D, w.layout),
-                     "kernel": "gqa_decode_kernel" if w.layout == 0 else "mla_decode_kernel",
-                     "peak_kind": f"{peaks_kind} HBM copy (burst)",
-                     "algorithmic_bytes_per_launch": dec_b},
-        "us_per_step_per_layer": round(step_ms_max * 1e3, 2),
-        "decode_kernel_us": round(part_ms_max * 1e3, 2),
-        "merge_kernel_us": round(merge_ms_max * 1e3, 2),
-        "merge_gbs": round(mrg_b / merge_ms_max / 1e6, 1),
-        "append_kernel_us": round(append_ms_max * 1e3, 2),
+        "roofline": fig["roofline"],
+        "us_per_step_per_layer": fig["us_per_step_per_layer"],
+        "decode_kernel_us": fig["decode_kernel_us"],
+        "merge_kernel_us": fig["merge_kernel_us"],
+        "merge_gbs": fig["merge_gbs"],
+        "merge_frac": fig["merge_frac"],
+        "merge_bound": fig["merge_bound"],
+        "append_kernel_us": round(append_ms * 1e3, 2),
         "append_bytes_per_step": w.batch * w.kv_bytes_per_token * (2 + cache_elem_bytes(w)) // 2,
-        "context_tokens_per_s": round(world * w.total_tokens / step_ms_max * 1e3, 1),
-        "query_tokens_per_s": round(world * w.batch * w.q_len / step_ms_max * 1e3, 1),
-        "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
-        "tensor": tensor_figures(w, part_ms_max, peaks, peaks_kind),
+        "context_tokens_per_s": fig["context_tokens_per_s"],
+        "query_tokens_per_s": fig["query_tokens_per_s"],
+        "frac_of_8tbs_spec": fig["frac_of_8tbs_spec"],
+        "tensor": fig["tensor"],
         "median_step_ms": round(step_med, 4),
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches,
         "clocks": clocks,
-        "e2e": {"value": round(job_value(world, kv_b, e2e_ms_max), 1), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 4),
-                "steps": args.e2e_steps, "api": "HostStepPipeline (one packed upload and one download per step, "
-                                                "overlapped with neighbouring steps)"},
+        "e2e": {"value": round(job_value(world, kv_b, e2e_ms), 1), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+                "steps": args.e2e_steps, "gpu_launches": launches_e2e,
+                "api": "dcp_decode_step_host (C ABI, host buffers): per step the H2D copies of query, "
+                       "lengths and tables, decode, merge and the D2H copies of O and LSE, steps serialised "
+                       "on one stream",
+                "pipelined": {"value": round(job_value(world, kv_b, pipe_ms), 1), "unit": "GB/s",
+                              "ms_per_step": round(pipe_ms, 4),
+                              "api": "HostStepPipeline: the same copies, overlapped with neighbouring steps"}},
         "other_D": other,
+        "extra": extra,
     }
     if world == 1 and not args.no_cpu_baseline and w.q_len == 1 and cache_elem_bytes(w) == 2:
-        gbs, secs, desc = cpu_baseline(w, D, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                "sample": desc, "seconds": round(secs, 2)}
+        line["cpu_baseline"] = cpu_baseline(w, D, args.cpu_seconds, args.batch_limit)
     return line
 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args, rank, world):
-    import synth
     if rank != 0:  # the oracle runs once, on rank 0; other ranks have no work
         return None
-    w = load_workload(args)
+    w = load_workload(args.workload, args.batch_limit, args.q_len, args.kv_dtype)
     D = args.shards or max(w.shards)
     total_budget = 150.0  # seconds of oracle work for warm-up + timed steps
     per_step = total_budget / max(1, args.steps + args.warmup)
@@ -477,13 +677,14 @@ def run_reference(args, rank, world):
         kv_total += s[4]
     wall = time.perf_counter() - t0
     value = kv_total / secs_total / 1e9
+    what = "(request, KV head)" if w.layout == 0 else f"(request, {MLA_SAMPLE_HEADS} of 64 heads)"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs_total / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{w.name}: {w.note}", "D": D, "batch": w.batch, "context_tokens": w.total_tokens},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: one (request, KV head) sample of {w.name}, at most {max_tok} tokens, "
+                         "sample": f"each step: one {what} sample of {w.name}, at most {max_tok} tokens, "
                                    f"D={D} float64 shard partials + merge, single thread"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": round(wall, 1),

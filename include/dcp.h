@@ -27,7 +27,8 @@
  *     data_ptr()); "host" pointers are ordinary CPU memory.
  *   - GPU calls are asynchronous on `stream` (a cudaStream_t passed as
  *     void*; NULL = legacy default stream).  They never synchronise, except
- *     dcp_read_device_error which is documented as synchronous.
+ *     dcp_read_device_error and dcp_noalloc_read_device_error, which are
+ *     documented as synchronous.
  *   - Return value: DCP_OK, or an error code.  Argument errors are detected
  *     on the host before anything is launched (nothing is written then).
  *     DCP_ERR_CUDA means a CUDA runtime call or a launch failed.
@@ -345,8 +346,11 @@ DCP_API dcp_status dcp_decode_partial_all(const dcp_attn_desc *desc, const void 
  *     `stream`, then launches the decode kernel.  It allocates nothing.
  *   - All calls share the scratch, which keeps the last call's contents:
  *     calls that overlap on the GPU (e.g. on two streams) race; serialise them.
- *   - Out-of-range page ids are skipped as in dcp_decode_partial_all but not
- *     reported (there is no caller-visible status word).
+ *   - The status bits that dcp_read_device_error reports for a workspace
+ *     (bit 0: an out-of-range page id was skipped; bit 1: a pipeline wait
+ *     timed out and that call's results are invalid) go to the scratch's own
+ *     status word; dcp_noalloc_read_device_error reads and clears it.  Each
+ *     call clears it first, so it describes the latest call only.
  * Errors: as dcp_decode_partial_all; DCP_ERR_UNSUPPORTED for MLA;
  * DCP_ERR_CAPACITY if the problem needs more than the 16 MiB scratch
  * (dcp_decode_workspace_bytes(desc, D) > 16 MiB, e.g. very wide head groups).
@@ -355,6 +359,14 @@ DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc *desc, con
                                                   const void *const *kv_pools, const int32_t *pool_pages,
                                                   const int32_t *const *tables, const int32_t *seq_lens, int32_t D,
                                                   float *const *O_parts, float *const *LSE_parts, void *stream);
+
+/*
+ * Status word of dcp_decode_partial_all_noalloc's scratch on the current
+ * device: waits for `stream`, stores the bits in *error_out (meanings as in
+ * dcp_read_device_error) and clears the word.  Allocates nothing; like the
+ * decode call, its first use on a device looks up the scratch address.
+ */
+DCP_API dcp_status dcp_noalloc_read_device_error(int32_t *error_out, void *stream);
 
 /*
  * LSE merge of D partials.  [P1 "A2 方法细节", merge equation;
@@ -369,6 +381,36 @@ DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc *desc, con
  */
 DCP_API dcp_status dcp_lse_merge(const float *const *O_parts, const float *const *LSE_parts, int32_t D, int32_t rows,
                          int32_t d_v, float *O, float *LSE_out, void *stream);
+
+/*
+ * One whole decode step with HOST inputs and outputs.  [P1 "A2 方法细节": the
+ * shards attend the full query against their local KV slices, then the
+ * partials are merged by the equation above.]  On `stream`, in order: the
+ * query, the lengths and the D block tables are copied from host memory into
+ * `staging`; the D shard partials run in one launch (as
+ * dcp_decode_partial_all) into `staging`; dcp_lse_merge combines them; the
+ * merged O (and LSE) are copied back to host memory.
+ *   host_q         host bf16 [batch][q_len][Hq][head_dim_qk].
+ *   host_seq_lens  host int32 [batch], global lengths.
+ *   host_tables    host int32 [D][batch][max_local_blocks] (as dcp_build_block_table writes them).
+ *   kv_pools       host array of D device pointers (pools already written); pool_pages host int32[D].
+ *   staging        device, >= dcp_host_step_staging_bytes(desc, D) bytes, 256-byte aligned: the
+ *                  uploaded inputs, the D partials and the merged output live there (caller-owned;
+ *                  one staging buffer may not serve two steps that overlap in time).
+ *   workspace      as for dcp_decode_partial_all (initialised).
+ *   host_O         host fp32 [batch][q_len][Hq][head_dim_v];  host_LSE host fp32 [batch][q_len][Hq] or NULL.
+ * Asynchronous like every GPU call: host_O / host_LSE are valid once `stream` has been
+ * synchronised, and the host inputs must stay untouched until then.  Pinned (page-locked)
+ * host memory keeps the copies asynchronous; pageable memory works, but the CUDA runtime
+ * then stages it and the call may block the calling thread.
+ * Errors: as dcp_decode_partial_all; DCP_ERR_CAPACITY if staging or workspace is too small.
+ */
+DCP_API size_t dcp_host_step_staging_bytes(const dcp_attn_desc *desc, int32_t D);
+DCP_API dcp_status dcp_decode_step_host(const dcp_attn_desc *desc, int32_t D, const void *host_q,
+                                        const int32_t *host_seq_lens, const int32_t *host_tables,
+                                        const void *const *kv_pools, const int32_t *pool_pages, void *staging,
+                                        size_t staging_bytes, void *workspace, size_t workspace_bytes,
+                                        float *host_O, float *host_LSE, void *stream);
 
 /*
  * Read (synchronously: waits for `stream`) and clear the status word of a

@@ -253,7 +253,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
       const int32_t* trow = p.table[si] + (size_t)b * p.mlb;
       for (int j = a; j < e; ++j) {
-        const int page = trow[j];
+        // a local block past the table row (lengths grown beyond max_local_blocks) is
+        // treated like an out-of-pool page: never read, flagged in the status word
+        const int page = j < p.mlb ? trow[j] : -1;
         const bool ok = page >= 0 && page < p.pool_pages[si];
         if (!ok) atomicOr(p.status, kDevBadPage);
         if (!mbar_wait(&empty[stage], phase ^ 1u)) {

@@ -65,7 +65,15 @@ constexpr uint32_t kOffKV = kTileBytes;               // two stages
 // P^T (64 heads x 64 tokens bf16, 8 KB) of a page lives in its stage's rope box (dims 512-575 of
 // the latent tile), which only QK^T reads: no separate buffer.
 constexpr uint32_t kOffMisc = 3 * kTileBytes;
-constexpr uint32_t kMlaSmem = kOffMisc + 3072;  // 224,256 bytes
+// Split combine: per-piece softmax weights of the 64 rows, up to kCombineMax pieces at once.
+constexpr int kCombineMax = 16;
+constexpr uint32_t kOffW = kOffMisc + 3072;
+constexpr uint32_t kMlaSmem = kOffW + kCombineMax * 64 * 4;  // 228,352 bytes
+// Pages prefetched into L2 ahead of the page whose tile load is being issued (0: none).
+#ifndef DCP_MLA_L2_AHEAD
+#define DCP_MLA_L2_AHEAD 0
+#endif
+constexpr int kL2Ahead = DCP_MLA_L2_AHEAD;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                         // O^T: 4 tiles x 64 columns
 constexpr uint32_t kColS = 256;                       // S: 2 buffers x 64 columns
@@ -95,6 +103,7 @@ static_assert(sizeof(MlaMisc) <= 3072, "misc block");
 struct MlaParams {
   CUtensorMap kvmap[kMaxShards];
   CUtensorMap qmap;
+  const uint8_t* pool[kMaxShards];
   const int32_t* table[kMaxShards];
   float* O[kMaxShards];
   float* LSE[kMaxShards];
@@ -136,8 +145,52 @@ __device__ __forceinline__ void wait_or_die_warp(uint64_t* bar, uint32_t parity,
   dead = __any_sync(0xffffffffu, dead);
 }
 
+// Walks the pages of a CTA's range in order (segment by segment), for the L2 prefetch.
+template <int RULE>
+struct PageCursor {
+  int sid, pre, si, b, j, e;
+  bool live;
+  __device__ __forceinline__ void init(int sid0, int pre0) {
+    sid = sid0;
+    pre = pre0;
+    j = e = si = b = 0;
+    live = true;
+  }
+  // Next page of the range: (slot, request, local block); false at its end.
+  __device__ __forceinline__ bool next(const MlaParams& p, int S, int T, int P, int cta, int lo, int hi, int* osi,
+                                       int* ob, int* oj) {
+    while (live) {
+      if (j < e) {
+        *osi = si;
+        *ob = b;
+        *oj = j++;
+        return true;
+      }
+      if (sid >= S) break;
+      const int si2 = sid / p.B, b2 = sid - si2 * p.B;
+      const int n2 = local_pages_r<RULE>(p.seq_lens[b2], kMlaBs, p.D, p.shard_of_si[si2]);
+      if (seg_first_cta(pre, n2, T, P) > cta) break;
+      si = si2;
+      b = b2;
+      j = max(pre, lo) - pre;
+      e = n2 > 0 ? min(pre + n2, hi) - pre : 0;
+      pre += n2;
+      ++sid;
+    }
+    live = false;
+    return false;
+  }
+};
+
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ bool page_ok(const MlaParams& p, int si, int b, int j, int* page_out) {
-  const int page = p.table[si][(size_t)b * p.mlb + j];
+  // a local block past the table row (lengths grown beyond max_local_blocks) is
+  // treated like an out-of-pool page: never read, flagged in the status word
+  const int page = j < p.mlb ? p.table[si][(size_t)b * p.mlb + j] : -1;
   *page_out = page;
   return page >= 0 && page < p.pool_pages[si];
 }
@@ -199,6 +252,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       long issued = 0;
       bool dead = false, q_issued = false;
       int pre = plan.pre0;
+      // L2 prefetch kL2Ahead pages ahead of the page whose tile load is issued next
+      PageCursor<RULE> ahead;
+      ahead.init(plan.sid0, plan.pre0);
+      auto prefetch_next = [&]() {
+        int asi, ab, aj, apage;
+        if (ahead.next(p, S, T, P, cta, lo, hi, &asi, &ab, &aj) && page_ok(p, asi, ab, aj, &apage))
+          prefetch_l2_bulk(p.pool[asi] + (size_t)apage * kTileBytes, kTileBytes);
+      };
+      if (kL2Ahead > 0)
+        for (int i = 0; i < kL2Ahead; ++i) prefetch_next();
       for (int sid = plan.sid0; sid < S; ++sid) {
         const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
         const int n = local_pages_r<RULE>(p.seq_lens[b], kMlaBs, D, shard);
@@ -217,6 +280,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           int page;
           const bool ok = page_ok(p, si, b, j, &page);
           if (!ok) atomicOr(p.status, kDevBadPage);
+          if (kL2Ahead > 0) prefetch_next();
           uint8_t* dst = smem + kOffKV + st * kTileBytes;
           // box groups in the order they are freed: value boxes 0-3, value boxes 4-7, rope box
           // (the rope box holds the page's P^T tile until its PV product is done)
@@ -605,40 +669,99 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         named_bar_sync(2, kSoftmaxThreads);
         if (misc->bcast) {
           __threadfence();
-          const int w8 = ts >> 5;
-          for (int r = w8; r < kMlaHeads; r += kSoftmaxWarps) {
-            float mx = -INFINITY;
-            for (int c = c0; c <= c1; ++c) {
-              const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-              mx = fmaxf(mx, __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + r));
-            }
-            float4 acc[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            float wsum = 0.f;
-            if (mx != -INFINITY) {
+          const int np = c1 - c0 + 1;
+          if (np <= kCombineMax) {
+            // Weights of every (piece, row) first, one thread per row, into shared memory;
+            // then every thread merges 16-byte chunks of the rows with all of its loads
+            // independent of one another (8 rows at a time, every piece), so the pieces
+            // stream from L2 with many requests in flight instead of one row at a time.
+            float* wt = reinterpret_cast<float*>(smem + kOffW);  // [piece][row]
+            if (ts < kMlaHeads) {
+              float mx = -INFINITY;
               for (int c = c0; c <= c1; ++c) {
                 const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-                const float* sl = p.slots + ((size_t)k * ql + jq) * p.slot_floats;
-                const float lk = __ldcg(sl + kMlaHeads * kMlaDv + r);
-                const float w = lk == -INFINITY ? 0.f : exp2f(lk - mx);
+                mx = fmaxf(mx, __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + ts));
+              }
+              float wsum = 0.f;
+              for (int i = 0; i < np; ++i) {
+                const int c = c0 + i, k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                const float lk = __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + ts);
+                const float w = (mx == -INFINITY || lk == -INFINITY) ? 0.f : exp2f(lk - mx);
                 wsum += w;
-                const float4* src = reinterpret_cast<const float4*>(sl + (size_t)r * kMlaDv) + lane * 4;
+                wt[i * kMlaHeads + ts] = w;
+              }
+              misc->inv_l[ts] = wsum > 0.f ? 1.f / wsum : 0.f;
+              Lout[ts] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+            }
+            named_bar_sync(2, kSoftmaxThreads);
+            const int ch = ts & 127, rh = ts >> 7;  // chunk of a row; rows 2u + rh
+#pragma unroll 1
+            for (int u0 = 0; u0 < kMlaHeads / 2; u0 += 8) {
+              float4 acc[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float4 x = __ldcg(src + i);
-                  acc[i].x += w * x.x;
-                  acc[i].y += w * x.y;
-                  acc[i].z += w * x.z;
-                  acc[i].w += w * x.w;
+              for (int u = 0; u < 8; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+              for (int i = 0; i < np; ++i) {
+                const int c = c0 + i, k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                const float4* src = reinterpret_cast<const float4*>(p.slots + ((size_t)k * ql + jq) * p.slot_floats) + ch;
+                float4 x[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) x[u] = __ldcg(src + (size_t)(2 * (u0 + u) + rh) * (kMlaDv / 4));
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                  const float w = wt[i * kMlaHeads + 2 * (u0 + u) + rh];
+                  acc[u].x += w * x[u].x;
+                  acc[u].y += w * x[u].y;
+                  acc[u].z += w * x[u].z;
+                  acc[u].w += w * x[u].w;
                 }
               }
-            }
-            const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-            float4* out = reinterpret_cast<float4*>(Oout + (size_t)r * kMlaDv) + lane * 4;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) out[i] = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
-            if (lane == 0) Lout[r] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+              for (int u = 0; u < 8; ++u) {
+                const int r = 2 * (u0 + u) + rh;
+                const float inv = misc->inv_l[r];
+                reinterpret_cast<float4*>(Oout + (size_t)r * kMlaDv)[ch] =
+                    make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
+              }
+            }
+          } else {
+            // many pieces (a segment cut across more than kCombineMax CTAs): row by row
+            const int w8 = ts >> 5;
+            for (int r = w8; r < kMlaHeads; r += kSoftmaxWarps) {
+              float mx = -INFINITY;
+              for (int c = c0; c <= c1; ++c) {
+                const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                mx = fmaxf(mx, __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + r));
+              }
+              float4 acc[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+              float wsum = 0.f;
+              if (mx != -INFINITY) {
+                for (int c = c0; c <= c1; ++c) {
+                  const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                  const float* sl = p.slots + ((size_t)k * ql + jq) * p.slot_floats;
+                  const float lk = __ldcg(sl + kMlaHeads * kMlaDv + r);
+                  const float w = lk == -INFINITY ? 0.f : exp2f(lk - mx);
+                  wsum += w;
+                  const float4* src = reinterpret_cast<const float4*>(sl + (size_t)r * kMlaDv) + lane * 4;
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const float4 x = __ldcg(src + i);
+                    acc[i].x += w * x.x;
+                    acc[i].y += w * x.y;
+                    acc[i].z += w * x.z;
+                    acc[i].w += w * x.w;
+                  }
+                }
+              }
+              const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+              float4* out = reinterpret_cast<float4*>(Oout + (size_t)r * kMlaDv) + lane * 4;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                out[i] = make_float4(acc[i].x * inv, acc[i].y * inv, acc[i].z * inv, acc[i].w * inv);
+              if (lane == 0) Lout[r] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+            }
           }
           if (ts == 0) *ctr = 0;  // ready for the next call
         }
@@ -685,6 +808,7 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   if (q_rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;
   if (encode_tiled_2d(&p.qmap, q, kMlaDqk, q_rows, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS) return DCP_ERR_CUDA;
   for (int si = 0; si < set.n; ++si) {
+    p.pool[si] = static_cast<const uint8_t*>(set.pool[si]);
     p.table[si] = set.table[si];
     p.O[si] = set.O[si];
     p.LSE[si] = set.LSE[si];

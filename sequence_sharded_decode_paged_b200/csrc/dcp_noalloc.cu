@@ -98,3 +98,20 @@ extern "C" DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc
   if (cudaGetLastError() != cudaSuccess) return DCP_ERR_CUDA;
   return launch_gqa_decode(*desc, D, set, q, seq_lens, scratch, kNoAllocScratchBytes, cs);
 }
+
+// Status word of the scratch (word 0, the same bits as a workspace's): read through
+// the device address looked up for this device, then cleared, like dcp_read_device_error.
+extern "C" DCP_API dcp_status dcp_noalloc_read_device_error(int32_t* error_out, void* stream) {
+  if (error_out == nullptr) return DCP_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  dcp_status st = scratch_address(&scratch);
+  if (st != DCP_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return DCP_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return DCP_ERR_CUDA;
+  noalloc_clear_kernel<<<1, 32, 0, cs>>>(static_cast<uint32_t*>(scratch), 1);
+  if (cudaGetLastError() != cudaSuccess) return DCP_ERR_CUDA;
+  *error_out = v;
+  return DCP_OK;
+}

@@ -28,7 +28,8 @@ EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_b
             "dcp_block_table_extent_rule", "dcp_build_block_table_rule",
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
-            "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_grow_block_table", "dcp_append_kv"]
+            "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_noalloc_read_device_error",
+            "dcp_grow_block_table", "dcp_append_kv", "dcp_host_step_staging_bytes", "dcp_decode_step_host"]
 
 
 class DcpError(RuntimeError):
@@ -68,6 +69,9 @@ def _load() -> C.CDLL:
         "dcp_read_device_error": (C.c_int, [p, p, p]),
         "dcp_validate_config": (C.c_int, [i32, i32, i32, i32]),
         "dcp_decode_partial_all_noalloc": (C.c_int, [p, p, p, p, p, p, i32, p, p, p]),
+        "dcp_noalloc_read_device_error": (C.c_int, [p, p]),
+        "dcp_host_step_staging_bytes": (sz, [p, i32]),
+        "dcp_decode_step_host": (C.c_int, [p, i32, p, p, p, p, p, p, sz, p, sz, p, p, p]),
         "dcp_grow_block_table": (C.c_int, [p, p, i32, i32, i32, i32, p, p, p, p]),
         "dcp_append_kv": (C.c_int, [p, i32, p, p, p, p, p, p, p, p]),
     }
@@ -103,6 +107,21 @@ def _stream(stream) -> Optional[int]:
         return int(stream) if isinstance(stream, int) else int(stream.cuda_stream)
     import torch
     return int(torch.cuda.current_stream().cuda_stream) if torch.cuda.is_available() else None
+
+
+def _haddr(x) -> Optional[int]:
+    """Address of a host buffer: a numpy array, a CPU torch tensor or a raw integer address."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        if not x.flags.c_contiguous:
+            raise TypeError("host arrays must be C-contiguous")
+        return int(x.ctypes.data)
+    if x.is_cuda:
+        raise TypeError("expected a host buffer, got a CUDA tensor")
+    return int(x.data_ptr())
 
 
 def _ptr_array(xs):
@@ -228,6 +247,30 @@ def dcp_decode_partial_all_noalloc(desc: dcp_attn_desc, q, kv_pools, pool_pages,
     _check("dcp_decode_partial_all_noalloc", _lib.dcp_decode_partial_all_noalloc(
         C.byref(desc), _addr(q), _ptr_array(kv_pools), pp.ctypes.data, _ptr_array(tables), _addr(seq_lens), D,
         _ptr_array(O_parts), _ptr_array(LSE_parts), _stream(stream)))
+
+
+def dcp_noalloc_read_device_error(stream=None) -> int:
+    """Read and clear the status word of the allocation-free call's scratch (synchronous)."""
+    err = C.c_int32(0)
+    _check("dcp_noalloc_read_device_error", _lib.dcp_noalloc_read_device_error(C.addressof(err), _stream(stream)))
+    return int(err.value)
+
+
+def dcp_host_step_staging_bytes(desc: dcp_attn_desc, D: int) -> int:
+    return int(_lib.dcp_host_step_staging_bytes(C.byref(desc), D))
+
+
+def dcp_decode_step_host(desc: dcp_attn_desc, D: int, host_q, host_seq_lens, host_tables, kv_pools, pool_pages,
+                         staging, workspace, host_O, host_LSE=None, staging_bytes: Optional[int] = None,
+                         workspace_bytes: Optional[int] = None, stream=None) -> None:
+    """One decode step with host inputs and outputs (see include/dcp.h); asynchronous on ``stream``."""
+    sb = staging_bytes if staging_bytes is not None else staging.numel() * staging.element_size()
+    wb = workspace_bytes if workspace_bytes is not None else workspace.numel() * workspace.element_size()
+    pp = _i32(pool_pages)
+    _check("dcp_decode_step_host", _lib.dcp_decode_step_host(
+        C.byref(desc), D, _haddr(host_q), _haddr(host_seq_lens), _haddr(host_tables), _ptr_array(kv_pools),
+        pp.ctypes.data, _addr(staging), sb, _addr(workspace), wb, _haddr(host_O), _haddr(host_LSE),
+        _stream(stream)))
 
 
 def dcp_lse_merge(O_parts, LSE_parts, D: int, rows: int, d_v: int, O, LSE_out=None, stream=None) -> None:

@@ -313,6 +313,32 @@ DCP_API dcp_status dcp_decode_partial(const dcp_attn_desc *desc, const void *q, 
                               float *LSE_i, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * One shard's partial laid out for the exchange between D ranks of the
+ * multi-GPU form.  [P1 "A2 方法细节", step 3: after computing, the ranks
+ * all-gather their (O_i, LSE_i) and reduce-scatter the reweighted sum, so
+ * that every rank ends with the merged output of its own slice of heads.]
+ * n_owners ranks own consecutive slices of Hk = Hq / n_owners query heads
+ * (rank k: heads k*Hk .. k*Hk + Hk - 1).  The partial of dcp_decode_partial
+ * is written owner by owner into `send`, fp32, n_owners chunks of
+ * dcp_owner_chunk_floats(desc, n_owners) floats each:
+ *   chunk k:  O rows  [batch][q_len][Hk][head_dim_v]   (row (b, j, h) at
+ *                     ((b*q_len + j)*Hk + h - k*Hk) * head_dim_v),
+ *             then LSE rows [batch][q_len][Hk], padded to a multiple of 64 floats.
+ * Chunk k is what this rank sends to rank k in an all-to-all; a rank that
+ * receives chunk k from every shard merges them with dcp_lse_merge (O parts
+ * at the chunk starts, LSE parts after their O rows, rows = batch*q_len*Hk).
+ * With n_owners = 1 chunk 0 is dcp_decode_partial's O_i followed by LSE_i.
+ *   send       device fp32, n_owners * dcp_owner_chunk_floats(desc, n_owners) floats, 16-byte aligned.
+ * Other arguments, results and errors as dcp_decode_partial; DCP_ERR_INVALID_ARG
+ * if n_owners < 1 or it does not divide num_q_heads.
+ */
+DCP_API size_t dcp_owner_chunk_floats(const dcp_attn_desc *desc, int32_t n_owners);
+DCP_API dcp_status dcp_decode_partial_owner_major(const dcp_attn_desc *desc, const void *q, const void *kv_pool,
+                                                  int32_t pool_pages, const int32_t *table, const int32_t *seq_lens,
+                                                  int32_t shard, int32_t D, int32_t n_owners, float *send,
+                                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * All D partials in one launch.  Host arrays of D device pointers:
  * kv_pools[s], tables[s], O_parts[s], LSE_parts[s]; pool_pages host int32[D].
  * Each launch splits the concatenated page lists of its shards into equal

@@ -385,6 +385,36 @@ dcp_status dcp_decode_partial(const dcp_attn_desc* desc, const void* q, const vo
   return run_decode(desc, D, set, q, seq_lens, workspace, workspace_bytes, stream);
 }
 
+size_t dcp_owner_chunk_floats(const dcp_attn_desc* desc, int32_t n_owners) {
+  if (desc == nullptr || n_owners < 1 || desc->num_q_heads % n_owners != 0 || desc->batch < 1 || desc->q_len < 1)
+    return 0;
+  const size_t rows = (size_t)desc->batch * desc->q_len * (desc->num_q_heads / n_owners);
+  return rows * desc->head_dim_v + ((rows + 63) / 64) * 64;  // O rows, then LSE rows padded to 256 B
+}
+
+dcp_status dcp_decode_partial_owner_major(const dcp_attn_desc* desc, const void* q, const void* kv_pool,
+                                          int32_t pool_pages, const int32_t* table, const int32_t* seq_lens,
+                                          int32_t shard, int32_t D, int32_t n_owners, float* send,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  dcp_status st = check_decode_args(desc, D, q, seq_lens, workspace, workspace_bytes);
+  if (st != DCP_OK) return st;
+  if (shard < 0 || shard >= D || send == nullptr) return DCP_ERR_INVALID_ARG;
+  const size_t chunk = dcp_owner_chunk_floats(desc, n_owners);
+  if (chunk == 0) return DCP_ERR_INVALID_ARG;  // n_owners must divide the query heads
+  const size_t rows = (size_t)desc->batch * desc->q_len * (desc->num_q_heads / n_owners);
+  ShardSet set;
+  set.n = 1;
+  set.shard[0] = shard;
+  set.pool[0] = kv_pool;
+  set.pool_pages[0] = pool_pages;
+  set.table[0] = table;
+  set.O[0] = send;
+  set.LSE[0] = send + rows * desc->head_dim_v;
+  set.owner_heads = desc->num_q_heads / n_owners;
+  set.owner_stride = chunk;
+  return run_decode(desc, D, set, q, seq_lens, workspace, workspace_bytes, stream);
+}
+
 dcp_status dcp_decode_partial_all(const dcp_attn_desc* desc, const void* q, const void* const* kv_pools,
                                   const int32_t* pool_pages, const int32_t* const* tables, const int32_t* seq_lens,
                                   int32_t D, float* const* O_parts, float* const* LSE_parts, void* workspace,

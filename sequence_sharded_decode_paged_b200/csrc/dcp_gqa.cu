@@ -44,7 +44,13 @@
 namespace dcp {
 
 constexpr int kGqaConsumerWarps = 8;
-constexpr int kGqaThreads = (kGqaConsumerWarps + 1) * 32;
+#ifndef DCP_GQA_REGSPLIT
+#define DCP_GQA_REGSPLIT 0
+#endif
+// With the register split the producer is a whole warpgroup (one working thread) that hands
+// its registers to the two consumer warpgroups (setmaxnreg): 4*40 + 8*232 = 384*168 per lane.
+constexpr int kGqaProducerWarps = DCP_GQA_REGSPLIT ? 4 : 1;
+constexpr int kGqaThreads = (kGqaConsumerWarps + kGqaProducerWarps) * 32;
 constexpr int kScratchInts = 64;
 constexpr float kLn2 = 0.69314718055994530942f;
 
@@ -67,13 +73,32 @@ struct GqaParams {
   int hpc, n_hg, stages, wph;
   uint32_t stage_bytes;
   int slot_floats;
+  // Output layout: query heads are owned in consecutive slices of Hk heads, and owner k's
+  // O rows (and LSE rows) start k * own_stride floats after owner 0's.  The standard
+  // layout is Hk = Hq (a single owner).
+  int Hk;
+  size_t own_stride;
 };
 
-// Output row of head-group row rr = h * R + r (KV head kv0 + h, local row r =
-// query token r / G, head r % G) of request b: [b][r / G][(kv0 + h) * G + r % G].
-__device__ __forceinline__ size_t gqa_out_row(int rr, int b, int ql, int Hq, int kv0, int G, int R) {
+// Output row of head-group row rr = h * R + r (KV head kv0 + h, local row r = query token
+// r / G, head r % G) of request b, as (owner block, row within it): head = (kv0 + h) * G + r % G
+// lies in owner block head / Hk at row (b * ql + r / G) * Hk + head % Hk.
+struct OutRow {
+  int own;
+  size_t row;
+};
+__device__ __forceinline__ OutRow gqa_out_row(int rr, int b, int ql, int kv0, int G, int R, int Hk) {
   const int h = rr / R, r = rr - h * R, jq = r / G;
-  return ((size_t)b * ql + jq) * Hq + (size_t)(kv0 + h) * G + (r - jq * G);
+  const int head = (kv0 + h) * G + (r - jq * G);
+  const int own = head / Hk;
+  return {own, ((size_t)b * ql + jq) * Hk + (head - own * Hk)};
+}
+template <int HEAD_DIM>
+__device__ __forceinline__ float* gqa_o_ptr(const GqaParams& p, int si, OutRow o) {
+  return p.O[si] + o.own * p.own_stride + o.row * HEAD_DIM;
+}
+__device__ __forceinline__ float* gqa_l_ptr(const GqaParams& p, int si, OutRow o) {
+  return p.LSE[si] + o.own * p.own_stride + o.row;
 }
 
 template <int HEAD_DIM, bool KV8>
@@ -239,8 +264,11 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   const int S = p.n_si * B;
 
   // ------------------------------------------------------------------ producer
-  if (warp == kGqaConsumerWarps) {
-    if (lane != 0) return;
+  if (warp >= kGqaConsumerWarps) {
+#if DCP_GQA_REGSPLIT
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+#endif
+    if (warp != kGqaConsumerWarps || lane != 0) return;
     int stage = 0;
     uint32_t phase = 0;
     long issued = 0;
@@ -297,6 +325,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   }
 
   // ------------------------------------------------------------------ consumers
+#if DCP_GQA_REGSPLIT
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+#endif
   const int hpc = p.hpc, G = p.G, wph = p.wph, R = MULTI ? p.R : p.G, ql = MULTI ? p.q_len : 1;
   const int hu = MULTI ? hpc * p.rt : hpc;  // (KV head, row tile) units of one CTA; one tile if q_len = 1
   const bool active = warp < hu * wph;
@@ -320,12 +351,10 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
     if (c0 > cta) break;
     const int c1 = seg_last_cta(pre, n, T, P);
     if (n == 0) {  // no token of this request in this shard
-      float* Obase = p.O[si];
-      float* Lbase = p.LSE[si];
       for (int i = tid; i < rows_hg * HEAD_DIM; i += kGqaConsumerWarps * 32)
-        Obase[gqa_out_row(i / HEAD_DIM, b, ql, p.Hq, hg * hpc, G, R) * HEAD_DIM + i % HEAD_DIM] = 0.f;
+        gqa_o_ptr<HEAD_DIM>(p, si, gqa_out_row(i / HEAD_DIM, b, ql, hg * hpc, G, R, p.Hk))[i % HEAD_DIM] = 0.f;
       for (int i = tid; i < rows_hg; i += kGqaConsumerWarps * 32)
-        Lbase[gqa_out_row(i, b, ql, p.Hq, hg * hpc, G, R)] = -INFINITY;
+        *gqa_l_ptr(p, si, gqa_out_row(i, b, ql, hg * hpc, G, R, p.Hk)) = -INFINITY;
       pre += n;
       continue;
     }
@@ -653,16 +682,14 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       const float lse1 = l1 > 0.f ? m1 + __log2f(l1) : -INFINITY;
       const float inv0 = l0 > 0.f ? p.v_scale / l0 : 0.f, inv1 = l1 > 0.f ? p.v_scale / l1 : 0.f;
       // destination rows: the outputs, or this CTA's slot (rows in head-group order)
-      float* Obase = p.O[si];
-      float* Lbase = p.LSE[si];
-      auto out_row = [=](int rr) { return gqa_out_row(rr, b, ql, p.Hq, hg * hpc, G, R); };
+      auto out_row = [=](int rr) { return gqa_out_row(rr, b, ql, hg * hpc, G, R, p.Hk); };
       const int r0 = tile * 16 + g4, r1 = r0 + 8;
       const bool row0 = r0 < R, row1 = r1 < R;
       float* sl = p.slots + ((size_t)slot * p.n_hg + hg) * p.slot_floats;
-      float* dO0 = complete ? Obase + out_row(hh * R + r0) * HEAD_DIM : sl + (size_t)(hh * R + r0) * HEAD_DIM;
-      float* dO1 = complete ? Obase + out_row(hh * R + r1) * HEAD_DIM : sl + (size_t)(hh * R + r1) * HEAD_DIM;
-      float* dL0 = complete ? Lbase + out_row(hh * R + r0) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r0;
-      float* dL1 = complete ? Lbase + out_row(hh * R + r1) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r1;
+      float* dO0 = complete ? gqa_o_ptr<HEAD_DIM>(p, si, out_row(hh * R + r0)) : sl + (size_t)(hh * R + r0) * HEAD_DIM;
+      float* dO1 = complete ? gqa_o_ptr<HEAD_DIM>(p, si, out_row(hh * R + r1)) : sl + (size_t)(hh * R + r1) * HEAD_DIM;
+      float* dL0 = complete ? gqa_l_ptr(p, si, out_row(hh * R + r0)) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r0;
+      float* dL1 = complete ? gqa_l_ptr(p, si, out_row(hh * R + r1)) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r1;
       if constexpr (KV8) {
         // n-tile i, column 2c (+1) holds dim 32c + i (+16): two runs of 16 consecutive dims
         if (row0) {
@@ -733,12 +760,11 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
             }
           }
           const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-          const size_t orow = gqa_out_row(r, b, ql, p.Hq, hg * hpc, G, R);
-          float* Obase = p.O[si];
-          float* Lbase = p.LSE[si];
+          const OutRow orow = gqa_out_row(r, b, ql, hg * hpc, G, R, p.Hk);
+          float* dO = gqa_o_ptr<HEAD_DIM>(p, si, orow);
 #pragma unroll
-          for (int i = 0; i < kPer; ++i) Obase[orow * HEAD_DIM + lane * kPer + i] = acc[i] * inv;
-          if (lane == 0) Lbase[orow] = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+          for (int i = 0; i < kPer; ++i) dO[lane * kPer + i] = acc[i] * inv;
+          if (lane == 0) *gqa_l_ptr(p, si, orow) = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
         }
         if (tid == 0) *ctr = 0;  // leave the counter ready for the next call
       }
@@ -807,6 +833,8 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);
   p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slots_off);
   p.slot_floats = L.slot_floats;
+  p.Hk = set.owner_heads > 0 ? set.owner_heads : d.num_q_heads;
+  p.own_stride = set.owner_stride;
   for (int si = 0; si < set.n; ++si) {
     p.table[si] = set.table[si];
     p.O[si] = set.O[si];

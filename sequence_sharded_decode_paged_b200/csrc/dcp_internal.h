@@ -22,6 +22,12 @@ struct ShardSet {
   const int32_t* table[kMaxShardsHost];
   float* O[kMaxShardsHost];
   float* LSE[kMaxShardsHost];
+  // Output layout.  owner_heads = 0: the standard [b][j][h] rows.  Otherwise query heads are
+  // owned in consecutive slices of owner_heads heads, row (b, j, h) goes to owner h / owner_heads
+  // at row (b * q_len + j) * owner_heads + h % owner_heads, and owner k's rows (O and LSE
+  // alike) start k * owner_stride floats after owner 0's.
+  int owner_heads = 0;
+  size_t owner_stride = 0;
 };
 
 // Workspace layout shared by the decode kernels.

@@ -29,7 +29,8 @@ EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_b
             "dcp_kv_page_bytes", "dcp_place_kv", "dcp_decode_workspace_bytes", "dcp_workspace_init",
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
             "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_noalloc_read_device_error",
-            "dcp_grow_block_table", "dcp_append_kv", "dcp_host_step_staging_bytes", "dcp_decode_step_host"]
+            "dcp_grow_block_table", "dcp_append_kv", "dcp_host_step_staging_bytes", "dcp_decode_step_host",
+            "dcp_owner_chunk_floats", "dcp_decode_partial_owner_major"]
 
 
 class DcpError(RuntimeError):
@@ -71,6 +72,8 @@ def _load() -> C.CDLL:
         "dcp_decode_partial_all_noalloc": (C.c_int, [p, p, p, p, p, p, i32, p, p, p]),
         "dcp_noalloc_read_device_error": (C.c_int, [p, p]),
         "dcp_host_step_staging_bytes": (sz, [p, i32]),
+        "dcp_owner_chunk_floats": (sz, [p, i32]),
+        "dcp_decode_partial_owner_major": (C.c_int, [p, p, p, i32, p, p, i32, i32, i32, p, p, sz, p]),
         "dcp_decode_step_host": (C.c_int, [p, i32, p, p, p, p, p, p, sz, p, sz, p, p, p]),
         "dcp_grow_block_table": (C.c_int, [p, p, i32, i32, i32, i32, p, p, p, p]),
         "dcp_append_kv": (C.c_int, [p, i32, p, p, p, p, p, p, p, p]),
@@ -229,6 +232,19 @@ def dcp_decode_partial(desc: dcp_attn_desc, q, kv_pool, pool_pages: int, table, 
     _check("dcp_decode_partial", _lib.dcp_decode_partial(
         C.byref(desc), _addr(q), _addr(kv_pool), pool_pages, _addr(table), _addr(seq_lens), shard, D, _addr(O_i),
         _addr(LSE_i), _addr(workspace), n, _stream(stream)))
+
+
+def dcp_owner_chunk_floats(desc: dcp_attn_desc, n_owners: int) -> int:
+    return int(_lib.dcp_owner_chunk_floats(C.byref(desc), n_owners))
+
+
+def dcp_decode_partial_owner_major(desc: dcp_attn_desc, q, kv_pool, pool_pages: int, table, seq_lens, shard: int,
+                                   D: int, n_owners: int, send, workspace, workspace_bytes: Optional[int] = None,
+                                   stream=None) -> None:
+    n = workspace_bytes if workspace_bytes is not None else workspace.numel() * workspace.element_size()
+    _check("dcp_decode_partial_owner_major", _lib.dcp_decode_partial_owner_major(
+        C.byref(desc), _addr(q), _addr(kv_pool), pool_pages, _addr(table), _addr(seq_lens), shard, D, n_owners,
+        _addr(send), _addr(workspace), n, _stream(stream)))
 
 
 def dcp_decode_partial_all(desc: dcp_attn_desc, q, kv_pools, pool_pages, tables, seq_lens, D: int, O_parts,

@@ -9,7 +9,17 @@ from gpu_cases import (D_INVARIANCE_TOL, LSE_TOL, O_BOUND_UNIT_AMP, O_TOL, asser
 
 pytestmark = pytest.mark.gpu
 
-HEADS_SAMPLE = [(0, 8), (56, 64)]  # head ranges checked on the big workloads
+# head ranges checked on the big workloads: one or more heads from each quarter of the 64
+HEADS_SAMPLE = [(0, 4), (16, 17), (32, 33), (48, 49), (60, 64)]
+HEADS_MIX = [(0, 1), (16, 17), (32, 33), (48, 49), (63, 64)]
+
+
+def _sample_requests(lens):
+    """The shortest, a middle-length and the longest request (the longest crosses the most
+    CTA boundaries and spans the widest score range)."""
+    lens = np.asarray(lens)
+    order = np.argsort(lens, kind="stable")
+    return sorted({int(order[0]), int(order[len(lens) // 2]), int(order[-1])})
 
 
 def _oracle(w, b, D, heads=None, src=None):
@@ -101,9 +111,7 @@ def test_full_size_workload_sampled(name):
     torch.cuda.synchronize()
     assert cache.device_error() == 0
     assert torch.isfinite(cache.O).all() and torch.isfinite(cache.LSE).all()
-    lens = np.array(w.seq_lens)
-    sample = sorted({int(lens.argmin()), int(np.argsort(lens)[len(lens) // 2])})
-    _check(w, D, cache, requests=sample, heads=HEADS_SAMPLE)
+    _check(w, D, cache, requests=_sample_requests(w.seq_lens), heads=HEADS_SAMPLE)
     del cache
     torch.cuda.empty_cache()
 
@@ -111,8 +119,7 @@ def test_full_size_workload_sampled(name):
 def test_agentic_mix_all_D_sampled_and_invariant():
     """256 requests, 17.8 M context tokens (20.5 GB of latent cache) at D = 1, 2, 4, 8."""
     w = synth.workload("mla_mix")
-    lens = np.array(w.seq_lens)
-    sample = sorted({int(lens.argmin()), int(np.argsort(lens)[128])})
+    sample = _sample_requests(w.seq_lens)
     ref = None
     for D in w.shards:
         cache, q = build_cache(w, D, device_kv=True)
@@ -122,7 +129,7 @@ def test_agentic_mix_all_D_sampled_and_invariant():
         O = cache.O.cpu().numpy()
         assert np.isfinite(O).all()
         if D in (1, 8):
-            _check(w, D, cache, requests=sample, heads=[(0, 4)])
+            _check(w, D, cache, requests=sample, heads=HEADS_MIX)
         if ref is None:
             ref = O
         else:

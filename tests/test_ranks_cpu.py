@@ -1,0 +1,137 @@
+"""The multi-GPU form of the method on CPU ranks: the exchange of owner-major partials.
+
+"Efficient Decode Context Parallelism with vLLM for Long Context Workloads",
+A2 方法细节, step 3: the D ranks exchange their partials (O_i, LSE_i) so that each
+ends with the merged output of its own slice of query heads.  Here every rank of
+a gloo group (2 or 4 spawned processes, no GPU) plays shard r: it takes its
+partial from the float64 oracle, lays it out in the owner-major order that
+include/dcp.h specifies for dcp_decode_partial_owner_major (written out again
+here from that specification), and runs the product's ``exchange``.  Checked:
+each rank receives, bit for bit, every shard's partial for its own heads, and
+merging them gives the direct (unsharded) attention of those heads to 1e-12.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import oracle
+import synth
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _chunk_floats(rows, d_v):
+    return rows * d_v + (rows + 63) // 64 * 64
+
+
+def _pack(Op, Lp, D, Hk, d_v, dtype):
+    """Owner-major send buffer of one shard: Op [B][Hq][d_v], Lp [B][Hq] -> D chunks of
+    (O rows [B][Hk][d_v], LSE rows [B][Hk], zero padding)."""
+    B = Op.shape[0]
+    rows = B * Hk
+    chunk = _chunk_floats(rows, d_v)
+    buf = np.zeros(D * chunk, dtype=dtype)
+    for k in range(D):
+        c = buf[k * chunk:(k + 1) * chunk]
+        c[:rows * d_v] = Op[:, k * Hk:(k + 1) * Hk, :].reshape(-1)
+        c[rows * d_v:rows * d_v + rows] = Lp[:, k * Hk:(k + 1) * Hk].reshape(-1)
+    return buf
+
+
+def _case(name):
+    if name == "gqa":
+        return synth.custom(synth.GQA, [130, 17, 300, 1], 8, 2, 64, 64, 16, seed=51)
+    return synth.custom(synth.MLA, [200, 64, 500], 64, 1, 576, 512, 64, seed=52)
+
+
+def _worker(rank, world, port, name, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import torch.distributed as dist
+    from sequence_sharded_decode_paged_b200 import ranks
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = _case(name)
+        D, Hq, d_v = world, w.num_q_heads, w.head_dim_v
+        Hk = Hq // D
+        res = [oracle.sharded(w.layout, Hq, w.num_kv_heads, w.head_dim_qk, d_v, w.query(b), w.kv_source(b),
+                              w.softmax_scale, w.block_size, D) for b in range(w.batch)]
+        Op = np.stack([r[2] for r in res])          # [B][D][Hq][d_v]
+        Lp = np.stack([r[3] for r in res])          # [B][D][Hq]
+        rows = w.batch * Hk
+        out = {}
+        for dtype, tname in ((np.float32, "f32"), (np.float64, "f64")):
+            send = torch.from_numpy(_pack(Op[:, rank], Lp[:, rank], D, Hk, d_v, dtype))
+            recv = torch.full_like(send, float("nan"))
+            ranks.exchange(send, recv)
+            Os, Ls = ranks.split_chunks(recv, D, rows, d_v)
+            mine = slice(rank * Hk, (rank + 1) * Hk)
+            exact = all(
+                np.array_equal(Os[j].numpy(), Op[:, j, mine, :].astype(dtype).reshape(rows, d_v)) and
+                np.array_equal(Ls[j].numpy(), Lp[:, j, mine].astype(dtype).reshape(rows))
+                for j in range(D))
+            O, L = oracle.merge(np.stack([o.numpy() for o in Os]).astype(np.float64),
+                                np.stack([l.numpy() for l in Ls]).astype(np.float64))
+            direct = [oracle.attend(w.layout, Hq, w.num_kv_heads, w.head_dim_qk, d_v, w.query(b), w.kv_source(b),
+                                    w.softmax_scale, w.block_size, 1, 0) for b in range(w.batch)]
+            Od = np.stack([x[0][mine] for x in direct]).reshape(rows, d_v)
+            Ld = np.stack([x[1][mine] for x in direct]).reshape(rows)
+            out[tname] = (exact, float(np.abs(O - Od).max()), float(np.abs(L - Ld).max()))
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, name):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, name, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    import queue as _queue
+    import time
+    out, t0 = {}, time.time()
+    while len(out) < world:
+        try:
+            r, res = q.get(timeout=2)
+            out[r] = res
+        except _queue.Empty:
+            dead = [p.exitcode for p in procs if p.exitcode not in (None, 0)]
+            assert not dead, f"a rank exited with {dead}"
+            assert time.time() - t0 < 300, "ranks did not finish"
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return out
+
+
+@pytest.mark.parametrize("world,name", [(2, "gqa"), (2, "mla"), (4, "gqa")])
+def test_exchange_gives_each_rank_its_heads(world, name):
+    out = _run(world, name)
+    assert sorted(out) == list(range(world))
+    for r, res in out.items():
+        exact32, dO32, dL32 = res["f32"]
+        exact64, dO64, dL64 = res["f64"]
+        assert exact32 and exact64, f"rank {r}: received partials differ from the shards' partials"
+        assert dO64 <= 1e-12 and dL64 <= 1e-12, f"rank {r}: merged float64 parts {dO64}, {dL64}"
+        assert dO32 <= 1e-6 and dL32 <= 1e-5, f"rank {r}: merged float32 parts {dO32}, {dL32}"
+
+
+def test_chunk_size_matches_the_library():
+    from sequence_sharded_decode_paged_b200 import dcp, ranks
+    for (B, ql, Hq, d_v, n) in [(2, 1, 8, 64, 2), (256, 1, 64, 512, 8), (3, 4, 64, 512, 4), (5, 2, 32, 128, 1)]:
+        desc = dcp.make_desc(dcp.DCP_LAYOUT_GQA, B, Hq, 8, d_v, d_v, 16, 4, 0.1, ql)
+        assert dcp.dcp_owner_chunk_floats(desc, n) == ranks.owner_chunk_floats(B, ql, Hq, d_v, n)
+        assert dcp.dcp_owner_chunk_floats(desc, n) % 64 == 0 or (B * ql * Hq // n * d_v) % 4 == 0
+    desc = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 2, 8, 2, 64, 64, 16, 4, 0.1)
+    assert dcp.dcp_owner_chunk_floats(desc, 3) == 0  # 3 owners do not split 8 heads

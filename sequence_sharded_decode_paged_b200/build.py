@@ -35,7 +35,7 @@ def build(force=False, verbose=False, extra_flags=()):
     if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra_flags, "-shared", "-o", tmp, *srcs, "-lcuda" if False else "-lrt"]
+    cmd = [_nvcc(), *NVCC_FLAGS, *extra_flags, "-shared", "-o", tmp, *srcs, "-lrt"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)

@@ -38,20 +38,32 @@
 //    (two token halves x two k halves) so that their latencies overlap.
 #include <float.h>
 
+#include <type_traits>
+
 #include "dcp_device.cuh"
 #include "dcp_internal.h"
 
 namespace dcp {
 
 constexpr int kGqaConsumerWarps = 8;
-#ifndef DCP_GQA_REGSPLIT
-#define DCP_GQA_REGSPLIT 0
-#endif
-// With the register split the producer is a whole warpgroup (one working thread) that hands
-// its registers to the two consumer warpgroups (setmaxnreg): 4*40 + 8*232 = 384*168 per lane.
-constexpr int kGqaProducerWarps = DCP_GQA_REGSPLIT ? 4 : 1;
+// The producer is a whole warpgroup (one working thread) so that it can hand its registers to
+// the two consumer warpgroups with setmaxnreg: at launch every thread has 168 registers (384
+// threads, three warps on some SM sub-partition); the producer group drops to 40 and the
+// consumers rise to 232, 4*40 + 8*232 = 12*168 per lane, so the split adds up to the launch's
+// allocation.  (With nine warps the consumers stayed at 168 and the FP8 and draft variants
+// spilled.)
+constexpr int kGqaProducerWarps = 4;
 constexpr int kGqaThreads = (kGqaConsumerWarps + kGqaProducerWarps) * 32;
+constexpr int kGqaProducerRegs = 40, kGqaConsumerRegs = 232;
+static_assert(kGqaProducerWarps * kGqaProducerRegs + kGqaConsumerWarps * kGqaConsumerRegs <=
+                  (kGqaProducerWarps + kGqaConsumerWarps) * 168, "register split must fit the launch allocation");
 constexpr int kScratchInts = 64;
+// Pages per step of the one-warp-per-head loop at block 16 (FP8 cache and draft tokens): more
+// pages give each warp more independent product chains and fewer softmax updates per token.
+#ifndef DCP_GQA_PAGES_PER_STEP
+#define DCP_GQA_PAGES_PER_STEP 2
+#endif
+constexpr int kPagesPerStep = DCP_GQA_PAGES_PER_STEP;
 constexpr float kLn2 = 0.69314718055994530942f;
 
 struct GqaParams {
@@ -265,9 +277,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
 
   // ------------------------------------------------------------------ producer
   if (warp >= kGqaConsumerWarps) {
-#if DCP_GQA_REGSPLIT
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
-#endif
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kGqaProducerRegs) : "memory");
     if (warp != kGqaConsumerWarps || lane != 0) return;
     int stage = 0;
     uint32_t phase = 0;
@@ -325,9 +335,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   }
 
   // ------------------------------------------------------------------ consumers
-#if DCP_GQA_REGSPLIT
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
-#endif
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kGqaConsumerRegs) : "memory");
   const int hpc = p.hpc, G = p.G, wph = p.wph, R = MULTI ? p.R : p.G, ql = MULTI ? p.q_len : 1;
   const int hu = MULTI ? hpc * p.rt : hpc;  // (KV head, row tile) units of one CTA; one tile if q_len = 1
   const bool active = warp < hu * wph;
@@ -416,117 +424,126 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       // its CTA streams few heads (several row tiles per head); single-token bf16 is HBM-bound
       // without it.
       if (wph == 1 && bs == 16) {
-        for (; j + 1 < e; j += 2) {
-          const int st0 = stage;
-          const uint32_t ph0 = phase;
-          const int st1 = stage + 1 == p.stages ? 0 : stage + 1;
-          const uint32_t ph1 = stage + 1 == p.stages ? phase ^ 1u : phase;
-          stage = st1 + 1 == p.stages ? 0 : st1 + 1;
-          phase = st1 + 1 == p.stages ? ph1 ^ 1u : ph1;
-          if (!dead && !mbar_wait(&full[st0], ph0)) {
-            atomicOr(p.status, kDevTimeout);
-            dead = true;
-          }
-          if (!dead && !mbar_wait(&full[st1], ph1)) {
-            atomicOr(p.status, kDevTimeout);
-            dead = true;
-          }
-          if (!dead && active) {
-            const bool ok0 = stage_ok[st0] != 0, ok1 = stage_ok[st1] != 0;
-            const int t0a = (g0 + j * gstride) * 16, t0b = (g0 + (j + 1) * gstride) * 16;
-            const int v0 = min(16, seq_len - t0a), v1 = min(16, seq_len - t0b);
-            const uint32_t kb0 = smem_u32(stage_mem + (size_t)st0 * p.stage_bytes);
-            const uint32_t kb1 = smem_u32(stage_mem + (size_t)st1 * p.stage_bytes);
-            float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-            if constexpr (KV8) {
-              if (ok0) kv8_scores(kb0, (uint32_t)(hh * 16), lane, qa, sa);
-              if (ok1) kv8_scores(kb1, (uint32_t)(hh * 16), lane, qa, sb);
-            } else {
-              if (ok0) bf16_scores(kb0, box_bytes, (uint32_t)(hh * 16), lane, qa, sa);
-              if (ok1) bf16_scores(kb1, box_bytes, (uint32_t)(hh * 16), lane, qa, sb);
-            }
-            // visible tokens of each page for rows g4 / g4 + 8 (a page that was not loaded adds nothing)
-            const int va0 = !ok0 ? 0 : (MULTI ? lim0 - t0a : v0), va1 = !ok0 ? 0 : (MULTI ? lim1 - t0a : v0);
-            const int vb0 = !ok1 ? 0 : (MULTI ? lim0 - t0b : v1), vb1 = !ok1 ? 0 : (MULTI ? lim1 - t0b : v1);
+        auto steps = [&](auto np_tag, int jj) {
+          constexpr int NP = decltype(np_tag)::value;
+          for (; jj + NP - 1 < e; jj += NP) {
+            int st[NP];
+            uint32_t ph[NP];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int tok = nt * 8 + c4 * 2 + (i & 1);
-                sa[nt][i] = tok < (i < 2 ? va0 : va1) ? sa[nt][i] * p.scale_log2 : -INFINITY;
-                sb[nt][i] = tok < (i < 2 ? vb0 : vb1) ? sb[nt][i] * p.scale_log2 : -INFINITY;
-              }
-            float mx0 = fmaxf(fmaxf(fmaxf(sa[0][0], sa[0][1]), fmaxf(sa[1][0], sa[1][1])),
-                              fmaxf(fmaxf(sb[0][0], sb[0][1]), fmaxf(sb[1][0], sb[1][1])));
-            float mx1 = fmaxf(fmaxf(fmaxf(sa[0][2], sa[0][3]), fmaxf(sa[1][2], sa[1][3])),
-                              fmaxf(fmaxf(sb[0][2], sb[0][3]), fmaxf(sb[1][2], sb[1][3])));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = mx0 > m0 ? ceilf(mx0) : m0, mn1 = mx1 > m1 ? ceilf(mx1) : m1;
-            const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
-            m0 = mn0;
-            m1 = mn1;
-            const float sub0 = mn0 == -INFINITY ? 0.f : mn0, sub1 = mn1 == -INFINITY ? 0.f : mn1;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              sa[nt][0] = ex2_approx(sa[nt][0] - sub0);
-              sa[nt][1] = ex2_approx(sa[nt][1] - sub0);
-              sa[nt][2] = ex2_approx(sa[nt][2] - sub1);
-              sa[nt][3] = ex2_approx(sa[nt][3] - sub1);
-              sb[nt][0] = ex2_approx(sb[nt][0] - sub0);
-              sb[nt][1] = ex2_approx(sb[nt][1] - sub0);
-              sb[nt][2] = ex2_approx(sb[nt][2] - sub1);
-              sb[nt][3] = ex2_approx(sb[nt][3] - sub1);
-            }
-            l0 = l0 * al0 + ((sa[0][0] + sa[0][1] + sa[1][0] + sa[1][1]) + (sb[0][0] + sb[0][1] + sb[1][0] + sb[1][1]));
-            l1 = l1 * al1 + ((sa[0][2] + sa[0][3] + sa[1][2] + sa[1][3]) + (sb[0][2] + sb[0][3] + sb[1][2] + sb[1][3]));
-            if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-              for (int i = 0; i < Geo::kNTiles; ++i) {
-                o[i][0] *= al0;
-                o[i][1] *= al0;
-                o[i][2] *= al1;
-                o[i][3] *= al1;
+            for (int k = 0; k < NP; ++k) {
+              st[k] = stage;
+              ph[k] = phase;
+              if (++stage == p.stages) {
+                stage = 0;
+                phase ^= 1u;
               }
             }
-            // values of tokens past the sequence end are zeroed (stale slots); causal masking
-            // within the sequence is carried by P = 0
-            if (ok0) {
-              if constexpr (KV8) {
-                const uint32_t pa[4] = {pack_f16x2(sa[0][0], sa[0][1]), pack_f16x2(sa[0][2], sa[0][3]),
-                                        pack_f16x2(sa[1][0], sa[1][1]), pack_f16x2(sa[1][2], sa[1][3])};
-                kv8_pv(kb0 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v0 < 16, keep_lo(c4, v0),
-                       keep_hi(c4, v0));
-              } else {
-                const uint32_t pa[4] = {pack_bf16x2(sa[0][0], sa[0][1]), pack_bf16x2(sa[0][2], sa[0][3]),
-                                        pack_bf16x2(sa[1][0], sa[1][1]), pack_bf16x2(sa[1][2], sa[1][3])};
-                bf16_pv(kb0 + Geo::kBoxes * box_bytes, box_bytes, (uint32_t)(hh * 16), lane, pa, o, v0 < 16,
-                        keep_lo(c4, v0), keep_hi(c4, v0));
+#pragma unroll
+            for (int k = 0; k < NP; ++k)
+              if (!dead && !mbar_wait(&full[st[k]], ph[k])) {
+                atomicOr(p.status, kDevTimeout);
+                dead = true;
+              }
+            if (!dead && active) {
+              bool ok[NP];
+              int vv[NP], t0[NP];
+              uint32_t kb[NP];
+              float sc[NP][2][4];
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                ok[k] = stage_ok[st[k]] != 0;
+                t0[k] = (g0 + (jj + k) * gstride) * 16;
+                vv[k] = min(16, seq_len - t0[k]);
+                kb[k] = smem_u32(stage_mem + (size_t)st[k] * p.stage_bytes);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) sc[k][nt][0] = sc[k][nt][1] = sc[k][nt][2] = sc[k][nt][3] = 0.f;
+              }
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                if constexpr (KV8) {
+                  if (ok[k]) kv8_scores(kb[k], (uint32_t)(hh * 16), lane, qa, sc[k]);
+                } else {
+                  if (ok[k]) bf16_scores(kb[k], box_bytes, (uint32_t)(hh * 16), lane, qa, sc[k]);
+                }
+              }
+              // visible tokens of each page for rows g4 / g4 + 8 (a page that was not loaded adds nothing)
+              float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                const int w0 = !ok[k] ? 0 : (MULTI ? lim0 - t0[k] : vv[k]);
+                const int w1 = !ok[k] ? 0 : (MULTI ? lim1 - t0[k] : vv[k]);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const int tok = nt * 8 + c4 * 2 + (i & 1);
+                    sc[k][nt][i] = tok < (i < 2 ? w0 : w1) ? sc[k][nt][i] * p.scale_log2 : -INFINITY;
+                  }
+                mx0 = fmaxf(mx0, fmaxf(fmaxf(sc[k][0][0], sc[k][0][1]), fmaxf(sc[k][1][0], sc[k][1][1])));
+                mx1 = fmaxf(mx1, fmaxf(fmaxf(sc[k][0][2], sc[k][0][3]), fmaxf(sc[k][1][2], sc[k][1][3])));
+              }
+              mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+              mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+              const float mn0 = mx0 > m0 ? ceilf(mx0) : m0, mn1 = mx1 > m1 ? ceilf(mx1) : m1;
+              const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
+              m0 = mn0;
+              m1 = mn1;
+              const float sub0 = mn0 == -INFINITY ? 0.f : mn0, sub1 = mn1 == -INFINITY ? 0.f : mn1;
+              float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                  sc[k][nt][0] = ex2_approx(sc[k][nt][0] - sub0);
+                  sc[k][nt][1] = ex2_approx(sc[k][nt][1] - sub0);
+                  sc[k][nt][2] = ex2_approx(sc[k][nt][2] - sub1);
+                  sc[k][nt][3] = ex2_approx(sc[k][nt][3] - sub1);
+                }
+                ls0 += sc[k][0][0] + sc[k][0][1] + sc[k][1][0] + sc[k][1][1];
+                ls1 += sc[k][0][2] + sc[k][0][3] + sc[k][1][2] + sc[k][1][3];
+              }
+              l0 = l0 * al0 + ls0;
+              l1 = l1 * al1 + ls1;
+              if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                for (int i = 0; i < Geo::kNTiles; ++i) {
+                  o[i][0] *= al0;
+                  o[i][1] *= al0;
+                  o[i][2] *= al1;
+                  o[i][3] *= al1;
+                }
+              }
+              // values of tokens past the sequence end are zeroed (stale slots); causal masking
+              // within the sequence is carried by P = 0
+#pragma unroll
+              for (int k = 0; k < NP; ++k) {
+                if (!ok[k]) continue;
+                if constexpr (KV8) {
+                  const uint32_t pa[4] = {pack_f16x2(sc[k][0][0], sc[k][0][1]), pack_f16x2(sc[k][0][2], sc[k][0][3]),
+                                          pack_f16x2(sc[k][1][0], sc[k][1][1]), pack_f16x2(sc[k][1][2], sc[k][1][3])};
+                  kv8_pv(kb[k] + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, vv[k] < 16,
+                         keep_lo(c4, vv[k]), keep_hi(c4, vv[k]));
+                } else {
+                  const uint32_t pa[4] = {pack_bf16x2(sc[k][0][0], sc[k][0][1]), pack_bf16x2(sc[k][0][2], sc[k][0][3]),
+                                          pack_bf16x2(sc[k][1][0], sc[k][1][1]), pack_bf16x2(sc[k][1][2], sc[k][1][3])};
+                  bf16_pv(kb[k] + Geo::kBoxes * box_bytes, box_bytes, (uint32_t)(hh * 16), lane, pa, o, vv[k] < 16,
+                          keep_lo(c4, vv[k]), keep_hi(c4, vv[k]));
+                }
               }
             }
-            if (ok1) {
-              if constexpr (KV8) {
-                const uint32_t pa[4] = {pack_f16x2(sb[0][0], sb[0][1]), pack_f16x2(sb[0][2], sb[0][3]),
-                                        pack_f16x2(sb[1][0], sb[1][1]), pack_f16x2(sb[1][2], sb[1][3])};
-                kv8_pv(kb1 + Geo::kBoxes * box_bytes, (uint32_t)(hh * 16), g4, c4, pa, o, v1 < 16, keep_lo(c4, v1),
-                       keep_hi(c4, v1));
-              } else {
-                const uint32_t pa[4] = {pack_bf16x2(sb[0][0], sb[0][1]), pack_bf16x2(sb[0][2], sb[0][3]),
-                                        pack_bf16x2(sb[1][0], sb[1][1]), pack_bf16x2(sb[1][2], sb[1][3])};
-                bf16_pv(kb1 + Geo::kBoxes * box_bytes, box_bytes, (uint32_t)(hh * 16), lane, pa, o, v1 < 16,
-                        keep_lo(c4, v1), keep_hi(c4, v1));
-              }
-            }
+            __syncwarp();
+            if (lane == 0)
+#pragma unroll
+              for (int k = 0; k < NP; ++k) mbar_arrive(&empty[st[k]]);
           }
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&empty[st0]);
-            mbar_arrive(&empty[st1]);
-          }
+          return jj;
+        };
+        if constexpr (kPagesPerStep > 2) {
+          if (p.stages >= kPagesPerStep + 2) j = steps(std::integral_constant<int, kPagesPerStep>{}, j);
         }
+        j = steps(std::integral_constant<int, 2>{}, j);
       }
     }
     for (; j < e; ++j) {
@@ -853,6 +870,13 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   auto kern = d.shard_rule == DCP_SHARD_INTERLEAVED ? gqa_decode_kernel<HEAD_DIM, MULTI, KV8, 0>
                                                     : gqa_decode_kernel<HEAD_DIM, MULTI, KV8, 1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return DCP_ERR_CUDA;
+  // setmaxnreg.inc waits until the registers it asks for are free: never launch a build whose
+  // launch allocation is smaller than the producer/consumer split
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return DCP_ERR_CUDA;
+  if (fa.numRegs * (kGqaProducerWarps + kGqaConsumerWarps) <
+      kGqaProducerWarps * kGqaProducerRegs + kGqaConsumerWarps * kGqaConsumerRegs)
     return DCP_ERR_CUDA;
   dim3 grid(L.nctas, p.n_hg);
   kern<<<grid, kGqaThreads, smem, st>>>(p);

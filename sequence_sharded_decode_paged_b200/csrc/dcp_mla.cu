@@ -403,7 +403,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const int tok = 32 * q4 + lane;                // token of the pair this thread holds
     const int slot = tok >> 6, trow = tok & 63;    // its page (0: a, 1: b) and row in that page
-    uint32_t od_ph = 0;
     long pc = 0;
     bool dead = false;
     int pre = plan.pre0;
@@ -540,9 +539,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             *reinterpret_cast<uint4*>(prow + ((((uint32_t)(4 * hf + c)) ^ (uint32_t)(tok & 7)) << 4)) = w4;
           }
         }
-        if (j > a) {  // O^T of the previous pair is complete: O^T may be rescaled
-          wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
-          od_ph ^= 1u;
+        if (resc) {
+          // O^T holds the earlier pairs: observe the previous pair's PV completion before
+          // rescaling it.  (That PV has finished by now -- it released the groups this pair's
+          // S^T needed -- so pairs without a rescale skip the wait.  The barrier completes
+          // once per pair and cannot pass this phase before this pair's P^T is ready, so the
+          // phase parity is the previous pair's index.)
+          wait_or_die_warp(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status);
           tc_fence_after();
         }
         if (resc && !dead) {
@@ -567,8 +570,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         ++pc;
       }
       // ---------------------------------------------------------- epilogue
-      wait_or_die_warp(&misc->o_done, od_ph, dead, p.status);
-      od_ph ^= 1u;
+      wait_or_die_warp(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status);  // the piece's last PV
       tc_fence_after();
       // row sums over the 128 token slots: over the warp's 32 (transposed), then the sub-partitions
       misc->part[q4][32 * hf + lane] = warp_transpose_reduce<false>(l, lane);
@@ -732,8 +734,18 @@ int mla_ctas(int q_len) {
   return n > 0 ? n : 1;
 }
 
+#ifndef DCP_MLA_X2
+#define DCP_MLA_X2 0
+#endif
+dcp_status launch_mla_decode_x2(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
+                                const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (DCP_MLA_X2) {
+    const dcp_status r = launch_mla_decode_x2(d, D, set, q, seq_lens, ws, ws_bytes, stream);
+    if (r != DCP_ERR_UNSUPPORTED) return r;
+  }
   WorkspaceLayout L;
   if (!workspace_layout(d, D, &L)) return DCP_ERR_UNSUPPORTED;
   if (ws_bytes < L.total) return DCP_ERR_CAPACITY;

@@ -70,13 +70,6 @@ static EncodeTiledFn encode_fn() {
 
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes) {
-  return encode_tiled_2d_swizzle(map, base, inner_elems, rows, row_stride_bytes, box_inner, box_rows, elem_bytes,
-                                 CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-CUresult encode_tiled_2d_swizzle(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes,
-                                 CUtensorMapSwizzle swizzle) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return CUDA_ERROR_NOT_SUPPORTED;
   cuuint64_t dims[2] = {inner_elems, rows};
@@ -84,7 +77,7 @@ CUresult encode_tiled_2d_swizzle(CUtensorMap* map, const void* base, uint64_t in
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
@@ -139,9 +132,7 @@ bool workspace_layout(const dcp_attn_desc& d, int D, WorkspaceLayout* L) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   L->status_off = 0;
   L->counters_off = 256;
-  // MLA pieces are counted per cluster rank (two counters per segment and query token)
-  const size_t ctr_per = d.layout == DCP_LAYOUT_MLA ? 2 : 1;
-  L->slots_off = L->counters_off + up((size_t)D * d.batch * L->n_hg * ctr_per * sizeof(int32_t));
+  L->slots_off = L->counters_off + up((size_t)D * d.batch * L->n_hg * sizeof(int32_t));
   L->total = L->slots_off + up((size_t)2 * L->nctas * L->n_hg * L->slot_floats * sizeof(float));
   return true;
 }

@@ -48,13 +48,9 @@ bool workspace_layout(const dcp_attn_desc& d, int D, WorkspaceLayout* out);
 // Device properties of the current device (cached per device ordinal).
 int device_sm_count();
 
-// cuTensorMapEncodeTiled obtained through the runtime's driver entry point (128-byte swizzle, or
-// the given one).
+// cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes = 2);
-CUresult encode_tiled_2d_swizzle(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                                 uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes,
-                                 CUtensorMapSwizzle swizzle);
 
 dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st);

@@ -734,18 +734,8 @@ int mla_ctas(int q_len) {
   return n > 0 ? n : 1;
 }
 
-#ifndef DCP_MLA_X2
-#define DCP_MLA_X2 0
-#endif
-dcp_status launch_mla_decode_x2(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
-                                const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream);
-
 dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (DCP_MLA_X2) {
-    const dcp_status r = launch_mla_decode_x2(d, D, set, q, seq_lens, ws, ws_bytes, stream);
-    if (r != DCP_ERR_UNSUPPORTED) return r;
-  }
   WorkspaceLayout L;
   if (!workspace_layout(d, D, &L)) return DCP_ERR_UNSUPPORTED;
   if (ws_bytes < L.total) return DCP_ERR_CAPACITY;

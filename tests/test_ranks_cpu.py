@@ -35,23 +35,43 @@ def _chunk_floats(rows, d_v):
 
 
 def _pack(Op, Lp, D, Hk, d_v, dtype):
-    """Owner-major send buffer of one shard: Op [B][Hq][d_v], Lp [B][Hq] -> D chunks of
-    (O rows [B][Hk][d_v], LSE rows [B][Hk], zero padding)."""
-    B = Op.shape[0]
-    rows = B * Hk
+    """Owner-major send buffer of one shard: Op [B][q_len][Hq][d_v], Lp [B][q_len][Hq] -> D chunks of
+    (O rows [B][q_len][Hk][d_v], LSE rows [B][q_len][Hk], zero padding)."""
+    rows = Op.shape[0] * Op.shape[1] * Hk
     chunk = _chunk_floats(rows, d_v)
     buf = np.zeros(D * chunk, dtype=dtype)
     for k in range(D):
         c = buf[k * chunk:(k + 1) * chunk]
-        c[:rows * d_v] = Op[:, k * Hk:(k + 1) * Hk, :].reshape(-1)
-        c[rows * d_v:rows * d_v + rows] = Lp[:, k * Hk:(k + 1) * Hk].reshape(-1)
+        c[:rows * d_v] = Op[:, :, k * Hk:(k + 1) * Hk, :].reshape(-1)
+        c[rows * d_v:rows * d_v + rows] = Lp[:, :, k * Hk:(k + 1) * Hk].reshape(-1)
     return buf
 
 
 def _case(name):
     if name == "gqa":
         return synth.custom(synth.GQA, [130, 17, 300, 1], 8, 2, 64, 64, 16, seed=51)
+    if name == "gqa_draft":  # three draft tokens per request, causal within the draft
+        return synth.custom(synth.GQA, [150, 3, 260], 8, 2, 64, 64, 16, seed=53, q_len=3)
     return synth.custom(synth.MLA, [200, 64, 500], 64, 1, 576, 512, 64, seed=52)
+
+
+def _partials(w, D):
+    """Per request: (O_parts [D][q_len][Hq][d_v], LSE_parts [D][q_len][Hq]) and the direct
+    attention (O [q_len][Hq][d_v], LSE [q_len][Hq]) over the unsharded cache."""
+    out = []
+    for b in range(w.batch):
+        args = (w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v)
+        if w.q_len == 1:
+            _, _, Op, Lp = oracle.sharded(*args, w.query(b), w.kv_source(b), w.softmax_scale, w.block_size, D)
+            Od, Ld = oracle.attend(*args, w.query(b), w.kv_source(b), w.softmax_scale, w.block_size, 1, 0)
+            out.append((Op[:, None], Lp[:, None], Od[None], Ld[None]))
+        else:
+            _, _, Op, Lp = oracle.sharded_mtp(*args, w.queries(b), w.kv_source(b), w.softmax_scale, w.q_len,
+                                              w.block_size, D)
+            Od, Ld = oracle.attend_mtp(*args, w.queries(b), w.kv_source(b), w.softmax_scale, w.q_len,
+                                       w.block_size, 1, 0)
+            out.append((Op, Lp, Od, Ld))
+    return out
 
 
 def _worker(rank, world, port, name, q):
@@ -61,31 +81,31 @@ def _worker(rank, world, port, name, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         w = _case(name)
-        D, Hq, d_v = world, w.num_q_heads, w.head_dim_v
+        D, Hq, d_v, ql = world, w.num_q_heads, w.head_dim_v, w.q_len
         Hk = Hq // D
-        res = [oracle.sharded(w.layout, Hq, w.num_kv_heads, w.head_dim_qk, d_v, w.query(b), w.kv_source(b),
-                              w.softmax_scale, w.block_size, D) for b in range(w.batch)]
-        Op = np.stack([r[2] for r in res])          # [B][D][Hq][d_v]
-        Lp = np.stack([r[3] for r in res])          # [B][D][Hq]
-        rows = w.batch * Hk
+        res = _partials(w, D)
+        Op = np.stack([r[0] for r in res])          # [B][D][q_len][Hq][d_v]
+        Lp = np.stack([r[1] for r in res])          # [B][D][q_len][Hq]
+        rows = w.batch * ql * Hk
+        mine = slice(rank * Hk, (rank + 1) * Hk)
+        Od = np.stack([r[2][:, mine] for r in res]).reshape(rows, d_v)
+        Ld = np.stack([r[3][:, mine] for r in res]).reshape(rows)
         out = {}
         for dtype, tname in ((np.float32, "f32"), (np.float64, "f64")):
             send = torch.from_numpy(_pack(Op[:, rank], Lp[:, rank], D, Hk, d_v, dtype))
             recv = torch.full_like(send, float("nan"))
             ranks.exchange(send, recv)
             Os, Ls = ranks.split_chunks(recv, D, rows, d_v)
-            mine = slice(rank * Hk, (rank + 1) * Hk)
             exact = all(
-                np.array_equal(Os[j].numpy(), Op[:, j, mine, :].astype(dtype).reshape(rows, d_v)) and
-                np.array_equal(Ls[j].numpy(), Lp[:, j, mine].astype(dtype).reshape(rows))
+                np.array_equal(Os[j].numpy(), Op[:, j, :, mine, :].astype(dtype).reshape(rows, d_v)) and
+                np.array_equal(Ls[j].numpy(), Lp[:, j, :, mine].astype(dtype).reshape(rows))
                 for j in range(D))
             O, L = oracle.merge(np.stack([o.numpy() for o in Os]).astype(np.float64),
                                 np.stack([l.numpy() for l in Ls]).astype(np.float64))
-            direct = [oracle.attend(w.layout, Hq, w.num_kv_heads, w.head_dim_qk, d_v, w.query(b), w.kv_source(b),
-                                    w.softmax_scale, w.block_size, 1, 0) for b in range(w.batch)]
-            Od = np.stack([x[0][mine] for x in direct]).reshape(rows, d_v)
-            Ld = np.stack([x[1][mine] for x in direct]).reshape(rows)
-            out[tname] = (exact, float(np.abs(O - Od).max()), float(np.abs(L - Ld).max()))
+            fin = ~np.isneginf(Ld)
+            dL = float(np.abs(L[fin] - Ld[fin]).max()) if fin.any() else 0.0
+            same_inf = bool(np.array_equal(np.isneginf(L), np.isneginf(Ld)))
+            out[tname] = (exact and same_inf, float(np.abs(O - Od).max()), dL)
         q.put((rank, out))
     finally:
         dist.destroy_process_group()
@@ -115,7 +135,7 @@ def _run(world, name):
     return out
 
 
-@pytest.mark.parametrize("world,name", [(2, "gqa"), (2, "mla"), (4, "gqa")])
+@pytest.mark.parametrize("world,name", [(2, "gqa"), (2, "mla"), (4, "gqa"), (2, "gqa_draft")])
 def test_exchange_gives_each_rank_its_heads(world, name):
     out = _run(world, name)
     assert sorted(out) == list(range(world))

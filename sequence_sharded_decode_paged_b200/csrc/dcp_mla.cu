@@ -31,7 +31,9 @@
 //    for the next pair as soon as the PV tile that reads it (or, for the rope
 //    boxes, the whole PV) completes, and S^T of the next pair starts on the
 //    groups that have landed.  Query + pair stage fill the shared memory.
-//  * Warp 1: TMEM allocator and the single MMA-issuing thread.
+//  * Warp 1: TMEM allocator; one thread issues S^T.  Each issue loop is fully
+//    unrolled with constant descriptor steps: a lone issuing thread feeds the
+//    tensor pipe only as fast as its own instruction latency allows.
 //  * Warps 2-9: softmax in the transposed layout: thread t of warp w holds
 //    token 32*(w%4) + t of the pair and heads 32*((w-2)/4) .. +31.  The
 //    reference maximum of each head is an integer (log2 units), raised only
@@ -41,7 +43,10 @@
 //    reference".  Each thread keeps running sums of its token slot; they are
 //    reduced over the 128 slots once per segment.  Tokens past the sequence
 //    end are masked in S and their value rows zeroed in shared memory before
-//    the PV product, so stale cache contents never leak in.
+//    the PV product, so stale cache contents never leak in.  Once the group
+//    has written P^T (a hardware barrier), one of its threads issues the PV
+//    product itself -- no mbarrier hand-off to another warp.  One warp waits on
+//    each mbarrier for the group; the others sleep on a hardware barrier.
 //    Epilogue: O^T rows (value dims) are read from TMEM, normalised per head
 //    and stored with coalesced 128-byte writes.
 //  * Multi-token decode (q_len > 1): blockIdx.y is the query token j; the
@@ -92,8 +97,7 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
 
 struct MlaMisc {
-  uint64_t q_full, q_empty, kv_full[kGroups], kv_empty[kGroups], s_full[2], s_empty[2], p_full, o_done, o_free,
-      mma_done;
+  uint64_t q_full, q_empty, kv_full[kGroups], kv_empty[kGroups], s_full[2], s_empty[2], o_done, mma_done, pv_done;
   uint32_t tmem_base;
   int bcast;
   alignas(16) float mref[kMlaHeads];  // integral reference maxima (log2 units); read as float4
@@ -147,6 +151,37 @@ __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   return r != 0;
 }
 
+// tcgen05.mma with the descriptors passed as 32-bit halves: the issue loops add constant
+// (byte offset >> 4) steps to the low words only, which hold the start-address field (a
+// shared-memory offset below 256 KB never carries out of its 14 bits).  One thread issues
+// back to back, so its own instruction latency sets how fast the tensor pipe is fed.
+__device__ __forceinline__ void umma_bf16_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                             uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tmov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\ttcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// O^T += V^T P^T for one pair: 4 tiles of 128 value dims x KST 16-token steps, each tile
+// releasing the two value boxes it read, then the rope boxes (P^T) and the pair's O^T.
+// V^T: MN-major, 64-dim atoms one pair box apart; P^T: MN-major, one 64-head atom.
+template <int KST>
+__device__ __forceinline__ void issue_pv(uint32_t t_o, uint32_t v_lo, uint32_t v_hi, uint32_t p_lo, uint32_t p_hi,
+                                         uint32_t idO, uint32_t acc0, MlaMisc* misc) {
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+    for (int ks = 0; ks < KST; ++ks)
+      umma_bf16_lo(t_o + mt * 64, v_lo + ((2 * mt * kPairBox + ks * 2048) >> 4), v_hi, p_lo + ((ks * 2048) >> 4),
+                   p_hi, idO, ks > 0 ? 1u : acc0);
+    umma_commit(&misc->kv_empty[mt]);  // value boxes 2mt, 2mt+1 are free
+  }
+  umma_commit(&misc->kv_empty[4]);  // the rope boxes (P^T) are free
+  umma_commit(&misc->o_done);
+}
+
 // Wait unless the caller has already given up; a failed wait marks it dead.
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
   if (dead) return;
@@ -156,11 +191,15 @@ __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool
   }
 }
 
-// Warp-wide variant: the verdict is made uniform across the warp, because the
-// tcgen05.ld / st that follow are warp-collective.
-__device__ __forceinline__ void wait_or_die_warp(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
-  wait_or_die(bar, parity, dead, status);
-  dead = __any_sync(0xffffffffu, dead);
+// Softmax-group variant: one warp (the group's first) waits on the mbarrier while the
+// others sleep on hardware barrier `id`, which releases them with the verdict made uniform
+// across the group (the tcgen05.ld / st that follow are warp-collective).  A whole group
+// polling the mbarrier would keep the shared-memory port busy while the tensor core reads
+// its operands from there.
+__device__ __forceinline__ void wait_or_die_group(uint64_t* bar, uint32_t parity, bool& dead, int* status,
+                                                  bool waiter, int id, int nthreads) {
+  if (waiter) wait_or_die(bar, parity, dead, status);
+  dead = bar_red_or(id, nthreads, dead);
 }
 
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
@@ -224,10 +263,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       mbar_init(&misc->s_full[i], 1);
       mbar_init(&misc->s_empty[i], kSoftmaxWarps);
     }
-    mbar_init(&misc->p_full, kSoftmaxWarps);
     mbar_init(&misc->o_done, 1);
-    mbar_init(&misc->o_free, kSoftmaxWarps);
     mbar_init(&misc->mma_done, 1);
+    mbar_init(&misc->pv_done, 1);
     fence_barrier_init();
   }
   // The products read every row of the pair stage, also rows no page fills (a pair's
@@ -329,8 +367,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     // releasing the value boxes it read, and the rope boxes (P^T) last.
     if (lane == 0) {
       const uint32_t idS = idesc_bf16_f32(128, 64, false, false);
-      const uint32_t idO = idesc_bf16_f32(128, 64, true, true);
-      uint32_t q_ph = 0, of_ph = 0;
+      // K rows (A) and the query (B): K-major, one 8-row group per 1,024 bytes
+      const uint64_t k_desc = sw128_desc(smem_u32(smem + kOffKV), 16, 1024);
+      const uint64_t q_desc = sw128_desc(smem_u32(smem + kOffQ), 16, 1024);
+      const uint32_t k_lo = (uint32_t)k_desc, k_hi = (uint32_t)(k_desc >> 32);
+      const uint32_t q_lo = (uint32_t)q_desc, q_hi = (uint32_t)(q_desc >> 32);
+      uint32_t q_ph = 0;
       long pc = 0;
       bool dead = false;
       int pre = plan.pre0;
@@ -344,47 +386,26 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         wait_or_die(&misc->q_full, q_ph, dead, p.status);
         q_ph ^= 1u;
         for (int j = a; j < e && !dead; j += 2) {
-          const bool two = j + 1 < e;
+          // Per pair: S^T = K Q^T group by group as the groups land.  (The softmax group
+          // issues the pair's PV product itself once P^T is written.)
           const uint32_t sb = (uint32_t)(pc & 1), par = (uint32_t)(pc & 1);
           wait_or_die(&misc->s_empty[sb], (uint32_t)((pc >> 1) & 1) ^ 1u, dead, p.status);
           const uint32_t dS = tbase + kColS + sb * 64;
-          for (int g = 0; g < kGroups && !dead; ++g) {
+#pragma unroll
+          for (int g = 0; g < kGroups; ++g) {
             wait_or_die(&misc->kv_full[g], par, dead, p.status);
             if (dead) break;
             tc_fence_after();
-            for (int cb = group_box0(g); cb < group_box0(g) + group_boxes(g); ++cb) {
-              // descriptors advance by adding (byte offset >> 4) to the start-address field
-              const uint64_t ad = sw128_desc(smem_u32(smem + kOffKV + cb * kPairBox), 16, 1024);
-              const uint64_t bd = sw128_desc(smem_u32(smem + kOffQ + cb * kBlockBytes), 16, 1024);
+#pragma unroll
+            for (int cb = group_box0(g); cb < group_box0(g) + group_boxes(g); ++cb)
 #pragma unroll
               for (int ks = 0; ks < 4; ++ks)
-                umma_bf16(dS, ad + (uint64_t)((ks * 32) >> 4), bd + (uint64_t)((ks * 32) >> 4), idS,
-                          (cb > 0 || ks > 0) ? 1u : 0u);
-            }
+                umma_bf16_lo(dS, k_lo + ((cb * kPairBox + ks * 32) >> 4), k_hi, q_lo + ((cb * kBlockBytes + ks * 32) >> 4),
+                             q_hi, idS, (cb > 0 || ks > 0) ? 1u : 0u);
           }
           if (dead) break;
           umma_commit(&misc->s_full[sb]);
           if (j + 2 >= e) umma_commit(&misc->q_empty);  // Q is free once these products are done
-          wait_or_die(&misc->p_full, par, dead, p.status);
-          if (j == a) {  // the previous segment piece's epilogue must have read O^T
-            wait_or_die(&misc->o_free, of_ph ^ 1u, dead, p.status);
-            of_ph ^= 1u;
-          }
-          if (dead) break;
-          tc_fence_after();
-          // V^T: MN-major, 64-dim atoms one pair box apart; P^T: MN-major, one 64-head atom
-          const uint64_t bd = sw128_desc(smem_u32(smem + kOffPT), kPairBox, 1024);
-          const int kst = two ? 8 : 4;  // 16-token steps; the missing second page's are skipped
-#pragma unroll
-          for (int mt = 0; mt < 4; ++mt) {
-            const uint64_t ad = sw128_desc(smem_u32(smem + kOffKV + 2 * mt * kPairBox), kPairBox, 1024);
-            for (int ks = 0; ks < kst; ++ks)
-              umma_bf16(tbase + kColO + mt * 64, ad + (uint64_t)((ks * 2048) >> 4), bd + (uint64_t)((ks * 2048) >> 4),
-                        idO, (j > a || ks > 0) ? 1u : 0u);
-            umma_commit(&misc->kv_empty[mt]);  // value boxes 2mt, 2mt+1 are free
-          }
-          umma_commit(&misc->kv_empty[4]);  // the rope boxes (P^T) are free
-          umma_commit(&misc->o_done);
           ++pc;
         }
       }
@@ -402,6 +423,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     const int ts = tid - 64;                       // 0..255
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const int tok = 32 * q4 + lane;                // token of the pair this thread holds
+    const bool waiter = warp == 2;                 // the warp that waits on the group's mbarriers
+    const uint32_t idO = idesc_bf16_f32(128, 64, true, true);
+    const uint64_t v_desc = sw128_desc(smem_u32(smem + kOffKV), kPairBox, 1024);
+    const uint64_t p_desc = sw128_desc(smem_u32(smem + kOffPT), kPairBox, 1024);
+    const uint32_t v_lo = (uint32_t)v_desc, v_hi = (uint32_t)(v_desc >> 32);
+    const uint32_t p_lo = (uint32_t)p_desc, p_hi = (uint32_t)(p_desc >> 32);
     const int slot = tok >> 6, trow = tok & 63;    // its page (0: a, 1: b) and row in that page
     long pc = 0;
     bool dead = false;
@@ -454,7 +481,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         const bool mine_ok = slot == 0 ? oka : okb;
         const bool visible = mine_ok && trow < lim - (slot == 0 ? tok0a : tok0b);
         const uint32_t sb = (uint32_t)(pc & 1);
-        wait_or_die_warp(&misc->s_full[sb], (uint32_t)((pc >> 1) & 1), dead, p.status);
+        wait_or_die_group(&misc->s_full[sb], (uint32_t)((pc >> 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
         tc_fence_after();
         float s[32];
         if (!dead) {
@@ -545,7 +572,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           // S^T needed -- so pairs without a rescale skip the wait.  The barrier completes
           // once per pair and cannot pass this phase before this pair's P^T is ready, so the
           // phase parity is the previous pair's index.)
-          wait_or_die_warp(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status);
+          wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
           tc_fence_after();
         }
         if (resc && !dead) {
@@ -563,14 +590,22 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             }
           tmem_st_wait();
         }
+        // P^T rows (and zeroed value rows) to the async proxy, O^T rescales ordered before
+        // the barrier; then one thread issues the pair's PV product.  (The previous piece's
+        // epilogue read O^T before this barrier too, so a fresh accumulation may begin.)
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&misc->p_full);
+        named_bar_sync(2, kSoftmaxThreads);
+        if (waiter && lane == 0 && !dead) {
+          tc_fence_after();
+          const uint32_t acc0 = j > a ? 1u : 0u;  // O^T holds earlier pairs of this piece
+          if (two) issue_pv<8>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);
+          else issue_pv<4>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);  // no second page
+        }
         ++pc;
       }
       // ---------------------------------------------------------- epilogue
-      wait_or_die_warp(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status);  // the piece's last PV
+      wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);  // the piece's last PV
       tc_fence_after();
       // row sums over the 128 token slots: over the warp's 32 (transposed), then the sub-partitions
       misc->part[q4][32 * hf + lane] = warp_transpose_reduce<false>(l, lane);
@@ -606,9 +641,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         if (complete) *l_ptr(ts) = misc->lse2[ts] * kLn2;
         else slot_base[kMlaHeads * kMlaDv + ts] = misc->lse2[ts];
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&misc->o_free);
+      tc_fence_before();  // O^T reads complete before the next piece's first PV (ordered by its barrier)
       if (!complete) {
         __threadfence();
         named_bar_sync(2, kSoftmaxThreads);
@@ -715,6 +748,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         }
       }
       pre += n;
+    }
+    if (waiter && lane == 0) {  // every PV product issued here has completed before TMEM is released
+      umma_commit(&misc->pv_done);
+      bool d2 = false;
+      wait_or_die(&misc->pv_done, 0, d2, p.status);
     }
   }
 

@@ -101,6 +101,8 @@ struct MlaMisc {
   uint32_t tmem_base;
   int bcast;
   alignas(16) float mref[kMlaHeads];  // integral reference maxima (log2 units); read as float4
+  alignas(16) float msub[kMlaHeads];  // what the weights subtract: mref, or 0 while it is -inf
+  alignas(16) float thr[kMlaHeads];   // raise when s*scale - msub passes it: the threshold, or -inf
   float alpha[kMlaHeads];     // factors of the latest raise (exact powers of two)
   float inv_l[kMlaHeads];
   float lse2[kMlaHeads];
@@ -109,6 +111,7 @@ struct MlaMisc {
 };
 static_assert(sizeof(MlaMisc) <= kMiscBytes, "misc block");
 static_assert(offsetof(MlaMisc, mref) % 16 == 0, "float4 reads of the reference maxima");
+static_assert(offsetof(MlaMisc, msub) % 16 == 0 && offsetof(MlaMisc, thr) % 16 == 0, "float4 reads");
 static_assert(kOffMisc % 16 == 0, "misc block alignment");
 
 // Load group g: its first box and box count.
@@ -164,6 +167,16 @@ __device__ __forceinline__ void umma_bf16_lo(uint32_t d_tmem, uint32_t a_lo, uin
       : "memory");
 }
 
+// One lane of a converged warp (the lowest): the warp that issues tcgen05.mma stays
+// converged around the issue, which lets the issue run at the tensor pipe's pace (a lone lane
+// of a diverged warp issued the same products ~20 % slower in a microbenchmark).  Products and
+// the commits that track them are issued from the same elected lane.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t is;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(is));
+  return is != 0;
+}
+
 // O^T += V^T P^T for one pair: 4 tiles of 128 value dims x KST 16-token steps, each tile
 // releasing the two value boxes it read, then the rope boxes (P^T) and the pair's O^T.
 // V^T: MN-major, 64-dim atoms one pair box apart; P^T: MN-major, one 64-head atom.
@@ -182,6 +195,17 @@ __device__ __forceinline__ void issue_pv(uint32_t t_o, uint32_t v_lo, uint32_t v
   umma_commit(&misc->o_done);
 }
 
+// This thread's P^T row: its token's weights for heads 32*hf .. +31 as bf16, four 16-byte
+// chunks of the 128-byte-swizzled row.
+__device__ __forceinline__ void write_pt(uint8_t* prow, const float (&w)[32], int hf, int tok) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w4 = make_uint4(pack_bf16x2(w[8 * c + 0], w[8 * c + 1]), pack_bf16x2(w[8 * c + 2], w[8 * c + 3]),
+                                pack_bf16x2(w[8 * c + 4], w[8 * c + 5]), pack_bf16x2(w[8 * c + 6], w[8 * c + 7]));
+    *reinterpret_cast<uint4*>(prow + ((((uint32_t)(4 * hf + c)) ^ (uint32_t)(tok & 7)) << 4)) = w4;
+  }
+}
+
 // Wait unless the caller has already given up; a failed wait marks it dead.
 __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
   if (dead) return;
@@ -189,6 +213,12 @@ __device__ __forceinline__ void wait_or_die(uint64_t* bar, uint32_t parity, bool
     atomicOr(status, kDevTimeout);
     dead = true;
   }
+}
+
+// Warp-wide variant: the verdict is made uniform across the warp.
+__device__ __forceinline__ void wait_or_die_warp(uint64_t* bar, uint32_t parity, bool& dead, int* status) {
+  wait_or_die(bar, parity, dead, status);
+  dead = __any_sync(0xffffffffu, dead);
 }
 
 // Softmax-group variant: one warp (the group's first) waits on the mbarrier while the
@@ -361,11 +391,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Per pair, in order: S^T = K Q^T group by group as the groups land; then,
-    // once the softmax has written P^T, O^T += V^T P^T tile by tile, each tile
-    // releasing the value boxes it read, and the rope boxes (P^T) last.
-    if (lane == 0) {
+    // ------------------------------------------------------------ S^T issuer
+    {  // the whole warp walks the pairs and waits; an elected lane issues
       const uint32_t idS = idesc_bf16_f32(128, 64, false, false);
       // K rows (A) and the query (B): K-major, one 8-row group per 1,024 bytes
       const uint64_t k_desc = sw128_desc(smem_u32(smem + kOffKV), 16, 1024);
@@ -383,33 +410,40 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
         pre += n;
         if (n == 0) continue;
-        wait_or_die(&misc->q_full, q_ph, dead, p.status);
+        wait_or_die_warp(&misc->q_full, q_ph, dead, p.status);
         q_ph ^= 1u;
         for (int j = a; j < e && !dead; j += 2) {
           // Per pair: S^T = K Q^T group by group as the groups land.  (The softmax group
           // issues the pair's PV product itself once P^T is written.)
           const uint32_t sb = (uint32_t)(pc & 1), par = (uint32_t)(pc & 1);
-          wait_or_die(&misc->s_empty[sb], (uint32_t)((pc >> 1) & 1) ^ 1u, dead, p.status);
+          wait_or_die_warp(&misc->s_empty[sb], (uint32_t)((pc >> 1) & 1) ^ 1u, dead, p.status);
           const uint32_t dS = tbase + kColS + sb * 64;
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
-            wait_or_die(&misc->kv_full[g], par, dead, p.status);
+            wait_or_die_warp(&misc->kv_full[g], par, dead, p.status);
             if (dead) break;
             tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-            for (int cb = group_box0(g); cb < group_box0(g) + group_boxes(g); ++cb)
+              for (int cb = group_box0(g); cb < group_box0(g) + group_boxes(g); ++cb)
 #pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                umma_bf16_lo(dS, k_lo + ((cb * kPairBox + ks * 32) >> 4), k_hi, q_lo + ((cb * kBlockBytes + ks * 32) >> 4),
-                             q_hi, idS, (cb > 0 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < 4; ++ks)
+                  umma_bf16_lo(dS, k_lo + ((cb * kPairBox + ks * 32) >> 4), k_hi,
+                               q_lo + ((cb * kBlockBytes + ks * 32) >> 4), q_hi, idS, (cb > 0 || ks > 0) ? 1u : 0u);
+            }
+            __syncwarp();
           }
           if (dead) break;
-          umma_commit(&misc->s_full[sb]);
-          if (j + 2 >= e) umma_commit(&misc->q_empty);  // Q is free once these products are done
+          if (elect_one()) {
+            umma_commit(&misc->s_full[sb]);
+            if (j + 2 >= e) umma_commit(&misc->q_empty);  // Q is free once these products are done
+          }
+          __syncwarp();
           ++pc;
         }
       }
-      umma_commit(&misc->mma_done);  // everything issued has completed before TMEM is released
+      if (elect_one()) umma_commit(&misc->mma_done);  // everything issued has completed before TMEM is released
+      __syncwarp();
       bool d2 = false;
       wait_or_die(&misc->mma_done, 0, d2, p.status);
     }
@@ -469,9 +503,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       float l[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) l[i] = 0.f;
-      if (ts < kMlaHeads) misc->mref[ts] = -INFINITY;
+      if (ts < kMlaHeads) {
+        misc->mref[ts] = -INFINITY;
+        misc->msub[ts] = 0.f;
+        misc->thr[ts] = -INFINITY;
+      }
       named_bar_sync(2, kSoftmaxThreads);  // the references are reset before any thread reads them
-      const float4* mref4 = reinterpret_cast<const float4*>(misc->mref + 32 * hf);
+      const float4* msub4 = reinterpret_cast<const float4*>(misc->msub + 32 * hf);
+      const float4* thr4 = reinterpret_cast<const float4*>(misc->thr + 32 * hf);
       for (int j = a; j < e; j += 2) {
         const bool two = j + 1 < e;
         int pa = -1, pb = -1;
@@ -491,44 +530,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&misc->s_empty[sb]);
-        bool raise = false;
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 m4 = mref4[i4];
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int i = 4 * i4 + k;
-            s[i] = (visible && !dead) ? s[i] * p.scale_log2 : -INFINITY;
-            raise = raise || s[i] > mm[k] + kRescaleThreshold;
-          }
-        }
-        bool resc = false;
-        if (bar_red_or(2, kSoftmaxThreads, raise)) {
-          // exact maxima of the pair per head: over the warp's 32 tokens (transposed: lane
-          // i gets head 32*hf + i), then over the four sub-partitions; heads whose maximum
-          // passes their reference by more than the threshold get a new integral reference
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = s[i];
-          misc->part[q4][32 * hf + lane] = warp_transpose_reduce<true>(v, lane);
-          named_bar_sync(2, kSoftmaxThreads);
-          bool changed = false;
-          if (ts < kMlaHeads) {
-            const float pm = fmaxf(fmaxf(misc->part[0][ts], misc->part[1][ts]),
-                                   fmaxf(misc->part[2][ts], misc->part[3][ts]));
-            const float mo = misc->mref[ts];
-            float mn = mo;
-            if (mo == -INFINITY || pm > mo + kRescaleThreshold) mn = ceilf(pm);
-            const float al = mn == mo ? 1.f : exp2_int(mo - mn);
-            misc->alpha[ts] = al;
-            misc->mref[ts] = mn;
-            changed = al != 1.f;
-          }
-          resc = bar_red_or(2, kSoftmaxThreads, changed) && j > a;  // O^T holds earlier pairs
-#pragma unroll
-          for (int i = 0; i < 32; ++i) l[i] *= misc->alpha[32 * hf + i];
-        }
         // zero the value rows past the sequence end (dims 0..511) of the pair's pages:
         // they may hold stale values, which the zero weights must not multiply
 #pragma unroll 1
@@ -543,64 +544,114 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
                 make_uint4(0u, 0u, 0u, 0u);
           }
         }
-        // weights, running sums and this token's P^T row (heads 32*hf .. +31: four
-        // 16-byte chunks of the 128-byte-swizzled row)
+        const bool see = visible && !dead;
+        // Weights against the current references, optimistically: w = 2^(s*scale - m) in one FMA
+        // (m: the head's reference, 0 while it has none).  A score past its reference by more
+        // than the threshold -- or any visible score of a head without a reference -- makes the
+        // whole group redo the pair below after raising references; a piece's first pair
+        // (references just reset) goes there directly.  The OR barrier that takes that
+        // decision also tells the issuing thread that every P^T row is written.
+        bool raise = j == a;
+        if (!raise) {
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 m4 = mref4[i4];
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 m4 = msub4[i4], t4 = thr4[i4];
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, th[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int i = 4 * i4 + k;
-            // a head that has seen no visible token keeps -inf: subtract 0 so ex2 gives 0
-            s[i] = ex2_approx(s[i] - (mm[k] == -INFINITY ? 0.f : mm[k]));
-            l[i] += s[i];
-          }
-        }
-        if (!dead) {
-          uint8_t* prow = smem + kOffPT + tok * 128;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 w4 = make_uint4(pack_bf16x2(s[8 * c + 0], s[8 * c + 1]), pack_bf16x2(s[8 * c + 2], s[8 * c + 3]),
-                                        pack_bf16x2(s[8 * c + 4], s[8 * c + 5]), pack_bf16x2(s[8 * c + 6], s[8 * c + 7]));
-            *reinterpret_cast<uint4*>(prow + ((((uint32_t)(4 * hf + c)) ^ (uint32_t)(tok & 7)) << 4)) = w4;
-          }
-        }
-        if (resc) {
-          // O^T holds the earlier pairs: observe the previous pair's PV completion before
-          // rescaling it.  (That PV has finished by now -- it released the groups this pair's
-          // S^T needed -- so pairs without a rescale skip the wait.  The barrier completes
-          // once per pair and cannot pass this phase before this pair's P^T is ready, so the
-          // phase parity is the previous pair's index.)
-          wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
-          tc_fence_after();
-        }
-        if (resc && !dead) {
-#pragma unroll 1
-          for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
-#pragma unroll 1
-            for (int c = 0; c < 64; c += 32) {
-              float v[32];
-              const uint32_t ta = tbase + lane_off + kColO + mt * 64 + c;
-              tmem_ld32(ta, v);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= misc->alpha[c + i];
-              tmem_st32(ta, v);
+            for (int k = 0; k < 4; ++k) {
+              const int i = 4 * i4 + k;
+              const float t = see ? fmaf(s[i], p.scale_log2, -mm[k]) : -INFINITY;
+              raise = raise || t > th[k];
+              s[i] = ex2_approx(t);
             }
-          tmem_st_wait();
+          }
+          if (!dead) write_pt(smem + kOffPT + tok * 128, s, hf, tok);
         }
-        // P^T rows (and zeroed value rows) to the async proxy, O^T rescales ordered before
-        // the barrier; then one thread issues the pair's PV product.  (The previous piece's
-        // epilogue read O^T before this barrier too, so a fresh accumulation may begin.)
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // P^T rows and zeroed value rows -> the async proxy
         tc_fence_before();
-        named_bar_sync(2, kSoftmaxThreads);
-        if (waiter && lane == 0 && !dead) {
+        if (bar_red_or(2, kSoftmaxThreads, raise)) {
+          // ---- references move (rare): the pair's scores again (S^T buffer sb is rewritten
+          // only for a pair whose groups this pair's PV releases), exact maxima per head: over
+          // the warp's 32 tokens (transposed: lane i gets head 32*hf + i), then over the four
+          // sub-partitions; heads whose maximum passes their reference by more than the
+          // threshold get a new integral reference
+          tc_fence_after();
+          if (!dead && j != a) {  // (a piece's first pair skipped the weights: s still holds the scores)
+            tmem_ld32(tbase + lane_off + kColS + sb * 64 + 32 * hf, s);
+            tmem_ld_wait();
+          }
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = see ? s[i] * p.scale_log2 : -INFINITY;
+          misc->part[q4][32 * hf + lane] = warp_transpose_reduce<true>(v, lane);
+          named_bar_sync(2, kSoftmaxThreads);
+          bool changed = false;
+          if (ts < kMlaHeads) {
+            const float pm = fmaxf(fmaxf(misc->part[0][ts], misc->part[1][ts]),
+                                   fmaxf(misc->part[2][ts], misc->part[3][ts]));
+            const float mo = misc->mref[ts];
+            float mn = mo;
+            if (mo == -INFINITY || pm > mo + kRescaleThreshold) mn = ceilf(pm);
+            const float al = mn == mo ? 1.f : exp2_int(mo - mn);
+            misc->alpha[ts] = al;
+            misc->mref[ts] = mn;
+            misc->msub[ts] = mn == -INFINITY ? 0.f : mn;
+            misc->thr[ts] = mn == -INFINITY ? -INFINITY : kRescaleThreshold;
+            changed = al != 1.f;
+          }
+          const bool resc = bar_red_or(2, kSoftmaxThreads, changed) && j > a;  // O^T holds earlier pairs
+#pragma unroll
+          for (int i = 0; i < 32; ++i) l[i] *= misc->alpha[32 * hf + i];
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 m4 = msub4[i4];
+            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = 4 * i4 + k;
+              s[i] = ex2_approx(see ? fmaf(s[i], p.scale_log2, -mm[k]) : -INFINITY);
+            }
+          }
+          if (!dead) write_pt(smem + kOffPT + tok * 128, s, hf, tok);
+          if (resc) {
+            // O^T holds the earlier pairs: observe the previous pair's PV completion before
+            // rescaling it.  (That PV has finished by now -- it released the groups this pair's
+            // S^T needed -- so pairs without a rescale skip the wait.  The barrier completes
+            // once per pair and cannot pass this phase before this pair's PV is issued, so the
+            // phase parity is the previous pair's index.)
+            wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
+            tc_fence_after();
+            if (!dead) {
+#pragma unroll 1
+              for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
+#pragma unroll 1
+                for (int c = 0; c < 64; c += 32) {
+                  const uint32_t ta = tbase + lane_off + kColO + mt * 64 + c;
+                  tmem_ld32(ta, v);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) v[i] *= misc->alpha[c + i];
+                  tmem_st32(ta, v);
+                }
+              tmem_st_wait();
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          named_bar_sync(2, kSoftmaxThreads);  // P^T rewritten, O^T rescaled
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) l[i] += s[i];
+        // one thread issues the pair's PV product.  (The previous piece's epilogue read O^T
+        // before the barriers above, so a fresh accumulation may begin.)
+        if (waiter && !dead) {  // (dead is uniform across the group)
           tc_fence_after();
           const uint32_t acc0 = j > a ? 1u : 0u;  // O^T holds earlier pairs of this piece
-          if (two) issue_pv<8>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);
-          else issue_pv<4>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);  // no second page
+          if (elect_one()) {
+            if (two) issue_pv<8>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);
+            else issue_pv<4>(tbase + kColO, v_lo, v_hi, p_lo, p_hi, idO, acc0, misc);  // no second page
+          }
+          __syncwarp();
         }
         ++pc;
       }
@@ -749,8 +800,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       }
       pre += n;
     }
-    if (waiter && lane == 0) {  // every PV product issued here has completed before TMEM is released
-      umma_commit(&misc->pv_done);
+    if (waiter) {  // every PV product issued here has completed before TMEM is released
+      if (elect_one()) umma_commit(&misc->pv_done);
+      __syncwarp();
       bool d2 = false;
       wait_or_die(&misc->pv_done, 0, d2, p.status);
     }

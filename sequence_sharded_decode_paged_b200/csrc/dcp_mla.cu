@@ -97,7 +97,7 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
 
 struct MlaMisc {
-  uint64_t q_full, q_empty, kv_full[kGroups], kv_empty[kGroups], s_full[2], s_empty[2], o_done, mma_done, pv_done;
+  uint64_t q_full, q_empty, kv_full[kGroups], kv_empty[kGroups], s_full[2], s_empty[2], mma_done, pv_done;
   uint32_t tmem_base;
   int bcast;
   alignas(16) float mref[kMlaHeads];  // integral reference maxima (log2 units); read as float4
@@ -107,6 +107,7 @@ struct MlaMisc {
   float inv_l[kMlaHeads];
   float lse2[kMlaHeads];
   float part[4][kMlaHeads];   // per-sub-partition partial maxima or sums
+  size_t rowoff[kMlaHeads];   // epilogue / combine: float offset of head h's output row
   int scratch[32];
 };
 static_assert(sizeof(MlaMisc) <= kMiscBytes, "misc block");
@@ -191,8 +192,7 @@ __device__ __forceinline__ void issue_pv(uint32_t t_o, uint32_t v_lo, uint32_t v
                    p_hi, idO, ks > 0 ? 1u : acc0);
     umma_commit(&misc->kv_empty[mt]);  // value boxes 2mt, 2mt+1 are free
   }
-  umma_commit(&misc->kv_empty[4]);  // the rope boxes (P^T) are free
-  umma_commit(&misc->o_done);
+  umma_commit(&misc->kv_empty[4]);  // the rope boxes (P^T) are free, and the pair's O^T is complete
 }
 
 // This thread's P^T row: its token's weights for heads 32*hf .. +31 as bf16, four 16-byte
@@ -293,7 +293,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       mbar_init(&misc->s_full[i], 1);
       mbar_init(&misc->s_empty[i], kSoftmaxWarps);
     }
-    mbar_init(&misc->o_done, 1);
     mbar_init(&misc->mma_done, 1);
     mbar_init(&misc->pv_done, 1);
     fence_barrier_init();
@@ -619,7 +618,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             // S^T needed -- so pairs without a rescale skip the wait.  The barrier completes
             // once per pair and cannot pass this phase before this pair's PV is issued, so the
             // phase parity is the previous pair's index.)
-            wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
+            wait_or_die_group(&misc->kv_empty[4], (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
             tc_fence_after();
             if (!dead) {
 #pragma unroll 1
@@ -640,8 +639,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           tc_fence_before();
           named_bar_sync(2, kSoftmaxThreads);  // P^T rewritten, O^T rescaled
         }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) l[i] += s[i];
         // one thread issues the pair's PV product.  (The previous piece's epilogue read O^T
         // before the barriers above, so a fresh accumulation may begin.)
         if (waiter && !dead) {  // (dead is uniform across the group)
@@ -653,24 +650,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           }
           __syncwarp();
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) l[i] += s[i];  // (off the path to the PV issue)
         ++pc;
       }
       // ---------------------------------------------------------- epilogue
-      wait_or_die_group(&misc->o_done, (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);  // the piece's last PV
+      // the piece's last PV: its final commit (the rope group's release) marks O^T complete
+      wait_or_die_group(&misc->kv_empty[4], (uint32_t)((pc - 1) & 1), dead, p.status, waiter, 2, kSoftmaxThreads);
       tc_fence_after();
       // row sums over the 128 token slots: over the warp's 32 (transposed), then the sub-partitions
       misc->part[q4][32 * hf + lane] = warp_transpose_reduce<false>(l, lane);
+      const bool complete = (c0 == c1);
+      const int slot_i = complete ? 0 : 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
+      float* slot_base = p.slots + ((size_t)slot_i * ql + jq) * p.slot_floats;
+      float* const obase = complete ? p.O[si] : slot_base;
       named_bar_sync(2, kSoftmaxThreads);
       if (ts < kMlaHeads) {
         const float lt = (misc->part[0][ts] + misc->part[1][ts]) + (misc->part[2][ts] + misc->part[3][ts]);
         const float mh = misc->mref[ts];
         misc->inv_l[ts] = lt > 0.f ? 1.f / lt : 0.f;
         misc->lse2[ts] = lt > 0.f ? mh + __log2f(lt) : -INFINITY;
+        // row offsets once per piece, so that the stores below need no owner arithmetic
+        misc->rowoff[ts] = complete ? (size_t)(o_row(ts) - p.O[si]) : (size_t)ts * kMlaDv;
       }
       named_bar_sync(2, kSoftmaxThreads);
-      const bool complete = (c0 == c1);
-      const int slot_i = complete ? 0 : 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
-      float* slot_base = p.slots + ((size_t)slot_i * ql + jq) * p.slot_floats;
 #pragma unroll 1
       for (int mt = 2 * hf; mt < 2 * hf + 2; ++mt)
 #pragma unroll 1
@@ -680,12 +683,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             tmem_ld32(tbase + lane_off + kColO + mt * 64 + c, v);
             tmem_ld_wait();
           }
-          const int dv = mt * 128 + 32 * q4 + lane;
+          float* const col = obase + (mt * 128 + 32 * q4 + lane);  // this thread's value dim
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float inv = misc->inv_l[c + i];
-            float* dst = complete ? o_row(c + i) : slot_base + (size_t)(c + i) * kMlaDv;
-            dst[dv] = (inv == 0.f || dead) ? 0.f : v[i] * inv;
+            col[misc->rowoff[c + i]] = (inv == 0.f || dead) ? 0.f : v[i] * inv;
           }
         }
       if (ts < kMlaHeads) {
@@ -702,6 +704,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         if (misc->bcast) {
           __threadfence();
           const int np = c1 - c0 + 1;
+          // every piece's slot into L2 with one bulk prefetch each (pieces finished long ago may
+          // have left L2 under the cache stream): the loads below then wait on L2, not HBM
+          if (ts < np) {
+            const int c = c0 + ts, k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+            prefetch_l2_bulk(p.slots + ((size_t)k * ql + jq) * p.slot_floats, (uint32_t)p.slot_floats * 4u);
+          }
           if (np <= kCombineMax) {
             // Weights of every (piece, row) first, one thread per row, into shared memory;
             // then every thread merges 16-byte chunks of the rows with all of its loads
@@ -709,21 +717,31 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             // stream from L2 with many requests in flight instead of one row at a time.
             float* wt = reinterpret_cast<float*>(smem + kOffW);  // [piece][row]
             if (ts < kMlaHeads) {
-              float mx = -INFINITY;
-              for (int c = c0; c <= c1; ++c) {
-                const int k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-                mx = fmaxf(mx, __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + ts));
+              // every piece's LSE of this row loaded at once (one round trip), then the weights
+              float lk[kCombineMax];
+#pragma unroll
+              for (int i = 0; i < kCombineMax; ++i) {
+                lk[i] = -INFINITY;
+                if (i < np) {
+                  const int c = c0 + i, k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
+                  lk[i] = __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + ts);
+                }
               }
+              float mx = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < kCombineMax; ++i) mx = fmaxf(mx, lk[i]);
               float wsum = 0.f;
-              for (int i = 0; i < np; ++i) {
-                const int c = c0 + i, k = 2 * c + ((c == c0 && pre != c0 * P) ? 1 : 0);
-                const float lk = __ldcg(p.slots + ((size_t)k * ql + jq) * p.slot_floats + kMlaHeads * kMlaDv + ts);
-                const float w = (mx == -INFINITY || lk == -INFINITY) ? 0.f : exp2f(lk - mx);
-                wsum += w;
-                wt[i * kMlaHeads + ts] = w;
+#pragma unroll
+              for (int i = 0; i < kCombineMax; ++i) {
+                if (i < np) {
+                  const float w = (mx == -INFINITY || lk[i] == -INFINITY) ? 0.f : exp2f(lk[i] - mx);
+                  wsum += w;
+                  wt[i * kMlaHeads + ts] = w;
+                }
               }
               misc->inv_l[ts] = wsum > 0.f ? 1.f / wsum : 0.f;
               *l_ptr(ts) = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
+              misc->rowoff[ts] = (size_t)(o_row(ts) - p.O[si]);
             }
             named_bar_sync(2, kSoftmaxThreads);
             const int ch = ts & 127, rh = ts >> 7;  // chunk of a row; rows 2u + rh
@@ -752,7 +770,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               for (int u = 0; u < 8; ++u) {
                 const int r = 2 * (u0 + u) + rh;
                 const float inv = misc->inv_l[r];
-                reinterpret_cast<float4*>(o_row(r))[ch] =
+                reinterpret_cast<float4*>(p.O[si] + misc->rowoff[r])[ch] =
                     make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
               }
             }

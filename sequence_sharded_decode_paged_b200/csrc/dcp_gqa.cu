@@ -419,8 +419,11 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       // its CTA streams few heads (several row tiles per head); single-token bf16 is HBM-bound
       // without it.
       if (wph == 1 && bs == 16) {
-        auto steps = [&](auto np_tag, int jj) {
+        // LO: rows 8..15 of the warp's tile are empty (single-token decode with G <= 8): their
+        // maxima, weights, sums and rescales are skipped (zero weights, no ex2 issued).
+        auto steps = [&](auto np_tag, auto lo_tag, int jj) {
           constexpr int NP = decltype(np_tag)::value;
+          constexpr bool LO = decltype(lo_tag)::value;
           for (; jj + NP - 1 < e; jj += NP) {
             int st[NP];
             uint32_t ph[NP];
@@ -470,17 +473,19 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) {
+                  for (int i = 0; i < (LO ? 2 : 4); ++i) {
                     const int tok = nt * 8 + c4 * 2 + (i & 1);
                     sc[k][nt][i] = tok < (i < 2 ? w0 : w1) ? sc[k][nt][i] * p.scale_log2 : -INFINITY;
                   }
                 mx0 = fmaxf(mx0, fmaxf(fmaxf(sc[k][0][0], sc[k][0][1]), fmaxf(sc[k][1][0], sc[k][1][1])));
-                mx1 = fmaxf(mx1, fmaxf(fmaxf(sc[k][0][2], sc[k][0][3]), fmaxf(sc[k][1][2], sc[k][1][3])));
+                if (!LO) mx1 = fmaxf(mx1, fmaxf(fmaxf(sc[k][0][2], sc[k][0][3]), fmaxf(sc[k][1][2], sc[k][1][3])));
               }
               mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
               mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-              mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+              if (!LO) {
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+              }
               const float mn0 = mx0 > m0 ? ceilf(mx0) : m0, mn1 = mx1 > m1 ? ceilf(mx1) : m1;
               const float al0 = exp2_int(m0 - mn0), al1 = exp2_int(m1 - mn1);
               m0 = mn0;
@@ -493,21 +498,23 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
                 for (int nt = 0; nt < 2; ++nt) {
                   sc[k][nt][0] = ex2_approx(sc[k][nt][0] - sub0);
                   sc[k][nt][1] = ex2_approx(sc[k][nt][1] - sub0);
-                  sc[k][nt][2] = ex2_approx(sc[k][nt][2] - sub1);
-                  sc[k][nt][3] = ex2_approx(sc[k][nt][3] - sub1);
+                  sc[k][nt][2] = LO ? 0.f : ex2_approx(sc[k][nt][2] - sub1);
+                  sc[k][nt][3] = LO ? 0.f : ex2_approx(sc[k][nt][3] - sub1);
                 }
                 ls0 += sc[k][0][0] + sc[k][0][1] + sc[k][1][0] + sc[k][1][1];
-                ls1 += sc[k][0][2] + sc[k][0][3] + sc[k][1][2] + sc[k][1][3];
+                if (!LO) ls1 += sc[k][0][2] + sc[k][0][3] + sc[k][1][2] + sc[k][1][3];
               }
               l0 = l0 * al0 + ls0;
-              l1 = l1 * al1 + ls1;
-              if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+              if (!LO) l1 = l1 * al1 + ls1;
+              if (__any_sync(0xffffffffu, al0 != 1.f || (!LO && al1 != 1.f))) {
 #pragma unroll
                 for (int i = 0; i < Geo::kNTiles; ++i) {
                   o[i][0] *= al0;
                   o[i][1] *= al0;
-                  o[i][2] *= al1;
-                  o[i][3] *= al1;
+                  if (!LO) {
+                    o[i][2] *= al1;
+                    o[i][3] *= al1;
+                  }
                 }
               }
               // values of tokens past the sequence end are zeroed (stale slots); causal masking
@@ -536,7 +543,8 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
           return jj;
         };
         // two pages per step (four measured slower on the FP8 layer: 560 vs 497 us, fewer stages in flight)
-        j = steps(std::integral_constant<int, 2>{}, j);
+        if (!MULTI && R <= 8) j = steps(std::integral_constant<int, 2>{}, std::true_type{}, j);
+        else j = steps(std::integral_constant<int, 2>{}, std::false_type{}, j);
       }
     }
     for (; j < e; ++j) {

@@ -136,3 +136,19 @@ def test_agentic_mix_all_D_sampled_and_invariant():
             assert np.abs(O - ref).max() <= D_INVARIANCE_TOL
         del cache, q
         torch.cuda.empty_cache()
+
+
+def test_wide_score_range_raises_mid_piece():
+    """Scores spread over tens of log2 units (query amplitude 8: a score's standard deviation is
+    about 20 log2 units): the reference maxima are raised inside CTA pieces many pairs long
+    (D = 2, ~10 pairs per piece), so the pair redo and the rescale of O^T in tensor memory run
+    mid-piece, not only on a piece's first pair."""
+    w = synth.custom(synth.MLA, [120000, 70000, 333], 64, 1, 576, 512, 64, seed=91, q_amp=8.0)
+    D = 2
+    cache, q = build_cache(w, D, device_kv=True)
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    _check(w, D, cache, heads=HEADS_SAMPLE)
+    del cache
+    torch.cuda.empty_cache()

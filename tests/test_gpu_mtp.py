@@ -175,3 +175,13 @@ def test_per_shard_calls_agree_with_one_launch(layout, kv_dtype):
     inf = torch.isinf(a[1])
     assert torch.equal(torch.isinf(cache.LSE_parts), inf)
     assert (cache.LSE_parts[~inf] - a[1][~inf]).abs().max().item() <= 1e-4
+
+
+def test_mla_wide_score_range():
+    # query amplitude 8: reference raises (and O^T rescales) inside pieces of several pairs, per draft token
+    w = synth.custom(synth.MLA, [40000, 9000], 64, 1, 576, 512, 64, seed=95, q_len=2, q_amp=8.0)
+    cache, q = build_cache(w, 1, device_kv=True)
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    _check(w, 1, cache)

@@ -267,10 +267,13 @@ struct CtaPlan {
 
 // Block-wide planner for shard rule RULE.  Every thread of the block must call it.  `scratch`
 // holds at least (blockDim.x / 32 + 4) ints of shared memory.
+// seg_cost: units charged to every non-empty segment ahead of its pages (its fixed work: query
+// load, epilogue), so that the equal ranges balance work rather than pages.  The kernel loops
+// then advance `pre` by seg_cost before each non-empty segment's pages (0: pages only).
 template <int RULE>
 __device__ __forceinline__ CtaPlan plan_cta_r(const int32_t* __restrict__ seq_lens, int B, int n_si,
                                               const int* shard_of_si, int bs, int D, int cta, int nctas,
-                                              int* scratch) {
+                                              int* scratch, int seg_cost = 0) {
   const int S = n_si * B;
   const int nt = blockDim.x;
   const int tid = threadIdx.x;
@@ -280,7 +283,8 @@ __device__ __forceinline__ CtaPlan plan_cta_r(const int32_t* __restrict__ seq_le
   int local = 0;
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
-    local += local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
+    const int n = local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
+    local += n + (n > 0 ? seg_cost : 0);
   }
   // block exclusive scan of `local`
   const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
@@ -316,6 +320,7 @@ __device__ __forceinline__ CtaPlan plan_cta_r(const int32_t* __restrict__ seq_le
   for (int sid = s_begin; sid < s_end; ++sid) {
     const int si = sid / B, b = sid - si * B;
     const int n = local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
+    if (n > 0) pre += seg_cost;
     if (seg_last_cta(pre, n, T, P) >= cta) {
       atomicMin(&scratch[nw + 1], sid);
       break;
@@ -333,7 +338,8 @@ __device__ __forceinline__ CtaPlan plan_cta_r(const int32_t* __restrict__ seq_le
     int p2 = scratch[warp] + incl - local;
     for (int sid = s_begin; sid < plan.sid0; ++sid) {
       const int si = sid / B, b = sid - si * B;
-      p2 += local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
+      const int n = local_pages_r<RULE>(seq_lens[b], bs, D, shard_of_si[si]);
+      p2 += n + (n > 0 ? seg_cost : 0);
     }
     scratch[nw + 2] = p2;
   }

@@ -395,6 +395,21 @@ DCP_API dcp_status dcp_decode_partial_all_noalloc(const dcp_attn_desc *desc, con
 DCP_API dcp_status dcp_noalloc_read_device_error(int32_t *error_out, void *stream);
 
 /*
+ * Diagnostic of the decode kernels' bounded pipeline waits (no attention is
+ * computed).  One thread waits, through the same bounded wait the decode
+ * kernels use for every mbarrier, on a barrier that nothing ever arrives on;
+ * when the wait gives up (after about 4 s) it sets bit 1 of the workspace's
+ * status word, as a decode kernel does when a pipeline wait times out.
+ *   workspace  device, a workspace as for dcp_decode_partial (only its status
+ *              word, the first int32, is touched); read the bit back with
+ *              dcp_read_device_error.
+ * Asynchronous on `stream`; the stream is busy for the wait limit.  Nothing
+ * is left in flight when the wait gives up, so the CUDA context stays usable.
+ * Errors: DCP_ERR_INVALID_ARG for a null workspace; DCP_ERR_CUDA if the launch fails.
+ */
+DCP_API dcp_status dcp_check_wait_timeout(void *workspace, void *stream);
+
+/*
  * LSE merge of D partials.  [P1 "A2 方法细节", merge equation;
  * P3 §2.3 equivalent local-max/local-sum form]
  *   O[r] = sum_i w_i O_i[r] / sum_i w_i,  w_i = exp(LSE_i[r] - max_j LSE_j[r]),

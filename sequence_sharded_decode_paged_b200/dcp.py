@@ -30,7 +30,7 @@ EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_b
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
             "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_noalloc_read_device_error",
             "dcp_grow_block_table", "dcp_append_kv", "dcp_host_step_staging_bytes", "dcp_decode_step_host",
-            "dcp_owner_chunk_floats", "dcp_decode_partial_owner_major"]
+            "dcp_owner_chunk_floats", "dcp_decode_partial_owner_major", "dcp_check_wait_timeout"]
 
 
 class DcpError(RuntimeError):
@@ -68,6 +68,7 @@ def _load() -> C.CDLL:
         "dcp_decode_partial_all": (C.c_int, [p, p, p, p, p, p, i32, p, p, p, sz, p]),
         "dcp_lse_merge": (C.c_int, [p, p, i32, i32, i32, p, p, p]),
         "dcp_read_device_error": (C.c_int, [p, p, p]),
+        "dcp_check_wait_timeout": (C.c_int, [p, p]),
         "dcp_validate_config": (C.c_int, [i32, i32, i32, i32]),
         "dcp_decode_partial_all_noalloc": (C.c_int, [p, p, p, p, p, p, i32, p, p, p]),
         "dcp_noalloc_read_device_error": (C.c_int, [p, p]),
@@ -292,6 +293,12 @@ def dcp_decode_step_host(desc: dcp_attn_desc, D: int, host_q, host_seq_lens, hos
 def dcp_lse_merge(O_parts, LSE_parts, D: int, rows: int, d_v: int, O, LSE_out=None, stream=None) -> None:
     _check("dcp_lse_merge", _lib.dcp_lse_merge(
         _ptr_array(O_parts), _ptr_array(LSE_parts), D, rows, d_v, _addr(O), _addr(LSE_out), _stream(stream)))
+
+
+def dcp_check_wait_timeout(workspace, stream=None) -> None:
+    """Launch the bounded-wait diagnostic: sets the timeout bit of the workspace status word after
+    the wait limit (asynchronous; read it back with dcp_read_device_error)."""
+    _check("dcp_check_wait_timeout", _lib.dcp_check_wait_timeout(_addr(workspace), _stream(stream)))
 
 
 def dcp_read_device_error(workspace, stream=None) -> int:

@@ -105,6 +105,8 @@ def test_device_calls_reject_bad_arguments_before_launch():
     assert st == dcp.DCP_ERR_INVALID_ARG
     lib.dcp_lse_merge.restype = ctypes.c_int
     assert lib.dcp_lse_merge(null, null, 2, 4, 64, null, null, null) == dcp.DCP_ERR_INVALID_ARG
+    lib.dcp_check_wait_timeout.restype = ctypes.c_int
+    assert lib.dcp_check_wait_timeout(null, null) == dcp.DCP_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("D", [1, 2, 3, 4, 8])

@@ -86,6 +86,9 @@ def _load():
             lib.oracle_place_request_u8.restype = None
             lib.oracle_place_request_u8.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
                                                     C.c_int, p, C.c_int64, p, p]
+            lib.oracle_place_request_mla_u8.restype = None
+            lib.oracle_place_request_mla_u8.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                                        C.c_int, p, C.c_int64, p, p]
             lib.oracle_merge.restype = None
             lib.oracle_merge.argtypes = [p, p, C.c_int, C.c_int64, C.c_int, p, p]
             lib.oracle_merge_ml.restype = None
@@ -277,6 +280,33 @@ def place_u8(Hkv: int, d: int, block_size: int, D: int, tables: np.ndarray, code
         c = np.ascontiguousarray(c, dtype=np.uint8)
         _load().oracle_place_request_u8(Hkv, d, block_size, D, rule, B, b, mlb, _ptr(t), c.shape[0], _ptr(c),
                                         C.cast(arr, C.c_void_p))
+    return pools
+
+
+def quantize_kv_mla(src: np.ndarray, scale: float) -> np.ndarray:
+    """MLA latent rows [n][576] (bf16 bits) -> E4M3 codes.  The latent is one tensor read as both key
+    (all 576 entries) and value (the first 512), so one per-tensor scale covers the whole row."""
+    return quantize_e4m3(src, scale)
+
+
+def dequantize_kv_mla(codes: np.ndarray, scale: float) -> np.ndarray:
+    """The float64 values an FP8 MLA latent cache stands for: [n][576]."""
+    return dequantize_e4m3(codes, scale)
+
+
+def place_mla_u8(block_size: int, D: int, tables: np.ndarray, codes: List[np.ndarray], num_pages: np.ndarray,
+                 fill: int = 0xFF, rule: int = INTERLEAVED, d: int = 576) -> List[np.ndarray]:
+    """Reference placement of quantised MLA latent rows: D byte pools of [bs][d] pages, unused bytes ``fill``."""
+    B = len(codes)
+    mlb = tables.shape[2]
+    page = block_size * d
+    pools = [np.full(int(num_pages[s]) * page, fill, dtype=np.uint8) for s in range(D)]
+    arr = (C.c_void_p * D)(*[p.ctypes.data for p in pools])
+    t = np.ascontiguousarray(tables, dtype=np.int32)
+    for b, c in enumerate(codes):
+        c = np.ascontiguousarray(c, dtype=np.uint8)
+        _load().oracle_place_request_mla_u8(d, block_size, D, rule, B, b, mlb, _ptr(t), c.shape[0], _ptr(c),
+                                            C.cast(arr, C.c_void_p))
     return pools
 
 

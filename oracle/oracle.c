@@ -400,6 +400,23 @@ void oracle_place_request_u8(int Hkv, int d, int block_size, int D, int rule, in
     }
 }
 
+/*
+ * Placement of one request's quantised MLA latent rows (codes [n_tok][576],
+ * one byte per element, the whole row quantised with the latent's one scale)
+ * into byte pools whose pages are [bs][576]: the same token walk as
+ * oracle_place_request_rule, one byte per element.
+ */
+void oracle_place_request_mla_u8(int d, int block_size, int D, int rule, int B, int b, int max_local_blocks,
+                                 const int32_t *tables, int64_t n_tok, const uint8_t *src, uint8_t **pools) {
+    for (int64_t t = 0; t < n_tok; ++t) {
+        int s = oracle_token_shard_rule(t, block_size, D, rule, n_tok);
+        int64_t j = oracle_token_local_block_rule(t, block_size, D, rule, n_tok);
+        int64_t page = tables[((int64_t)s * B + b) * max_local_blocks + j];
+        int64_t slot = t % block_size;
+        for (int k = 0; k < d; ++k) pools[s][(page * block_size + slot) * d + k] = src[t * d + k];
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Merge of partial results                                            */
 /* ------------------------------------------------------------------ */

@@ -547,6 +547,79 @@ def test_fp8_placement_roundtrip():
     assert sum(int((p != 0x7F).sum()) for p in pools) <= used
 
 
+# FP8 MLA latent cache: one scale for the latent row (key = all 576 entries, value = the first 512)
+@pytest.mark.parametrize("rule", [oracle.INTERLEAVED, oracle.CONTIGUOUS])
+def test_fp8_mla_placement_roundtrip(rule):
+    w = synth.custom(MLA, [130, 1, 64, 65], 4, 1, 576, 512, 64, seed=12)
+    D = 3
+    tables, _, pages = oracle.block_tables(w.seq_lens, 64, D, perm_seed=7, rule=rule)
+    codes = [oracle.quantize_kv_mla(w.kv_source(b), 0.75) for b in range(w.batch)]
+    pools = oracle.place_mla_u8(64, D, tables, codes, pages, fill=0x7F, rule=rule)
+    for b, n in enumerate(w.seq_lens):
+        for t in range(n):
+            s = oracle.token_shard_rule(t, 64, D, rule, n)
+            j = oracle.token_local_block_rule(t, 64, D, rule, n)
+            off = (int(tables[s, b, j]) * 64 + t % 64) * 576
+            np.testing.assert_array_equal(pools[s][off:off + 576], codes[b][t])
+    used = sum(int(n) for n in w.seq_lens) * 576
+    assert sum(int((p != 0x7F).sum()) for p in pools) <= used
+
+
+def _exact_latent_codes(n, seed):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(n, 576)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x01  # no NaN codes
+    codes[codes == 0x80] = 0x00           # no negative zero
+    return codes
+
+
+def test_fp8_mla_exact_codes_give_the_bf16_attention():
+    # latent values that are E4M3 values times a power-of-two scale are exact in bf16 and quantise back to
+    # the same codes, so attention over the FP8 cache's values equals bf16 attention over them, bit for bit
+    scale = 2.0 ** -3
+    codes = _exact_latent_codes(150, 3)
+    vals = oracle.e4m3_decode(codes) * scale
+    bits = synth.f32_to_bf16_bits(vals.astype(np.float32))
+    np.testing.assert_array_equal(synth.bf16_bits_to_f64(bits), vals)
+    np.testing.assert_array_equal(oracle.quantize_kv_mla(bits, scale), codes)
+    np.testing.assert_array_equal(oracle.dequantize_kv_mla(codes, scale), vals)
+    w = synth.custom(MLA, [150], 4, 1, 576, 512, 64, seed=8)
+    q = w.query(0)
+    for D, s in [(1, -1), (3, 2)]:
+        a = oracle.attend(MLA, 4, 1, 576, 512, q, bits, w.softmax_scale, 64, D, s)
+        b = oracle.attend_values(MLA, 4, 1, 576, 512, q, oracle.dequantize_kv_mla(codes, scale), w.softmax_scale,
+                                 64, D, s)
+        np.testing.assert_array_equal(a[0], b[0])
+        np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_fp8_mla_attention_matches_torch_sdpa():
+    # scores over all 576 dequantised entries, values = the first 512 (a library routine, float64)
+    w = synth.custom(MLA, [200], 4, 1, 576, 512, 64, seed=31)
+    scale = 0.37
+    vals = oracle.dequantize_kv_mla(oracle.quantize_kv_mla(w.kv_source(0), scale), scale)
+    O, LSE = oracle.attend_values(MLA, 4, 1, 576, 512, w.query(0), vals, w.softmax_scale)
+    qd = torch.from_numpy(synth.bf16_bits_to_f64(w.query(0)))
+    K = torch.from_numpy(vals)
+    Ot = torch.nn.functional.scaled_dot_product_attention(qd[:, None], K[None].expand(4, -1, -1),
+                                                          K[None, :, :512].expand(4, -1, -1),
+                                                          scale=w.softmax_scale)[:, 0]
+    Lt = torch.logsumexp(qd @ K.T * w.softmax_scale, dim=1)
+    np.testing.assert_allclose(O, Ot.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE, Lt.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("rule", [oracle.INTERLEAVED, oracle.CONTIGUOUS])
+@pytest.mark.parametrize("D", [2, 3, 8])
+def test_fp8_mla_sharded_merge_equals_direct(D, rule):
+    w = synth.custom(MLA, [333], 4, 1, 576, 512, 64, seed=D + 40)
+    vals = oracle.dequantize_kv_mla(oracle.quantize_kv_mla(w.kv_source(0), 0.5), 0.5)
+    O, LSE = oracle.attend_values(MLA, 4, 1, 576, 512, w.query(0), vals, w.softmax_scale)
+    Om, Lm, _, _ = oracle.sharded_values(MLA, 4, 1, 576, 512, w.query(0), vals, w.softmax_scale, 64, D, rule)
+    np.testing.assert_allclose(Om, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lm, LSE, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # contiguous-chunk shard rule ([P1] A2 illustration: "GPU0 holds 0-50K, GPU1 50K-100K, ...")
 # ---------------------------------------------------------------------------

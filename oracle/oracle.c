@@ -368,16 +368,29 @@ uint8_t oracle_e4m3_encode(double x) {
  * 1 / scale.  The value a code stands for is scale * e4m3_value(code).
  */
 void oracle_quantize_e4m3(const uint16_t *src, int64_t n, float inv_scale, uint8_t *out) {
+    /* The code is a function of the 16-bit input alone: encode each of the 65,536 bf16 patterns
+       once (only when the input is long enough to make that cheaper) and look the rest up. */
+    uint8_t *table = n > 65536 ? (uint8_t *)malloc(65536) : NULL;
+    int use_table = table != NULL;
+    if (use_table)
+        for (int b = 0; b < 65536; ++b) table[b] = oracle_e4m3_encode((double)((float)bf16_to_double((uint16_t)b) * inv_scale));
     for (int64_t i = 0; i < n; ++i) {
+        if (use_table) {
+            out[i] = table[src[i]];
+            continue;
+        }
         float x = (float)bf16_to_double(src[i]);
         float p = x * inv_scale;
         out[i] = oracle_e4m3_encode((double)p);
     }
+    free(table);
 }
 
 /* scale * value(code) for n codes (exact in double). */
 void oracle_dequantize_e4m3(const uint8_t *codes, int64_t n, double scale, double *out) {
-    for (int64_t i = 0; i < n; ++i) out[i] = scale * oracle_e4m3_decode(codes[i]);
+    double value[256];
+    for (int c = 0; c < 256; ++c) value[c] = scale * oracle_e4m3_decode((uint8_t)c);
+    for (int64_t i = 0; i < n; ++i) out[i] = value[codes[i]];
 }
 
 /*

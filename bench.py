@@ -64,7 +64,7 @@ def parse(argv=None):
     ap.add_argument("--q-len", type=int, default=1,
                     help="query tokens per request (multi-token decode, causal within the draft; 1..4)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
-                    help="cache element type (fp8: E4M3 codes, per-tensor scales 2^-7; GQA head_dim 128)")
+                    help="cache element type (fp8: E4M3 codes, per-tensor scales 2^-7; GQA and MLA)")
     ap.add_argument("--batch-limit", type=int, default=None,
                     help="keep only the first N requests (small cases for profiling)")
     return ap.parse_args(argv)

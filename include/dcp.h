@@ -46,7 +46,8 @@
  *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.
  *       Multi-token decode: 1 <= q_len <= 4 query tokens per request
  *       (GQA and MLA).
- *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA with head_dim 128 only.
+ *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA with head_dim 128, and MLA
+ *       (whose latent takes one scale: k_scale == v_scale).
  *       Shard rules: interleaved (default) or contiguous chunks (dcp_shard_rule).
  */
 #ifndef DCP_H
@@ -86,7 +87,10 @@ typedef enum dcp_layout {
  *   DCP_KV_FP8_E4M3  one byte per value: an E4M3 code (the OCP FP8 E4M3 "fn"
  *                    format: bias 7, no infinities, largest finite 448) and a
  *                    per-tensor scale, value = scale * e4m3(code); K uses
- *                    k_scale, V uses v_scale.  The cache writes quantise bf16
+ *                    k_scale, V uses v_scale.  The MLA latent is one tensor
+ *                    (key = all 576 entries, value = the first 512), so it has
+ *                    one scale: k_scale, which v_scale must equal
+ *                    (DCP_ERR_INVALID_ARG otherwise).  The cache writes quantise bf16
  *                    rows as code = e4m3_rn_satfinite(float32(x) * inv), inv =
  *                    float32(1 / scale): the product rounded to float32, then to
  *                    the nearest code (ties to even), magnitudes past 448
@@ -225,7 +229,7 @@ DCP_API size_t dcp_kv_page_bytes(const dcp_attn_desc *desc);
  *   kv_pools    host array of D device pointers; pool s holds pool_pages[s] pages:
  *               GQA page [2 (K,V)][Hkv][block_size][head_dim] of the pool's
  *               kv_dtype (bf16, or FP8 codes quantised on the way in);
- *               MLA page [block_size][576] bf16.
+ *               MLA page [block_size][576] of the pool's kv_dtype.
  *   pool_pages  host int32[D].
  *   device_error optional device int32 (may be NULL): set to 1 if a table entry
  *               lies outside its pool; such rows are skipped, never written.

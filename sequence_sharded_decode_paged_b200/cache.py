@@ -100,7 +100,7 @@ class ShardedPagedCache:
         """KV bytes the method reads per step (tokens x bytes per token; padding excluded)."""
         d = self.desc
         eb = 1 if d.kv_dtype == dcp.DCP_KV_FP8_E4M3 else 2
-        per = 2 * d.num_kv_heads * d.head_dim_qk * eb if d.layout == dcp.DCP_LAYOUT_GQA else d.head_dim_qk * 2
+        per = 2 * d.num_kv_heads * d.head_dim_qk * eb if d.layout == dcp.DCP_LAYOUT_GQA else d.head_dim_qk * eb
         return int(sum(self.seq_lens)) * per
 
 

@@ -94,7 +94,11 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
     return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.q_len > kMaxQLen) return false;
-  if (d.kv_dtype == DCP_KV_FP8_E4M3 && (d.layout != DCP_LAYOUT_GQA || d.head_dim_qk != 128)) return false;
+  // MLA's latent is one tensor (key = all 576 entries, value = the first 512): one scale for both
+  *why = DCP_ERR_INVALID_ARG;
+  if (d.kv_dtype == DCP_KV_FP8_E4M3 && d.layout == DCP_LAYOUT_MLA && d.k_scale != d.v_scale) return false;
+  *why = DCP_ERR_UNSUPPORTED;
+  if (d.kv_dtype == DCP_KV_FP8_E4M3 && d.layout == DCP_LAYOUT_GQA && d.head_dim_qk != 128) return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.layout == DCP_LAYOUT_GQA) {
     if (d.head_dim_qk != d.head_dim_v || (d.head_dim_qk != 64 && d.head_dim_qk != 128)) return false;
@@ -247,7 +251,7 @@ size_t dcp_kv_page_bytes(const dcp_attn_desc* desc) {
   dcp_status why;
   if (!desc_supported(d, 1, &why)) return 0;
   if (d.layout == DCP_LAYOUT_GQA) return (size_t)2 * d.num_kv_heads * d.block_size * d.head_dim_qk * kv_elem_bytes(d);
-  return (size_t)d.block_size * d.head_dim_qk * 2;
+  return (size_t)d.block_size * d.head_dim_qk * kv_elem_bytes(d);
 }
 
 dcp_status dcp_place_kv(const dcp_attn_desc* desc, int32_t D, const void* kv_src, const int64_t* cu_seqlens,

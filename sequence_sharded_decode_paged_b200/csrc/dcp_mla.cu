@@ -54,6 +54,19 @@
 //    ranges within one wave), so each latent page is fetched from HBM about
 //    once and the other reads hit L2.  Token j masks the scores of tokens at
 //    or past seq_len - (q_len - 1 - j).
+//  * FP8 latent cache (KV8): pages hold E4M3 codes, 576 bytes per token, one
+//    per-tensor scale.  The codes land inside the 16-bit pair stage itself and
+//    are widened there, so the stage, the products and the softmax keep their
+//    shapes: a value group's codes (dims 128g .. 128g+127, one 128-byte row per
+//    token) land in the group's second box, the rope codes (dims 512-575, a
+//    128-byte box half past the row end, which TMA fills with zeros and does
+//    not read) in the rope box.  Two more warps (10-11, one per page of the
+//    pair) widen each row to f16 in place -- every E4M3 value is an f16, so
+//    exactly -- each thread rewriting only the rows it read, and convert the
+//    query tile from bf16 to f16 (exact within f16's normal range) when it
+//    lands.  Products run as kind::f16 with f16 operands; P^T is written as
+//    f16; the scale multiplies the scores (folded into the exponent's FMA) and
+//    the normalisation of O.
 #include <float.h>
 #include <stddef.h>
 
@@ -99,9 +112,15 @@ constexpr float kRescaleThreshold = 8.0f;             // log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kSoftmaxWarps = 8;
+// FP8 cache: warps 10-11 widen the codes (warp 10: page a of a pair, warp 11: page b).
+constexpr int kConvWarp0 = 10;
+constexpr int kConvThreads = 64;
+template <bool KV8>
+__host__ __device__ constexpr int mla_threads() { return KV8 ? kMlaThreads + kConvThreads : kMlaThreads; }
 
 struct MlaMisc {
   uint64_t q_full, q_empty, kv_full[kGroups], kv_empty[kGroups], s_full[2], s_empty[2], mma_done, pv_done;
+  uint64_t cv_full[kGroups], qc_full;  // FP8: a group's codes / the query tile converted to f16
   uint32_t tmem_base;
   int bcast;
   alignas(16) float mref[kMlaHeads];  // integral reference maxima (log2 units); read as float4
@@ -139,6 +158,7 @@ struct MlaParams {
   int* counters;
   float* slots;
   float scale_log2;
+  float v_scale;  // multiplies the normalised O (the FP8 latent's scale; 1 for bf16)
   int n_si, B, D, mlb, slot_floats, q_len;
   // Output layout: query heads are owned in consecutive slices of Hk heads, and owner k's
   // O rows (and LSE rows) start k * own_stride floats after owner 0's.  The standard layout
@@ -199,14 +219,57 @@ __device__ __forceinline__ void issue_pv(uint32_t t_o, uint32_t v_lo, uint32_t v
   umma_commit(&misc->kv_empty[4]);  // the rope boxes (P^T) are free, and the pair's O^T is complete
 }
 
-// This thread's P^T row: its token's weights for heads 32*hf .. +31 as bf16, four 16-byte
-// chunks of the 128-byte-swizzled row.
+// This thread's P^T row: its token's weights for heads 32*hf .. +31 as bf16 (f16 for the FP8
+// cache, whose products take f16 operands), four 16-byte chunks of the 128-byte-swizzled row.
+template <bool F16>
 __device__ __forceinline__ void write_pt(uint8_t* prow, const float (&w)[32], int hf, int tok) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
-    const uint4 w4 = make_uint4(pack_bf16x2(w[8 * c + 0], w[8 * c + 1]), pack_bf16x2(w[8 * c + 2], w[8 * c + 3]),
-                                pack_bf16x2(w[8 * c + 4], w[8 * c + 5]), pack_bf16x2(w[8 * c + 6], w[8 * c + 7]));
+    uint4 w4;
+    if constexpr (F16)
+      w4 = make_uint4(pack_f16x2(w[8 * c + 0], w[8 * c + 1]), pack_f16x2(w[8 * c + 2], w[8 * c + 3]),
+                      pack_f16x2(w[8 * c + 4], w[8 * c + 5]), pack_f16x2(w[8 * c + 6], w[8 * c + 7]));
+    else
+      w4 = make_uint4(pack_bf16x2(w[8 * c + 0], w[8 * c + 1]), pack_bf16x2(w[8 * c + 2], w[8 * c + 3]),
+                      pack_bf16x2(w[8 * c + 4], w[8 * c + 5]), pack_bf16x2(w[8 * c + 6], w[8 * c + 7]));
     *reinterpret_cast<uint4*>(prow + ((((uint32_t)(4 * hf + c)) ^ (uint32_t)(tok & 7)) << 4)) = w4;
+  }
+}
+
+// FP8 cache: widen page slot x of load group g in place.  The group's codes sit in its landing
+// box (value group g: box 2g+1, rope group: box 8), one 128-byte row per token (128-byte
+// swizzled, as TMA wrote them): codes of dims 16k .. 16k+15 of the group in chunk k.  Chunks
+// 0-3 become the f16 row of the group's first box (value: box 2g; rope: box 8 itself), chunks
+// 4-7 the f16 row of box 2g+1 (value groups only).  A thread handles rows lane and lane + 32
+// and reads a whole row before writing it: the only code bytes its stores overwrite are those
+// of its own rows, so no other thread's input is touched.
+__device__ __forceinline__ void widen_group(uint8_t* kv, int g, int x, int lane) {
+  uint8_t* land = kv + (g < 4 ? 2 * g + 1 : 8) * kPairBox + x * kBlockBytes;
+  uint8_t* first = kv + (g < 4 ? 2 * g : 8) * kPairBox + x * kBlockBytes;
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const uint32_t r = (uint32_t)(lane + 32 * rr), sw = r & 7u;
+    uint4 c[8];
+    if (g < 4) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) c[k] = *reinterpret_cast<const uint4*>(land + r * 128 + (((uint32_t)k ^ sw) << 4));
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) c[k] = *reinterpret_cast<const uint4*>(land + r * 128 + (((uint32_t)k ^ sw) << 4));
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (g == 4 && k >= 4) break;
+      uint4 lo, hi;  // f16 of codes 16k .. 16k+7, 16k+8 .. 16k+15
+      e4m3x4_to_f16x2x2(c[k].x, lo.x, lo.y);
+      e4m3x4_to_f16x2x2(c[k].y, lo.z, lo.w);
+      e4m3x4_to_f16x2x2(c[k].z, hi.x, hi.y);
+      e4m3x4_to_f16x2x2(c[k].w, hi.z, hi.w);
+      uint8_t* row = (k < 4 ? first : land) + r * 128;
+      const uint32_t m = (uint32_t)(2 * (k & 3));
+      *reinterpret_cast<uint4*>(row + ((m ^ sw) << 4)) = lo;
+      *reinterpret_cast<uint4*>(row + (((m + 1) ^ sw) << 4)) = hi;
+    }
   }
 }
 
@@ -273,8 +336,10 @@ __device__ __forceinline__ float warp_transpose_reduce(float (&v)[32], int lane)
 }  // namespace
 
 // RULE: the shard rule (0 interleaved, 1 contiguous chunks), fixed at compile time.
-template <int RULE>
-__global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid_constant__ MlaParams p) {
+// KV8: the pools hold FP8 E4M3 codes (warps 10-11 widen them in shared memory).
+template <int RULE, bool KV8>
+__global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const __grid_constant__ MlaParams p) {
+  constexpr int kThreads = mla_threads<KV8>();
   extern __shared__ __align__(1024) uint8_t smem[];
   MlaMisc* misc = reinterpret_cast<MlaMisc*>(smem + kOffMisc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -299,12 +364,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     }
     mbar_init(&misc->mma_done, 1);
     mbar_init(&misc->pv_done, 1);
+    if (KV8) {
+      for (int g = 0; g < kGroups; ++g) mbar_init(&misc->cv_full[g], kConvThreads);
+      mbar_init(&misc->qc_full, kConvThreads);
+    }
     fence_barrier_init();
   }
   // The products read every row of the pair stage, also rows no page fills (a pair's
   // missing second page, a skipped page): their scores are masked and their weights are
   // zero, so they only need to be finite -- zero the stage once.
-  for (uint32_t i = tid; i < 9 * kPairBox / 16; i += kMlaThreads)
+  for (uint32_t i = tid; i < 9 * kPairBox / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + kOffKV)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   if (warp == 0 && lane == 0) {
@@ -368,17 +437,24 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
             wait_or_die(&misc->kv_empty[g], par ^ 1u, dead, p.status);
             if (dead) break;
             const int nb = group_boxes(g), cb0 = group_box0(g);
-            const uint32_t bytes = nb * kBlockBytes * ((oka ? 1u : 0u) + (okb ? 1u : 0u));
+            // FP8: one 128-byte box of codes per page (the rope box reads 64 bytes, the rest is fill)
+            const uint32_t bytes = (KV8 ? kBlockBytes : nb * kBlockBytes) * ((oka ? 1u : 0u) + (okb ? 1u : 0u));
             last[g] = pc;
             if (bytes == 0) {
               mbar_arrive(&misc->kv_full[g]);
               continue;
             }
             mbar_arrive_expect_tx(&misc->kv_full[g], bytes);
-            for (int cb = cb0; cb < cb0 + nb; ++cb) {
-              uint8_t* dst = smem + kOffKV + cb * kPairBox;
-              if (oka) tma_load_2d(dst, &p.kvmap[si], cb * 64, pa * kMlaBs, &misc->kv_full[g]);
-              if (okb) tma_load_2d(dst + kBlockBytes, &p.kvmap[si], cb * 64, pb * kMlaBs, &misc->kv_full[g]);
+            if (KV8) {
+              uint8_t* dst = smem + kOffKV + (g < 4 ? 2 * g + 1 : 8) * kPairBox;  // the group's landing box
+              if (oka) tma_load_2d(dst, &p.kvmap[si], 128 * g, pa * kMlaBs, &misc->kv_full[g]);
+              if (okb) tma_load_2d(dst + kBlockBytes, &p.kvmap[si], 128 * g, pb * kMlaBs, &misc->kv_full[g]);
+            } else {
+              for (int cb = cb0; cb < cb0 + nb; ++cb) {
+                uint8_t* dst = smem + kOffKV + cb * kPairBox;
+                if (oka) tma_load_2d(dst, &p.kvmap[si], cb * 64, pa * kMlaBs, &misc->kv_full[g]);
+                if (okb) tma_load_2d(dst + kBlockBytes, &p.kvmap[si], cb * 64, pb * kMlaBs, &misc->kv_full[g]);
+              }
             }
           }
           ++pc;
@@ -398,7 +474,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
   } else if (warp == 1) {
     // ------------------------------------------------------------ S^T issuer
     {  // the whole warp walks the pairs and waits; an elected lane issues
-      const uint32_t idS = idesc_bf16_f32(128, 64, false, false);
+      const uint32_t idS = KV8 ? idesc_f16_f32(128, 64, false, false) : idesc_bf16_f32(128, 64, false, false);
       // K rows (A) and the query (B): K-major, one 8-row group per 1,024 bytes
       const uint64_t k_desc = sw128_desc(smem_u32(smem + kOffKV), 16, 1024);
       const uint64_t q_desc = sw128_desc(smem_u32(smem + kOffQ), 16, 1024);
@@ -416,7 +492,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
         const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
         pre += n;
         if (n == 0) continue;
-        wait_or_die_warp(&misc->q_full, q_ph, dead, p.status);
+        wait_or_die_warp(KV8 ? &misc->qc_full : &misc->q_full, q_ph, dead, p.status);
         q_ph ^= 1u;
         for (int j = a; j < e && !dead; j += 2) {
           // Per pair: S^T = K Q^T group by group as the groups land.  (The softmax group
@@ -426,7 +502,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
           const uint32_t dS = tbase + kColS + sb * 64;
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
-            wait_or_die_warp(&misc->kv_full[g], par, dead, p.status);
+            wait_or_die_warp(KV8 ? &misc->cv_full[g] : &misc->kv_full[g], par, dead, p.status);
             if (dead) break;
             tc_fence_after();
             if (elect_one()) {
@@ -453,7 +529,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       bool d2 = false;
       wait_or_die(&misc->mma_done, 0, d2, p.status);
     }
-  } else {
+  } else if (warp < kConvWarp0) {
     // ------------------------------------------------------------ softmax + epilogue (warps 2-9)
     // Warp w reads TMEM sub-partition q4 = w % 4: lanes 32*q4 .. +31 hold the pair's tokens
     // 32*q4 .. +31 (page a below 64, page b from 64); half hf = (w - 2) / 4 takes the heads
@@ -464,7 +540,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
     const int tok = 32 * q4 + lane;                // token of the pair this thread holds
     const bool waiter = warp == 2;                 // the warp that waits on the group's mbarriers
-    const uint32_t idO = idesc_bf16_f32(128, 64, true, true);
+    const uint32_t idO = KV8 ? idesc_f16_f32(128, 64, true, true) : idesc_bf16_f32(128, 64, true, true);
     const uint64_t v_desc = sw128_desc(smem_u32(smem + kOffKV), kPairBox, 1024);
     const uint64_t p_desc = sw128_desc(smem_u32(smem + kOffPT), kPairBox, 1024);
     const uint32_t v_lo = (uint32_t)v_desc, v_hi = (uint32_t)(v_desc >> 32);
@@ -572,7 +648,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               s[i] = ex2_approx(t);
             }
           }
-          if (!dead) write_pt(smem + kOffPT + tok * 128, s, hf, tok);
+          if (!dead) write_pt<KV8>(smem + kOffPT + tok * 128, s, hf, tok);
         }
         fence_proxy_async_smem();  // P^T rows and zeroed value rows -> the async proxy
         tc_fence_before();
@@ -619,7 +695,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
               s[i] = ex2_approx(see ? fmaf(s[i], p.scale_log2, -mm[k]) : -INFINITY);
             }
           }
-          if (!dead) write_pt(smem + kOffPT + tok * 128, s, hf, tok);
+          if (!dead) write_pt<KV8>(smem + kOffPT + tok * 128, s, hf, tok);
           if (resc) {
             // O^T holds the earlier pairs: observe the previous pair's PV completion before
             // rescaling it.  (That PV has finished by now -- it released the groups this pair's
@@ -676,7 +752,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
       if (ts < kMlaHeads) {
         const float lt = (misc->part[0][ts] + misc->part[1][ts]) + (misc->part[2][ts] + misc->part[3][ts]);
         const float mh = misc->mref[ts];
-        misc->inv_l[ts] = lt > 0.f ? 1.f / lt : 0.f;
+        misc->inv_l[ts] = lt > 0.f ? (KV8 ? p.v_scale / lt : 1.f / lt) : 0.f;
         misc->lse2[ts] = lt > 0.f ? mh + __log2f(lt) : -INFINITY;
         // row offsets once per piece, so that the stores below need no owner arithmetic
         misc->rowoff[ts] = complete ? (size_t)(o_row(ts) - p.O[si]) : (size_t)ts * kMlaDv;
@@ -834,6 +910,57 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_decode_kernel(const __grid
     }
   }
 
+  if (KV8 && warp >= kConvWarp0) {
+    // ------------------------------------------------------------ FP8 -> f16 (warps 10-11)
+    // The same walk as the producer: per segment piece the query tile, per pair the five load
+    // groups.  Warp 10 widens page a of every pair, warp 11 page b; a page that was not loaded
+    // (a pair's missing second page, an invalid page id) keeps what its rows held, as in the
+    // bf16 stage.  Every converter thread arrives on the group's barrier after its own stores
+    // and a proxy fence, so the products see every row.
+    const int x = warp - kConvWarp0, ct = tid - kMlaThreads;
+    uint32_t q_ph = 0;
+    long pc = 0;
+    bool dead = false;
+    int pre = plan.pre0;
+    for (int sid = plan.sid0; sid < S && !dead; ++sid) {
+      const int si = sid / B, b = sid - si * B, shard = p.shard_of_si[si];
+      const int n = local_pages_r<RULE>(p.seq_lens[b], kMlaBs, D, shard);
+      if (n > 0) pre += kMlaSegCost;  // the segment's fixed-work units precede its pages
+      if (seg_first_cta(pre, n, T, P) > cta) break;
+      const int a = max(pre, lo) - pre, e = min(pre + n, hi) - pre;
+      pre += n;
+      if (n == 0) continue;
+      wait_or_die_warp(&misc->q_full, q_ph, dead, p.status);
+      q_ph ^= 1u;
+      if (dead) break;
+      for (int i = ct; i < (int)(kTileBytes / 16); i += kConvThreads) {  // bf16 -> f16, in place
+        uint4* c = reinterpret_cast<uint4*>(smem + kOffQ) + i;
+        uint4 v = *c;
+        v.x = bf16x2_to_f16x2(v.x);
+        v.y = bf16x2_to_f16x2(v.y);
+        v.z = bf16x2_to_f16x2(v.z);
+        v.w = bf16x2_to_f16x2(v.w);
+        *c = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&misc->qc_full);
+      for (int j = a; j < e && !dead; j += 2) {
+        int pg = -1;
+        const bool ok = x == 0 ? page_ok(p, si, b, j, &pg) : (j + 1 < e && page_ok(p, si, b, j + 1, &pg));
+        const uint32_t par = (uint32_t)(pc & 1);
+#pragma unroll 1
+        for (int g = 0; g < kGroups; ++g) {
+          wait_or_die_warp(&misc->kv_full[g], par, dead, p.status);
+          if (dead) break;
+          if (ok) widen_group(smem + kOffKV, g, x, lane);
+          fence_proxy_async_smem();
+          mbar_arrive(&misc->cv_full[g]);
+        }
+        ++pc;
+      }
+    }
+  }
+
   // ---------------------------------------------------------------- release TMEM
   tc_fence_before();
   __syncthreads();
@@ -862,7 +989,11 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   p.D = D;
   p.mlb = d.max_local_blocks;
   p.slot_floats = L.slot_floats;
-  p.scale_log2 = d.softmax_scale * 1.4426950408889634f;
+  const bool kv8 = d.kv_dtype == DCP_KV_FP8_E4M3;
+  // FP8: the latent's scale multiplies every score (folded into the exponent) and the normalised O
+  p.scale_log2 = kv8 ? (float)((double)d.softmax_scale * (double)d.k_scale * 1.4426950408889634)
+                     : d.softmax_scale * 1.4426950408889634f;
+  p.v_scale = kv8 ? d.v_scale : 1.f;
   p.q_len = d.q_len;
   p.Hk = set.owner_heads > 0 ? set.owner_heads : kMlaHeads;
   p.own_stride = set.owner_stride;
@@ -883,14 +1014,18 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
     if (set.pool_pages[si] > 0) {
       const uint64_t rows = (uint64_t)set.pool_pages[si] * kMlaBs;
       if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32
-      if (encode_tiled_2d(&p.kvmap[si], set.pool[si], kMlaDqk, rows, kMlaDqk * 2, 64, 64) != CUDA_SUCCESS)
-        return DCP_ERR_CUDA;
+      // FP8: 128-byte boxes of codes (the rope group's box starts at byte 512 and runs past the
+      // 576-byte row: TMA fills the missing part and does not read it)
+      const CUresult r = kv8 ? encode_tiled_2d(&p.kvmap[si], set.pool[si], kMlaDqk, rows, kMlaDqk, 128, 64, 1)
+                             : encode_tiled_2d(&p.kvmap[si], set.pool[si], kMlaDqk, rows, kMlaDqk * 2, 64, 64);
+      if (r != CUDA_SUCCESS) return DCP_ERR_CUDA;
     }
   }
-  auto kern = d.shard_rule == DCP_SHARD_INTERLEAVED ? mla_decode_kernel<0> : mla_decode_kernel<1>;
+  auto kern = d.shard_rule == DCP_SHARD_INTERLEAVED ? (kv8 ? mla_decode_kernel<0, true> : mla_decode_kernel<0, false>)
+                                                    : (kv8 ? mla_decode_kernel<1, true> : mla_decode_kernel<1, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMlaSmem) != cudaSuccess)
     return DCP_ERR_CUDA;
-  kern<<<dim3(L.nctas, d.q_len), kMlaThreads, kMlaSmem, stream>>>(p);
+  kern<<<dim3(L.nctas, d.q_len), kv8 ? mla_threads<true>() : mla_threads<false>(), kMlaSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
 }
 

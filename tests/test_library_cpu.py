@@ -179,9 +179,14 @@ def test_descriptor_layout_matches_header():
     assert dcp.dcp_attn_desc.v_scale.offset == 48
 
 
-def test_fp8_rejected_for_mla_and_head_dim_64():
-    # FP8 pools: GQA with head_dim 128 only; a page is one byte per value
-    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == 0
+def test_fp8_page_bytes_and_rejections():
+    # FP8 pools: GQA with head_dim 128 and MLA; a page is one byte per value.  The MLA latent is one
+    # tensor, so its key and value scales must be the same number.
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1,
+                                               dcp.DCP_KV_FP8_E4M3, 0.5, 0.5)) == 64 * 576
+    unequal = dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 0.5)
+    assert dcp.dcp_kv_page_bytes(unequal) == 0
+    assert dcp.dcp_decode_workspace_bytes(unequal, 2) == 0
     assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == 0
     assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == \
         2 * 2 * 16 * 128
@@ -240,5 +245,9 @@ def test_descriptor_option_matrix(q_len, rule):
         other = dcp.dcp_attn_desc.from_buffer_copy(dsc)
         other.shard_rule = 1 - rule
         assert dcp.dcp_decode_workspace_bytes(other, 4) == ws
-    assert dcp.dcp_kv_page_bytes(desc(1, 1, 64, 1, 576, 64)) == 0  # FP8 MLA
+    # FP8 MLA (one scale for the latent): half a bf16 page, the same workspace
+    m8 = dcp.make_desc(1, 8, 64, 1, 576, 512, 64, 32, 0.1, q_len, 1, 0.5, 0.5, rule)
+    assert dcp.dcp_kv_page_bytes(m8) * 2 == dcp.dcp_kv_page_bytes(mla)
+    assert dcp.dcp_decode_workspace_bytes(m8, 4) == dcp.dcp_decode_workspace_bytes(mla, 4)
+    assert dcp.dcp_kv_page_bytes(desc(1, 1, 64, 1, 576, 64)) == 0  # FP8 MLA with unequal scales
     assert dcp.dcp_kv_page_bytes(desc(0, 1, 16, 2, 64)) == 0      # FP8 head_dim 64

@@ -46,7 +46,7 @@
  *       1 <= D <= 16 shards; batch >= 1; seq_lens[b] >= 0.
  *       Multi-token decode: 1 <= q_len <= 4 query tokens per request
  *       (GQA and MLA).
- *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA with head_dim 128, and MLA
+ *       FP8 cache (kv_dtype DCP_KV_FP8_E4M3): GQA (head_dim 64 or 128) and MLA
  *       (whose latent takes one scale: k_scale == v_scale).
  *       Shard rules: interleaved (default) or contiguous chunks (dcp_shard_rule).
  */

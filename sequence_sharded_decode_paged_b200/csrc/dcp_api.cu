@@ -69,7 +69,8 @@ static EncodeTiledFn encode_fn() {
 }
 
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes) {
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes,
+                         int swizzle_bytes) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return CUDA_ERROR_NOT_SUPPORTED;
   cuuint64_t dims[2] = {inner_elems, rows};
@@ -77,7 +78,8 @@ CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elem
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
@@ -97,8 +99,6 @@ bool desc_supported(const dcp_attn_desc& d, int D, dcp_status* why) {
   // MLA's latent is one tensor (key = all 576 entries, value = the first 512): one scale for both
   *why = DCP_ERR_INVALID_ARG;
   if (d.kv_dtype == DCP_KV_FP8_E4M3 && d.layout == DCP_LAYOUT_MLA && d.k_scale != d.v_scale) return false;
-  *why = DCP_ERR_UNSUPPORTED;
-  if (d.kv_dtype == DCP_KV_FP8_E4M3 && d.layout == DCP_LAYOUT_GQA && d.head_dim_qk != 128) return false;
   *why = DCP_ERR_UNSUPPORTED;
   if (d.layout == DCP_LAYOUT_GQA) {
     if (d.head_dim_qk != d.head_dim_v || (d.head_dim_qk != 64 && d.head_dim_qk != 128)) return false;

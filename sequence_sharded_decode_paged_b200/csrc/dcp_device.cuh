@@ -216,6 +216,19 @@ __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
+// Byte offset of 16-byte chunk `chunk` (0-3) of row `row` inside a 64-byte-swizzled tile of
+// 64-byte rows (TMA CU_TENSOR_MAP_SWIZZLE_64B: the chunk index XOR bits 7-8 of the byte offset,
+// i.e. row / 2 % 4; the tile base must be 512-byte aligned).
+__device__ __forceinline__ uint32_t sw64(uint32_t row, uint32_t chunk) {
+  return row * 64u + ((chunk ^ ((row >> 1) & 3u)) << 4);
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 // ---------------------------------------------------------------- work planning
 // Segments are (shard slot si, request b) pairs, sid = si * B + b, laid out in
 // that order; segment sid holds n(sid) local pages (the blocks g < ceil(len/bs)

@@ -24,15 +24,17 @@
 //    the V fragments, so stale cache contents (even NaN) never leak in.
 //  * Multi-token decode (q_len > 1): row r sees only the tokens before
 //    seq_len - (q_len - 1 - r / G); the rest of its scores are masked.
-//  * FP8 cache (KV8, head_dim 128): pages hold E4M3 codes, a 128-byte row per
-//    token and head, so one swizzled box carries a head's K (or V) block and a
-//    stage is half the size.  Codes convert exactly to f16 and the products
+//  * FP8 cache (KV8, head_dim 128 or 64): pages hold E4M3 codes, a 128-byte
+//    (64-byte) row per token and head, so one swizzled box carries a head's K
+//    (or V) block and a stage is half the size.  Codes convert exactly to f16 and the products
 //    run as f16 mma.  K: each lane reads 4 consecutive codes of a token with
 //    one 32-bit load; the query's dimensions are permuted the same way inside
 //    each 16-wide k-tile (dims 4c..4c+3 play k = 2c, 2c+1, 2c+8, 2c+9).  V:
 //    each lane reads 16 codes (dims 16g..16g+15) of tokens 2c, 2c+1, 2c+8 and
 //    2c+9 with 16-byte loads and pairs them by byte permutes, so n-tile nt,
 //    column n stands for dim 16n + nt; the output store undoes that order.
+//    At head_dim 64 a lane reads 8 codes (dims 8g..8g+7, 8-byte loads) and
+//    column n of n-tile nt stands for dim 8n + nt.
 //    k_scale is folded into the score scale and v_scale into the final
 //    normalisation.  The K products of a chunk run as four independent chains
 //    (two token halves x two k halves) so that their latencies overlap.
@@ -110,15 +112,24 @@ __device__ __forceinline__ float* gqa_l_ptr(const GqaParams& p, int si, OutRow o
 
 template <int HEAD_DIM, bool KV8>
 struct GqaGeom {
-  // 128-byte swizzled boxes per row: 64 bf16 or 128 FP8 codes each
-  static constexpr int kBoxes = KV8 ? HEAD_DIM / 128 : HEAD_DIM / 64;
-  static constexpr int kBoxElems = KV8 ? 128 : 64;
+  // swizzled boxes per row: 64 bf16 (128 bytes) each, or one box of the row's HEAD_DIM FP8 codes
+  static constexpr int kBoxes = KV8 ? 1 : HEAD_DIM / 64;
+  static constexpr int kBoxElems = KV8 ? HEAD_DIM : 64;
+  static constexpr int kRowBytes = KV8 ? HEAD_DIM : 128;  // bytes of one token's row in a box
   static constexpr int kNTiles = HEAD_DIM / 8;  // n-tiles of O
   static constexpr int kKTiles = HEAD_DIM / 16; // k-tiles of Q K^T
   static constexpr int kCombineFloats = kNTiles * 4 + 4;  // per lane per warp
 };
 
-// ---- FP8 building blocks: one 16-token chunk of one KV head (128 dims) ----
+// ---- FP8 building blocks: one 16-token chunk of one KV head (128 or 64 dims) ----
+// Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled box of ROWB-byte rows (the
+// 128-byte swizzle for 128-byte rows, the 64-byte swizzle for 64-byte rows).
+template <int ROWB>
+__device__ __forceinline__ uint32_t kv8_off(uint32_t row, uint32_t chunk) {
+  if constexpr (ROWB == 128) return sw128(row, chunk);
+  else return sw64(row, chunk);
+}
+
 // S (16 q rows x 16 tokens, f32) = Q K^T from E4M3 K rows at `kbase`, rows krow0 ..
 // krow0 + 15 of the swizzled tile.  Lane (g, c) needs codes 4c..4c+3 of k-tile kt of
 // tokens g and 8 + g: one ldmatrix (8 x 16-byte rows per matrix) gives that word for
@@ -127,12 +138,13 @@ struct GqaGeom {
 template <int KT>
 __device__ __forceinline__ void kv8_scores(uint32_t kbase, uint32_t krow0, int lane, const uint32_t (&qa)[KT][4],
                                            float (&s)[2][4]) {
+  constexpr int ROWB = KT * 16;  // one code per dim
   const uint32_t lrow = krow0 + (lane & 7) + (((lane >> 3) & 1) << 3);
   float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
   for (int kt = 0; kt < KT; kt += 2) {
     uint32_t w0, w1, w2, w3;  // (tokens 0-7, kt), (8-15, kt), (0-7, kt+1), (8-15, kt+1)
-    ldsm_x4(kbase + sw128(lrow, (uint32_t)(kt + (lane >> 4))), w0, w1, w2, w3);
+    ldsm_x4(kbase + kv8_off<ROWB>(lrow, (uint32_t)(kt + (lane >> 4))), w0, w1, w2, w3);
     uint32_t k0[2], k1[2], k2[2], k3[2];
     e4m3x4_to_f16x2x2(w0, k0[0], k0[1]);
     e4m3x4_to_f16x2x2(w1, k1[0], k1[1]);
@@ -158,6 +170,33 @@ template <int NT>
 __device__ __forceinline__ void kv8_pv(uint32_t vbase, uint32_t vrow0, int g4, int c4, const uint32_t (&pa)[4],
                                        float (&o)[NT][4], bool tail, uint32_t keep0, uint32_t keep1) {
   const uint32_t vr = vrow0 + 2u * c4;
+  if constexpr (NT == 8) {
+    // head_dim 64: dims 8g..8g+7 (half g % 2 of the row's chunk g / 2); n-tile 4w + k, column n
+    // stands for dim 8n + 4w + k
+    const uint32_t off = (uint32_t)(g4 & 1) * 8u;
+    const uint2 ta = lds64(vbase + kv8_off<64>(vr, (uint32_t)(g4 >> 1)) + off);
+    const uint2 tb = lds64(vbase + kv8_off<64>(vr + 1u, (uint32_t)(g4 >> 1)) + off);
+    const uint2 tc = lds64(vbase + kv8_off<64>(vr + 8u, (uint32_t)(g4 >> 1)) + off);
+    const uint2 td = lds64(vbase + kv8_off<64>(vr + 9u, (uint32_t)(g4 >> 1)) + off);
+    const uint32_t xa[2] = {ta.x, ta.y}, xb[2] = {tb.x, tb.y}, xc[2] = {tc.x, tc.y}, xd[2] = {td.x, td.y};
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      uint32_t b0[4], b1[4];
+      e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x5140), b0[0], b0[1]);
+      e4m3x4_to_f16x2x2(__byte_perm(xa[w], xb[w], 0x7362), b0[2], b0[3]);
+      e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x5140), b1[0], b1[1]);
+      e4m3x4_to_f16x2x2(__byte_perm(xc[w], xd[w], 0x7362), b1[2], b1[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (tail) {
+          b0[k] &= keep0;
+          b1[k] &= keep1;
+        }
+        mma_f16_16816(o[4 * w + k], pa, b0[k], b1[k]);
+      }
+    }
+    return;
+  }
   const uint4 ta = lds128(vbase + sw128(vr, (uint32_t)g4));
   const uint4 tb = lds128(vbase + sw128(vr + 1u, (uint32_t)g4));
   const uint4 tc = lds128(vbase + sw128(vr + 8u, (uint32_t)g4));
@@ -234,7 +273,7 @@ __device__ __forceinline__ uint32_t keep_hi(int c4, int vrem) {  // tokens 2c+8,
 template <int HEAD_DIM, bool MULTI, bool KV8, int RULE>
 __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid_constant__ GqaParams p) {
   using Geo = GqaGeom<HEAD_DIM, KV8>;
-  static_assert(!KV8 || HEAD_DIM == 128, "FP8 pages use one 128-byte row per token and head");
+  static_assert(!KV8 || HEAD_DIM == 128 || HEAD_DIM == 64, "FP8 pages: one 128- or 64-byte row per token and head");
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* stage_mem = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * p.stage_bytes);
@@ -247,7 +286,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hg = blockIdx.y, cta = blockIdx.x, nctas = gridDim.x;
   const int B = p.B, bs = p.bs, D = p.D;
-  const uint32_t box_bytes = (uint32_t)p.hpc * bs * 128u;
+  const uint32_t box_bytes = (uint32_t)(p.hpc * bs * Geo::kRowBytes);
 
   if ((smem_u32(smem) & 1023u) != 0u) {  // swizzled TMA tiles need 1024-byte aligned stages
     if (tid == 0) atomicOr(p.status, kDevTimeout);
@@ -709,13 +748,15 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
       float* dL0 = complete ? gqa_l_ptr(p, si, out_row(hh * R + r0)) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r0;
       float* dL1 = complete ? gqa_l_ptr(p, si, out_row(hh * R + r1)) : sl + (size_t)rows_hg * HEAD_DIM + hh * R + r1;
       if constexpr (KV8) {
-        // n-tile i, column 2c (+1) holds dim 32c + i (+16): two runs of 16 consecutive dims
+        // n-tile i, column 2c (+1) holds dim 2c * NT + i (+NT), NT = kNTiles: two runs of NT
+        // consecutive dims (head_dim 128: 32c + i, +16; head_dim 64: 16c + i, +8)
+        constexpr int NT = Geo::kNTiles;
         if (row0) {
 #pragma unroll
           for (int i = 0; i < Geo::kNTiles; i += 4) {
-            *reinterpret_cast<float4*>(dO0 + 32 * c4 + i) =
+            *reinterpret_cast<float4*>(dO0 + 2 * NT * c4 + i) =
                 make_float4(o[i][0] * inv0, o[i + 1][0] * inv0, o[i + 2][0] * inv0, o[i + 3][0] * inv0);
-            *reinterpret_cast<float4*>(dO0 + 32 * c4 + 16 + i) =
+            *reinterpret_cast<float4*>(dO0 + 2 * NT * c4 + NT + i) =
                 make_float4(o[i][1] * inv0, o[i + 1][1] * inv0, o[i + 2][1] * inv0, o[i + 3][1] * inv0);
           }
           if (c4 == 0) *dL0 = complete ? lse0 * kLn2 : lse0;
@@ -723,9 +764,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1) gqa_decode_kernel(const __grid
         if (row1) {
 #pragma unroll
           for (int i = 0; i < Geo::kNTiles; i += 4) {
-            *reinterpret_cast<float4*>(dO1 + 32 * c4 + i) =
+            *reinterpret_cast<float4*>(dO1 + 2 * NT * c4 + i) =
                 make_float4(o[i][2] * inv1, o[i + 1][2] * inv1, o[i + 2][2] * inv1, o[i + 3][2] * inv1);
-            *reinterpret_cast<float4*>(dO1 + 32 * c4 + 16 + i) =
+            *reinterpret_cast<float4*>(dO1 + 2 * NT * c4 + NT + i) =
                 make_float4(o[i][3] * inv1, o[i + 1][3] * inv1, o[i + 2][3] * inv1, o[i + 3][3] * inv1);
           }
           if (c4 == 0) *dL1 = complete ? lse1 * kLn2 : lse1;
@@ -862,8 +903,9 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
     if (set.pool_pages[si] > 0) {
       const uint64_t rows = (uint64_t)set.pool_pages[si] * 2 * p.Hkv * p.bs;
       if (rows > (uint64_t)INT32_MAX) return DCP_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+      // boxes of 128-byte rows use the 128-byte swizzle; FP8 at head_dim 64 (64-byte rows) the 64-byte one
       if (encode_tiled_2d(&p.tmap[si], set.pool[si], HEAD_DIM, rows, HEAD_DIM * eb, GqaGeom<HEAD_DIM, KV8>::kBoxElems,
-                          (uint32_t)(p.hpc * p.bs), eb) != CUDA_SUCCESS)
+                          (uint32_t)(p.hpc * p.bs), eb, GqaGeom<HEAD_DIM, KV8>::kRowBytes) != CUDA_SUCCESS)
         return DCP_ERR_CUDA;
     }
   }
@@ -888,9 +930,13 @@ dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st) {
   const bool multi = d.q_len > 1;
   if (d.kv_dtype == DCP_KV_FP8_E4M3) {
-    if (d.head_dim_qk != 128) return DCP_ERR_UNSUPPORTED;
-    return multi ? launch_gqa_impl<128, true, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
-                 : launch_gqa_impl<128, false, true>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+    if (d.head_dim_qk == 128)
+      return multi ? launch_gqa_impl<128, true, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                   : launch_gqa_impl<128, false, true>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+    if (d.head_dim_qk == 64)
+      return multi ? launch_gqa_impl<64, true, true>(d, D, set, q, seq_lens, ws, ws_bytes, st)
+                   : launch_gqa_impl<64, false, true>(d, D, set, q, seq_lens, ws, ws_bytes, st);
+    return DCP_ERR_UNSUPPORTED;
   }
   if (d.head_dim_qk == 128)
     return multi ? launch_gqa_impl<128, true, false>(d, D, set, q, seq_lens, ws, ws_bytes, st)

@@ -50,7 +50,8 @@ int device_sm_count();
 
 // cuTensorMapEncodeTiled obtained through the runtime's driver entry point.
 CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t inner_elems, uint64_t rows,
-                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes = 2);
+                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows, int elem_bytes = 2,
+                         int swizzle_bytes = 128);  // 128: SWIZZLE_128B (rows of 128 bytes); 64: SWIZZLE_64B
 
 dcp_status launch_gqa_decode(const dcp_attn_desc& d, int D, const ShardSet& set, const void* q,
                              const int32_t* seq_lens, void* ws, size_t ws_bytes, cudaStream_t st);

@@ -1,6 +1,6 @@
-"""FP8 (E4M3) KV cache on the GPU: the cache write's codes must equal the oracle's byte for
-byte, and decoding the FP8 cache must match the oracle's attention over the values the codes
-stand for (scale * e4m3(code)), per shard and merged."""
+"""FP8 (E4M3) GQA KV cache on the GPU (head_dim 128 and 64): the cache write's codes must equal
+the oracle's byte for byte, and decoding the FP8 cache must match the oracle's attention over the
+values the codes stand for (scale * e4m3(code)), per shard and merged."""
 import numpy as np
 import pytest
 import torch
@@ -70,10 +70,11 @@ def _check(w, D, cache, k_scale, v_scale):
 LENS = [1, 15, 16, 17, 300, 1000, 2500]
 
 
+@pytest.mark.parametrize("hd", [128, 64])
 @pytest.mark.parametrize("D,perm", [(1, 0), (3, 7), (4, 0)])
 @pytest.mark.parametrize("scales", [(0.05, 0.02), (1.0, 1.0), (0.001, 0.5)])  # the last one saturates K
-def test_cache_write_is_byte_exact(D, perm, scales):
-    w = synth.custom(synth.GQA, LENS, 16, 2, 128, 128, 16, seed=80 + D)
+def test_cache_write_is_byte_exact(D, perm, scales, hd):
+    w = synth.custom(synth.GQA, LENS, 16, 2, hd, hd, 16, seed=80 + D)
     cache, _ = _cache(w, D, *scales, perm_seed=perm)
     want = _oracle_pools(w, D, *scales, cache.max_local_blocks, perm)
     got = _pools_u8(cache)
@@ -81,15 +82,39 @@ def test_cache_write_is_byte_exact(D, perm, scales):
         np.testing.assert_array_equal(got[s][:want[s].size], want[s])
 
 
+@pytest.mark.parametrize("hd", [128, 64])
 @pytest.mark.parametrize("D", [1, 3, 4])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_decode_parity(D, bs):
-    w = synth.custom(synth.GQA, LENS, 16, 2, 128, 128, bs, seed=90 + D + bs)
+def test_decode_parity(D, bs, hd):
+    w = synth.custom(synth.GQA, LENS, 16, 2, hd, hd, bs, seed=90 + D + bs)
     cache, q = _cache(w, D, 0.05, 0.02)
     cache.step(q)
     torch.cuda.synchronize()
     _check(w, D, cache, 0.05, 0.02)
     assert cache.device_error() == 0
+
+
+def test_head_dim_64_wide_blocks_and_contiguous_rule():
+    # head_dim 64 allows blocks up to 256 tokens; the contiguous-chunk rule through the FP8 kernel
+    w = synth.custom(synth.GQA, [1, 255, 256, 257, 3000], 8, 2, 64, 64, 256, seed=33)
+    cache, q = _cache(w, 2, 0.05, 0.05)
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, 2, cache, 0.05, 0.05)
+    wc = synth.custom(synth.GQA, [5, 700, 1600], 16, 2, 64, 64, 16, seed=34)
+    cc = ShardedPagedCache(wc.layout, wc.num_q_heads, wc.num_kv_heads, wc.head_dim_qk, wc.head_dim_v, wc.block_size,
+                           3, wc.seq_lens, wc.softmax_scale, 0, "cuda", pool_fill=0xFFFF, kv_dtype=FP8, k_scale=0.05,
+                           v_scale=0.05, shard_rule=dcp.DCP_SHARD_CONTIGUOUS)
+    cc.place(torch.from_numpy(host_kv(wc).view(np.int16)).cuda())
+    cc.step(torch.from_numpy(host_q(wc).view(np.int16)).cuda())
+    torch.cuda.synchronize()
+    O, L = cc.O.cpu().numpy(), cc.LSE.cpu().numpy()
+    for b in range(wc.batch):
+        vals = oracle.dequantize_kv_gqa(oracle.quantize_kv_gqa(wc.kv_source(b), 0.05, 0.05), 0.05, 0.05)
+        Ob, Lb, _, _ = oracle.sharded_values(wc.layout, 16, 2, 64, 64, wc.query(b), vals, wc.softmax_scale, 16, 3,
+                                             oracle.CONTIGUOUS)
+        assert_o_close(O[b], Ob, O_TOL, f"O[{b}]")
+        assert_lse_close(L[b], Lb, LSE_TOL, f"LSE[{b}]")
 
 
 def test_decode_parity_70b_heads():
@@ -100,17 +125,19 @@ def test_decode_parity_70b_heads():
     _check(w, 4, cache, 0.01, 0.01)
 
 
+@pytest.mark.parametrize("hd", [128, 64])
 @pytest.mark.parametrize("q_len", [2, 4])
-def test_multi_token_decode(q_len):
-    w = synth.custom(synth.GQA, [2, 17, 333, 1500], 16, 2, 128, 128, 16, seed=50 + q_len, q_len=q_len)
+def test_multi_token_decode(q_len, hd):
+    w = synth.custom(synth.GQA, [2, 17, 333, 1500], 16, 2, hd, hd, 16, seed=50 + q_len, q_len=q_len)
     cache, q = _cache(w, 3, 0.05, 0.05)
     cache.step(q)
     torch.cuda.synchronize()
     _check(w, 3, cache, 0.05, 0.05)
 
 
-def test_d_invariance():
-    w = synth.custom(synth.GQA, [3, 700, 5000], 16, 2, 128, 128, 16, seed=13)
+@pytest.mark.parametrize("hd", [128, 64])
+def test_d_invariance(hd):
+    w = synth.custom(synth.GQA, [3, 700, 5000], 16, 2, hd, hd, 16, seed=13)
     outs = []
     for D in (1, 2, 5):
         cache, q = _cache(w, D, 0.05, 0.05)
@@ -146,11 +173,12 @@ def test_append_writes_the_same_codes_as_placement():
 
 
 
-@pytest.mark.parametrize("D,q_len", [(1, 1), (2, 1), (3, 1), (3, 2), (2, 4)])
-def test_two_pages_per_step_path(D, q_len):
+@pytest.mark.parametrize("D,q_len,hd", [(1, 1, 128), (2, 1, 128), (3, 1, 128), (3, 2, 128), (2, 4, 128),
+                                        (1, 1, 64), (3, 1, 64), (3, 2, 64)])
+def test_two_pages_per_step_path(D, q_len, hd):
     # eight KV heads at block 16 (one warp per head and row tile, one chunk per page): pages go two
     # at a time, odd page counts leave a single page, partial last pages and one-token requests included
-    w = synth.custom(synth.GQA, [1, 16, 17, 31, 32, 33, 48, 500, 1111], 64, 8, 128, 128, 16, seed=17 + D,
+    w = synth.custom(synth.GQA, [1, 16, 17, 31, 32, 33, 48, 500, 1111], 64, 8, hd, hd, 16, seed=17 + D,
                      kv_amp=0.5, q_len=q_len)
     cache, q = _cache(w, D, 0.01, 0.01)
     cache.step(q)

@@ -180,14 +180,15 @@ def test_descriptor_layout_matches_header():
 
 
 def test_fp8_page_bytes_and_rejections():
-    # FP8 pools: GQA with head_dim 128 and MLA; a page is one byte per value.  The MLA latent is one
+    # FP8 pools: GQA (head_dim 64 and 128) and MLA; a page is one byte per value.  The MLA latent is one
     # tensor, so its key and value scales must be the same number.
     assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1,
                                                dcp.DCP_KV_FP8_E4M3, 0.5, 0.5)) == 64 * 576
     unequal = dcp.make_desc(dcp.DCP_LAYOUT_MLA, 1, 64, 1, 576, 512, 64, 1, 0.07, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 0.5)
     assert dcp.dcp_kv_page_bytes(unequal) == 0
     assert dcp.dcp_decode_workspace_bytes(unequal, 2) == 0
-    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == 0
+    assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 64, 64, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == \
+        2 * 2 * 16 * 64
     assert dcp.dcp_kv_page_bytes(dcp.make_desc(dcp.DCP_LAYOUT_GQA, 1, 8, 2, 128, 128, 16, 1, 0.1, 1, dcp.DCP_KV_FP8_E4M3, 1.0, 1.0)) == \
         2 * 2 * 16 * 128
     for ks, vs in ((0.0, 1.0), (1.0, float("inf")), (-1.0, 1.0), (float("nan"), 1.0)):
@@ -250,4 +251,4 @@ def test_descriptor_option_matrix(q_len, rule):
     assert dcp.dcp_kv_page_bytes(m8) * 2 == dcp.dcp_kv_page_bytes(mla)
     assert dcp.dcp_decode_workspace_bytes(m8, 4) == dcp.dcp_decode_workspace_bytes(mla, 4)
     assert dcp.dcp_kv_page_bytes(desc(1, 1, 64, 1, 576, 64)) == 0  # FP8 MLA with unequal scales
-    assert dcp.dcp_kv_page_bytes(desc(0, 1, 16, 2, 64)) == 0      # FP8 head_dim 64
+    assert dcp.dcp_kv_page_bytes(desc(0, 1, 16, 2, 64)) == 2 * 2 * 16 * 64  # FP8 head_dim 64: one byte per value

@@ -68,11 +68,13 @@ class RankShardedDecode:
     Holds that shard's pool and block table only; ``place`` writes this shard's tokens of the
     unsharded KV, ``step`` runs one decode step (partial, exchange, merge) and returns the merged
     ``(O, LSE)`` of this rank's heads: ``O[batch][q_len][Hk][d_v]``, ``LSE[batch][q_len][Hk]``.
+    ``kv_dtype`` / ``k_scale`` / ``v_scale`` select an FP8 E4M3 pool as in ``dcp_attn_desc``.
     """
 
     def __init__(self, layout: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
                  block_size: int, seq_lens: Sequence[int], softmax_scale: float, group=None, device="cuda",
-                 q_len: int = 1, perm_seed: int = 0):
+                 q_len: int = 1, perm_seed: int = 0, kv_dtype: int = 0, k_scale: float = 1.0,
+                 v_scale: float = 1.0):
         import torch.distributed as dist
         self.group = group
         self.rank = dist.get_rank(group)
@@ -88,7 +90,8 @@ class RankShardedDecode:
         tables, self.local_len = dcp.dcp_build_block_table(self.seq_lens, block_size, self.D, perm_seed,
                                                            self.max_local_blocks)
         self.desc = dcp.make_desc(layout, self.batch, num_q_heads, num_kv_heads, head_dim_qk, head_dim_v,
-                                  block_size, self.max_local_blocks, softmax_scale, q_len)
+                                  block_size, self.max_local_blocks, softmax_scale, q_len, kv_dtype, k_scale,
+                                  v_scale)
         page_bytes = dcp.dcp_kv_page_bytes(self.desc)
         if page_bytes == 0:
             raise ValueError("unsupported attention shape")

@@ -20,20 +20,38 @@ from sequence_sharded_decode_paged_b200 import dcp
 pytestmark = pytest.mark.gpu
 
 
+FP8_SCALE = 2.0 ** -6
+
+
 def _cases():
+    # (name, workload, D, FP8 cache)
     return [
-        ("gqa", synth.custom(synth.GQA, [3000, 17, 900, 0, 1], 32, 4, 128, 128, 16, seed=61, kv_amp=0.5), 3),
-        ("gqa_draft", synth.custom(synth.GQA, [2000, 5, 700], 16, 2, 64, 64, 16, seed=62, q_len=3), 2),
-        ("mla", synth.custom(synth.MLA, [5000, 65, 1, 3000], 64, 1, 576, 512, 64, seed=63), 4),
-        ("mla_draft", synth.custom(synth.MLA, [1500, 130], 64, 1, 576, 512, 64, seed=64, q_len=2), 2),
+        ("gqa", synth.custom(synth.GQA, [3000, 17, 900, 0, 1], 32, 4, 128, 128, 16, seed=61, kv_amp=0.5), 3, False),
+        ("gqa_draft", synth.custom(synth.GQA, [2000, 5, 700], 16, 2, 64, 64, 16, seed=62, q_len=3), 2, False),
+        ("mla", synth.custom(synth.MLA, [5000, 65, 1, 3000], 64, 1, 576, 512, 64, seed=63), 4, False),
+        ("mla_draft", synth.custom(synth.MLA, [1500, 130], 64, 1, 576, 512, 64, seed=64, q_len=2), 2, False),
+        ("mla_fp8", synth.custom(synth.MLA, [2500, 65, 1], 64, 1, 576, 512, 64, seed=69), 2, True),
+        ("gqa64_fp8", synth.custom(synth.GQA, [1800, 40, 3], 16, 2, 64, 64, 16, seed=70), 3, True),
     ]
 
 
-@pytest.mark.parametrize("idx", range(4))
+def _fp8_cache(w, D):
+    from gpu_cases import host_kv, host_q
+    from sequence_sharded_decode_paged_b200.cache import ShardedPagedCache
+    cache = ShardedPagedCache(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size, D,
+                              w.seq_lens, w.softmax_scale, 0, "cuda", pool_fill=0xFFFF, q_len=w.q_len,
+                              kv_dtype=dcp.DCP_KV_FP8_E4M3, k_scale=FP8_SCALE, v_scale=FP8_SCALE)
+    cache.place(torch.from_numpy(host_kv(w).view(np.int16)).cuda())
+    return cache, torch.from_numpy(host_q(w).view(np.int16)).cuda()
+
+
+@pytest.mark.parametrize("idx", range(6))
 @pytest.mark.parametrize("n_owners", [1, 2, 4, 8])
 def test_owner_major_partial_is_the_standard_partial_permuted(idx, n_owners):
-    name, w, D = _cases()[idx]
-    cache, q = build_cache(w, D)
+    name, w, D, fp8 = _cases()[idx]
+    if w.num_q_heads % n_owners != 0:
+        pytest.skip("owners must split the query heads evenly")
+    cache, q = _fp8_cache(w, D) if fp8 else build_cache(w, D)
     d = cache.desc
     Hq, dv, B, ql = w.num_q_heads, w.head_dim_v, w.batch, w.q_len
     Hk = Hq // n_owners
@@ -67,21 +85,22 @@ def test_owner_major_rejects_uneven_owners():
     assert e.value.status == dcp.DCP_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("layout", [synth.GQA, synth.MLA])
-def test_rank_step_on_a_one_rank_nccl_group(layout, tmp_path):
+@pytest.mark.parametrize("layout,fp8", [(synth.GQA, False), (synth.MLA, False), (synth.MLA, True)])
+def test_rank_step_on_a_one_rank_nccl_group(layout, fp8, tmp_path):
     import torch.distributed as dist
     from sequence_sharded_decode_paged_b200.ranks import RankShardedDecode
     if layout == synth.GQA:
         w = synth.custom(synth.GQA, [2500, 40, 0, 800], 16, 2, 128, 128, 16, seed=66, kv_amp=0.5)
     else:
         w = synth.custom(synth.MLA, [3000, 70, 900], 64, 1, 576, 512, 64, seed=67)
-    cache, q = build_cache(w, 1)
+    cache, q = _fp8_cache(w, 1) if fp8 else build_cache(w, 1)
     O_ref, L_ref = [t.clone() for t in cache.step(q)]
     store = dist.FileStore(str(tmp_path / "store"), 1)
     dist.init_process_group("nccl", store=store, rank=0, world_size=1)
     try:
+        extra = dict(kv_dtype=dcp.DCP_KV_FP8_E4M3, k_scale=FP8_SCALE, v_scale=FP8_SCALE) if fp8 else {}
         r = RankShardedDecode(w.layout, w.num_q_heads, w.num_kv_heads, w.head_dim_qk, w.head_dim_v, w.block_size,
-                              w.seq_lens, w.softmax_scale, device="cuda")
+                              w.seq_lens, w.softmax_scale, device="cuda", **extra)
         from gpu_cases import host_kv
         kv = torch.from_numpy(host_kv(w).view(np.int16)).cuda()
         r.place(kv, cache.cu_seqlens)

@@ -22,7 +22,7 @@
  * Conventions for every call:
  *   - The caller owns all memory.  The library never allocates device or
  *     host memory on the compute path and keeps no global state (it caches
- *     one driver entry point, looked up once).  Calls are thread-safe.
+ *     two driver entry points, each looked up once).  Calls are thread-safe.
  *   - "device" pointers are CUDA device addresses (e.g. a torch tensor's
  *     data_ptr()); "host" pointers are ordinary CPU memory.
  *   - GPU calls are asynchronous on `stream` (a cudaStream_t passed as
@@ -334,13 +334,58 @@ DCP_API dcp_status dcp_decode_partial(const dcp_attn_desc *desc, const void *q, 
  * With n_owners = 1 chunk 0 is dcp_decode_partial's O_i followed by LSE_i.
  *   send       device fp32, n_owners * dcp_owner_chunk_floats(desc, n_owners) floats, 16-byte aligned.
  * Other arguments, results and errors as dcp_decode_partial; DCP_ERR_INVALID_ARG
- * if n_owners < 1 or it does not divide num_q_heads.
+ * if n_owners < 1, n_owners > 16 or it does not divide num_q_heads.
  */
 DCP_API size_t dcp_owner_chunk_floats(const dcp_attn_desc *desc, int32_t n_owners);
 DCP_API dcp_status dcp_decode_partial_owner_major(const dcp_attn_desc *desc, const void *q, const void *kv_pool,
                                                   int32_t pool_pages, const int32_t *table, const int32_t *seq_lens,
                                                   int32_t shard, int32_t D, int32_t n_owners, float *send,
                                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The same partial with the exchange folded into the decode kernel: owner k's
+ * chunk (the layout above) is written straight to owner_chunks[k], so no send
+ * buffer and no separate all-to-all are needed.  [P1 "A2 方法细节", step 3.]
+ * owner_chunks[k] may point into another GPU's memory that this process has
+ * mapped (peer access, or dcp_ipc_open below): the kernel's epilogue and split
+ * combine store the rows with ordinary global stores, so the transfer happens
+ * while the last pieces of the partial are still being computed.  The caller
+ * orders the stores before the owner reads its chunks (e.g. the stream's
+ * completion followed by a barrier of the rank group) and, when it reuses a
+ * chunk buffer, the owner's previous read before this call.
+ *   owner_chunks  host array of n_owners device pointers, each 16-byte aligned,
+ *                 dcp_owner_chunk_floats(desc, n_owners) floats.
+ * Other arguments, results and errors as dcp_decode_partial_owner_major;
+ * DCP_ERR_INVALID_ARG for a null or misaligned chunk pointer.
+ */
+DCP_API dcp_status dcp_decode_partial_to_owners(const dcp_attn_desc *desc, const void *q, const void *kv_pool,
+                                                int32_t pool_pages, const int32_t *table, const int32_t *seq_lens,
+                                                int32_t shard, int32_t D, int32_t n_owners,
+                                                float *const *owner_chunks, void *workspace,
+                                                size_t workspace_bytes, void *stream);
+
+/*
+ * Mapping a device buffer of another process (CUDA IPC), for owner chunks on
+ * other GPUs.  [The multi-GPU form above; the pages name no mechanism.]
+ *   dcp_ipc_handle_bytes  size of a handle (host bytes).
+ *   dcp_ipc_export        device_ptr: device memory of this process.  Writes the
+ *                         handle of the allocation that holds it to handle_out
+ *                         (host, dcp_ipc_handle_bytes()) and device_ptr's byte
+ *                         offset inside that allocation to *offset_out.
+ *                         DCP_ERR_INVALID_ARG if device_ptr is not device memory.
+ *   dcp_ipc_open          maps the allocation a handle names (from another
+ *                         process; peer access is enabled when needed) and
+ *                         returns its base in *base_out; the buffer is at
+ *                         base + offset.  Must not be called on a handle that
+ *                         this process exported.
+ *   dcp_ipc_close         unmaps a base returned by dcp_ipc_open.
+ * Host calls; DCP_ERR_CUDA when the CUDA runtime refuses.  No multicast object
+ * is created.
+ */
+DCP_API size_t dcp_ipc_handle_bytes(void);
+DCP_API dcp_status dcp_ipc_export(const void *device_ptr, void *handle_out, uint64_t *offset_out);
+DCP_API dcp_status dcp_ipc_open(const void *handle, void **base_out);
+DCP_API dcp_status dcp_ipc_close(void *base);
 
 /*
  * All D partials in one launch.  Host arrays of D device pointers:

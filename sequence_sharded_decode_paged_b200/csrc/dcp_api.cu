@@ -402,7 +402,7 @@ dcp_status dcp_decode_partial_owner_major(const dcp_attn_desc* desc, const void*
                                           void* workspace, size_t workspace_bytes, void* stream) {
   dcp_status st = check_decode_args(desc, D, q, seq_lens, workspace, workspace_bytes);
   if (st != DCP_OK) return st;
-  if (shard < 0 || shard >= D || send == nullptr) return DCP_ERR_INVALID_ARG;
+  if (shard < 0 || shard >= D || send == nullptr || n_owners > kMaxShardsHost) return DCP_ERR_INVALID_ARG;
   const size_t chunk = dcp_owner_chunk_floats(desc, n_owners);
   if (chunk == 0) return DCP_ERR_INVALID_ARG;  // n_owners must divide the query heads
   const size_t rows = (size_t)desc->batch * desc->q_len * (desc->num_q_heads / n_owners);
@@ -415,7 +415,39 @@ dcp_status dcp_decode_partial_owner_major(const dcp_attn_desc* desc, const void*
   set.O[0] = send;
   set.LSE[0] = send + rows * desc->head_dim_v;
   set.owner_heads = desc->num_q_heads / n_owners;
-  set.owner_stride = chunk;
+  for (int k = 1; k < n_owners; ++k) {
+    set.owner_O[k] = send + k * chunk;
+    set.owner_L[k] = send + k * chunk + rows * desc->head_dim_v;
+  }
+  return run_decode(desc, D, set, q, seq_lens, workspace, workspace_bytes, stream);
+}
+
+dcp_status dcp_decode_partial_to_owners(const dcp_attn_desc* desc, const void* q, const void* kv_pool,
+                                        int32_t pool_pages, const int32_t* table, const int32_t* seq_lens,
+                                        int32_t shard, int32_t D, int32_t n_owners, float* const* owner_chunks,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  dcp_status st = check_decode_args(desc, D, q, seq_lens, workspace, workspace_bytes);
+  if (st != DCP_OK) return st;
+  if (shard < 0 || shard >= D || owner_chunks == nullptr || n_owners > kMaxShardsHost) return DCP_ERR_INVALID_ARG;
+  const size_t chunk = dcp_owner_chunk_floats(desc, n_owners);
+  if (chunk == 0) return DCP_ERR_INVALID_ARG;  // n_owners must divide the query heads
+  const size_t rows = (size_t)desc->batch * desc->q_len * (desc->num_q_heads / n_owners);
+  for (int k = 0; k < n_owners; ++k)
+    if (owner_chunks[k] == nullptr || (reinterpret_cast<uintptr_t>(owner_chunks[k]) & 15u) != 0)
+      return DCP_ERR_INVALID_ARG;
+  ShardSet set;
+  set.n = 1;
+  set.shard[0] = shard;
+  set.pool[0] = kv_pool;
+  set.pool_pages[0] = pool_pages;
+  set.table[0] = table;
+  set.O[0] = owner_chunks[0];
+  set.LSE[0] = owner_chunks[0] + rows * desc->head_dim_v;
+  set.owner_heads = desc->num_q_heads / n_owners;
+  for (int k = 1; k < n_owners; ++k) {
+    set.owner_O[k] = owner_chunks[k];
+    set.owner_L[k] = owner_chunks[k] + rows * desc->head_dim_v;
+  }
   return run_decode(desc, D, set, q, seq_lens, workspace, workspace_bytes, stream);
 }
 

@@ -82,11 +82,13 @@ struct GqaParams {
   int hpc, n_hg, stages, wph;
   uint32_t stage_bytes;
   int slot_floats;
-  // Output layout: query heads are owned in consecutive slices of Hk heads, and owner k's
-  // O rows (and LSE rows) start k * own_stride floats after owner 0's.  The standard
-  // layout is Hk = Hq (a single owner).
+  // Output layout: query heads are owned in consecutive slices of Hk heads; owner 0's O and
+  // LSE rows start at O[si] / LSE[si], owner k's (k >= 1) at own_O[k] / own_L[k] (any address
+  // this GPU can store to, a peer GPU's memory included).  The standard layout is Hk = Hq (a
+  // single owner).
   int Hk;
-  size_t own_stride;
+  float* own_O[kMaxShards];
+  float* own_L[kMaxShards];
 };
 
 // Output row of head-group row rr = h * R + r (KV head kv0 + h, local row r = query token
@@ -104,10 +106,10 @@ __device__ __forceinline__ OutRow gqa_out_row(int rr, int b, int ql, int kv0, in
 }
 template <int HEAD_DIM>
 __device__ __forceinline__ float* gqa_o_ptr(const GqaParams& p, int si, OutRow o) {
-  return p.O[si] + o.own * p.own_stride + o.row * HEAD_DIM;
+  return (o.own == 0 ? p.O[si] : p.own_O[o.own]) + o.row * HEAD_DIM;
 }
 __device__ __forceinline__ float* gqa_l_ptr(const GqaParams& p, int si, OutRow o) {
-  return p.LSE[si] + o.own * p.own_stride + o.row;
+  return (o.own == 0 ? p.LSE[si] : p.own_L[o.own]) + o.row;
 }
 
 template <int HEAD_DIM, bool KV8>
@@ -893,7 +895,10 @@ static dcp_status launch_gqa_impl(const dcp_attn_desc& d, int D, const ShardSet&
   p.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slots_off);
   p.slot_floats = L.slot_floats;
   p.Hk = set.owner_heads > 0 ? set.owner_heads : d.num_q_heads;
-  p.own_stride = set.owner_stride;
+  for (int k = 0; k < kMaxShards; ++k) {
+    p.own_O[k] = set.owner_O[k];
+    p.own_L[k] = set.owner_L[k];
+  }
   for (int si = 0; si < set.n; ++si) {
     p.table[si] = set.table[si];
     p.O[si] = set.O[si];

@@ -23,11 +23,14 @@ struct ShardSet {
   float* O[kMaxShardsHost];
   float* LSE[kMaxShardsHost];
   // Output layout.  owner_heads = 0: the standard [b][j][h] rows.  Otherwise query heads are
-  // owned in consecutive slices of owner_heads heads, row (b, j, h) goes to owner h / owner_heads
-  // at row (b * q_len + j) * owner_heads + h % owner_heads, and owner k's rows (O and LSE
-  // alike) start k * owner_stride floats after owner 0's.
+  // owned in consecutive slices of owner_heads heads, and row (b, j, h) goes to owner
+  // k = h / owner_heads at row (b * q_len + j) * owner_heads + h % owner_heads of that owner's
+  // block: owner 0's O and LSE rows start at O[0] / LSE[0], owner k's (k >= 1) at owner_O[k] /
+  // owner_L[k] (set only with a single shard slot; any device address this GPU can store to,
+  // a peer GPU's memory included).
   int owner_heads = 0;
-  size_t owner_stride = 0;
+  float* owner_O[kMaxShardsHost] = {};
+  float* owner_L[kMaxShardsHost] = {};
 };
 
 // Workspace layout shared by the decode kernels.

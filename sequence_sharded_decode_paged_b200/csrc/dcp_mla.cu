@@ -130,7 +130,7 @@ struct MlaMisc {
   float inv_l[kMlaHeads];
   float lse2[kMlaHeads];
   float part[4][kMlaHeads];   // per-sub-partition partial maxima or sums
-  size_t rowoff[kMlaHeads];   // epilogue / combine: float offset of head h's output row
+  float* rowptr[kMlaHeads];   // epilogue / combine: head h's output row
   int scratch[32];
 };
 static_assert(sizeof(MlaMisc) <= kMiscBytes, "misc block");
@@ -160,11 +160,13 @@ struct MlaParams {
   float scale_log2;
   float v_scale;  // multiplies the normalised O (the FP8 latent's scale; 1 for bf16)
   int n_si, B, D, mlb, slot_floats, q_len;
-  // Output layout: query heads are owned in consecutive slices of Hk heads, and owner k's
-  // O rows (and LSE rows) start k * own_stride floats after owner 0's.  The standard layout
-  // is Hk = 64 (a single owner).
+  // Output layout: query heads are owned in consecutive slices of Hk heads; owner 0's O and
+  // LSE rows start at O[si] / LSE[si], owner k's (k >= 1) at own_O[k] / own_L[k] (any address
+  // this GPU can store to, a peer GPU's memory included).  The standard layout is Hk = 64 (a
+  // single owner).
   int Hk;
-  size_t own_stride;
+  float* own_O[kMaxShards];
+  float* own_L[kMaxShards];
 };
 
 namespace {
@@ -561,11 +563,11 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
       const size_t row0 = ((size_t)b * ql + jq) * p.Hk;
       auto o_row = [&](int h) -> float* {
         const int own = h / p.Hk;
-        return p.O[si] + own * p.own_stride + (row0 + (h - own * p.Hk)) * kMlaDv;
+        return (own == 0 ? p.O[si] : p.own_O[own]) + (row0 + (h - own * p.Hk)) * kMlaDv;
       };
       auto l_ptr = [&](int h) -> float* {
         const int own = h / p.Hk;
-        return p.LSE[si] + own * p.own_stride + row0 + (h - own * p.Hk);
+        return (own == 0 ? p.LSE[si] : p.own_L[own]) + row0 + (h - own * p.Hk);
       };
       const int lim = seq_len - (ql - 1 - jq);  // tokens this query token sees
       // logical block of local page j: g0 + j * gstride (computed once per segment)
@@ -747,7 +749,6 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
       const bool complete = (c0 == c1);
       const int slot_i = complete ? 0 : 2 * cta + ((cta == c0 && pre != c0 * P) ? 1 : 0);
       float* slot_base = p.slots + ((size_t)slot_i * ql + jq) * p.slot_floats;
-      float* const obase = complete ? p.O[si] : slot_base;
       named_bar_sync(2, kSoftmaxThreads);
       if (ts < kMlaHeads) {
         const float lt = (misc->part[0][ts] + misc->part[1][ts]) + (misc->part[2][ts] + misc->part[3][ts]);
@@ -755,7 +756,7 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
         misc->inv_l[ts] = lt > 0.f ? (KV8 ? p.v_scale / lt : 1.f / lt) : 0.f;
         misc->lse2[ts] = lt > 0.f ? mh + __log2f(lt) : -INFINITY;
         // row offsets once per piece, so that the stores below need no owner arithmetic
-        misc->rowoff[ts] = complete ? (size_t)(o_row(ts) - p.O[si]) : (size_t)ts * kMlaDv;
+        misc->rowptr[ts] = complete ? o_row(ts) : slot_base + (size_t)ts * kMlaDv;
       }
       named_bar_sync(2, kSoftmaxThreads);
 #pragma unroll 1
@@ -767,11 +768,11 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
             tmem_ld32(tbase + lane_off + kColO + mt * 64 + c, v);
             tmem_ld_wait();
           }
-          float* const col = obase + (mt * 128 + 32 * q4 + lane);  // this thread's value dim
+          const int col = mt * 128 + 32 * q4 + lane;  // this thread's value dim
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float inv = misc->inv_l[c + i];
-            col[misc->rowoff[c + i]] = (inv == 0.f || dead) ? 0.f : v[i] * inv;
+            misc->rowptr[c + i][col] = (inv == 0.f || dead) ? 0.f : v[i] * inv;
           }
         }
       if (ts < kMlaHeads) {
@@ -825,7 +826,7 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
               }
               misc->inv_l[ts] = wsum > 0.f ? 1.f / wsum : 0.f;
               *l_ptr(ts) = wsum > 0.f ? (mx + __log2f(wsum)) * kLn2 : -INFINITY;
-              misc->rowoff[ts] = (size_t)(o_row(ts) - p.O[si]);
+              misc->rowptr[ts] = o_row(ts);
             }
             named_bar_sync(2, kSoftmaxThreads);
             const int ch = ts & 127, rh = ts >> 7;  // chunk of a row; rows 2u + rh
@@ -854,7 +855,7 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
               for (int u = 0; u < 8; ++u) {
                 const int r = 2 * (u0 + u) + rh;
                 const float inv = misc->inv_l[r];
-                reinterpret_cast<float4*>(p.O[si] + misc->rowoff[r])[ch] =
+                reinterpret_cast<float4*>(misc->rowptr[r])[ch] =
                     make_float4(acc[u].x * inv, acc[u].y * inv, acc[u].z * inv, acc[u].w * inv);
               }
             }
@@ -996,7 +997,10 @@ dcp_status launch_mla_decode(const dcp_attn_desc& d, int D, const ShardSet& set,
   p.v_scale = kv8 ? d.v_scale : 1.f;
   p.q_len = d.q_len;
   p.Hk = set.owner_heads > 0 ? set.owner_heads : kMlaHeads;
-  p.own_stride = set.owner_stride;
+  for (int k = 0; k < kMaxShards; ++k) {
+    p.own_O[k] = set.owner_O[k];
+    p.own_L[k] = set.owner_L[k];
+  }
   p.seq_lens = seq_lens;
   p.status = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.status_off);
   p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + L.counters_off);

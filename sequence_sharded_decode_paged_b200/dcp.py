@@ -12,7 +12,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -30,7 +30,9 @@ EXPORTED = ["dcp_version", "dcp_status_string", "dcp_block_table_extent", "dcp_b
             "dcp_decode_partial", "dcp_decode_partial_all", "dcp_lse_merge", "dcp_read_device_error",
             "dcp_validate_config", "dcp_decode_partial_all_noalloc", "dcp_noalloc_read_device_error",
             "dcp_grow_block_table", "dcp_append_kv", "dcp_host_step_staging_bytes", "dcp_decode_step_host",
-            "dcp_owner_chunk_floats", "dcp_decode_partial_owner_major", "dcp_check_wait_timeout"]
+            "dcp_owner_chunk_floats", "dcp_decode_partial_owner_major", "dcp_check_wait_timeout",
+            "dcp_decode_partial_to_owners", "dcp_ipc_handle_bytes", "dcp_ipc_export", "dcp_ipc_open",
+            "dcp_ipc_close"]
 
 
 class DcpError(RuntimeError):
@@ -75,6 +77,11 @@ def _load() -> C.CDLL:
         "dcp_host_step_staging_bytes": (sz, [p, i32]),
         "dcp_owner_chunk_floats": (sz, [p, i32]),
         "dcp_decode_partial_owner_major": (C.c_int, [p, p, p, i32, p, p, i32, i32, i32, p, p, sz, p]),
+        "dcp_decode_partial_to_owners": (C.c_int, [p, p, p, i32, p, p, i32, i32, i32, p, p, sz, p]),
+        "dcp_ipc_handle_bytes": (sz, []),
+        "dcp_ipc_export": (C.c_int, [p, p, p]),
+        "dcp_ipc_open": (C.c_int, [p, p]),
+        "dcp_ipc_close": (C.c_int, [p]),
         "dcp_decode_step_host": (C.c_int, [p, i32, p, p, p, p, p, p, sz, p, sz, p, p, p]),
         "dcp_grow_block_table": (C.c_int, [p, p, i32, i32, i32, i32, p, p, p, p]),
         "dcp_append_kv": (C.c_int, [p, i32, p, p, p, p, p, p, p, p]),
@@ -246,6 +253,42 @@ def dcp_decode_partial_owner_major(desc: dcp_attn_desc, q, kv_pool, pool_pages: 
     _check("dcp_decode_partial_owner_major", _lib.dcp_decode_partial_owner_major(
         C.byref(desc), _addr(q), _addr(kv_pool), pool_pages, _addr(table), _addr(seq_lens), shard, D, n_owners,
         _addr(send), _addr(workspace), n, _stream(stream)))
+
+
+def dcp_decode_partial_to_owners(desc: dcp_attn_desc, q, kv_pool, pool_pages: int, table, seq_lens, shard: int,
+                                 D: int, owner_chunks, workspace, workspace_bytes: Optional[int] = None,
+                                 stream=None) -> None:
+    """``owner_chunks``: one chunk per owner, each a device tensor or a raw device address (int), e.g. a
+    peer GPU's buffer mapped with ``dcp_ipc_open``."""
+    n = workspace_bytes if workspace_bytes is not None else workspace.numel() * workspace.element_size()
+    ptrs = (C.c_void_p * len(owner_chunks))(*[c if isinstance(c, int) else _addr(c) for c in owner_chunks])
+    _check("dcp_decode_partial_to_owners", _lib.dcp_decode_partial_to_owners(
+        C.byref(desc), _addr(q), _addr(kv_pool), pool_pages, _addr(table), _addr(seq_lens), shard, D,
+        len(owner_chunks), ptrs, _addr(workspace), n, _stream(stream)))
+
+
+def dcp_ipc_handle_bytes() -> int:
+    return int(_lib.dcp_ipc_handle_bytes())
+
+
+def dcp_ipc_export(device_tensor) -> Tuple[bytes, int]:
+    """(handle of the allocation holding the tensor's first byte, byte offset inside it)."""
+    h = C.create_string_buffer(dcp_ipc_handle_bytes())
+    off = C.c_uint64(0)
+    _check("dcp_ipc_export", _lib.dcp_ipc_export(_addr(device_tensor), h, C.byref(off)))
+    return h.raw, int(off.value)
+
+
+def dcp_ipc_open(handle: bytes) -> int:
+    """Maps another process's allocation; returns its base address in this process."""
+    h = C.create_string_buffer(handle, len(handle))
+    base = C.c_void_p(0)
+    _check("dcp_ipc_open", _lib.dcp_ipc_open(h, C.byref(base)))
+    return int(base.value)
+
+
+def dcp_ipc_close(base: int) -> None:
+    _check("dcp_ipc_close", _lib.dcp_ipc_close(C.c_void_p(base)))
 
 
 def dcp_decode_partial_all(desc: dcp_attn_desc, q, kv_pools, pool_pages, tables, seq_lens, D: int, O_parts,

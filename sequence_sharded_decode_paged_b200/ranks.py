@@ -22,6 +22,15 @@ Hk = Hq / D):
 * ``dcp_lse_merge`` (one launch) merges the D received chunks into the merged
   O and LSE of the rank's heads.
 
+With ``exchange="p2p"`` the first two steps are one: every rank maps every
+other rank's receive buffer into its address space (CUDA IPC, plain device
+memory, no multicast) and ``dcp_decode_partial_to_owners`` stores each owner's
+rows straight into that owner's buffer from the decode kernel's epilogue, so
+the transfer runs while the partial is still being finished.  The stream's
+completion and a barrier of the group then order those stores before the
+merge; two receive buffers alternate between steps, so that a rank writing
+step t+1's rows never touches a buffer an owner may still be merging.
+
 The query is an input of the step: the pages' AllGather-Q is the caller's
 (on one node every rank usually computes the same q already).
 """
@@ -74,8 +83,11 @@ class RankShardedDecode:
     def __init__(self, layout: int, num_q_heads: int, num_kv_heads: int, head_dim_qk: int, head_dim_v: int,
                  block_size: int, seq_lens: Sequence[int], softmax_scale: float, group=None, device="cuda",
                  q_len: int = 1, perm_seed: int = 0, kv_dtype: int = 0, k_scale: float = 1.0,
-                 v_scale: float = 1.0):
+                 v_scale: float = 1.0, exchange: str = "nccl"):
         import torch.distributed as dist
+        if exchange not in ("nccl", "p2p"):
+            raise ValueError("exchange must be 'nccl' (all-to-all) or 'p2p' (stores into the owners' buffers)")
+        self.exchange_kind = exchange
         self.group = group
         self.rank = dist.get_rank(group)
         self.D = dist.get_world_size(group)
@@ -104,8 +116,28 @@ class RankShardedDecode:
         dcp.dcp_workspace_init(self.workspace)
         self.chunk = dcp.dcp_owner_chunk_floats(self.desc, self.D)
         self.rows = self.batch * q_len * self.Hk
-        self.send = torch.empty(self.D * self.chunk, dtype=torch.float32, device=self.device)
-        self.recv = torch.empty_like(self.send)
+        self._mapped = []
+        if exchange == "nccl":
+            self.send = torch.empty(self.D * self.chunk, dtype=torch.float32, device=self.device)
+            self.recv = torch.empty_like(self.send)
+        else:
+            # two receive buffers in one allocation; every rank learns where every other rank's are
+            self.recv_pair = torch.empty(2 * self.D * self.chunk, dtype=torch.float32, device=self.device)
+            handle, offset = dcp.dcp_ipc_export(self.recv_pair)
+            peers = [None] * self.D
+            dist.all_gather_object(peers, (self.rank, handle, offset), group=group)
+            base_of = {}
+            for r, h, off in peers:
+                if r == self.rank:
+                    base_of[r] = self.recv_pair.data_ptr()
+                else:
+                    mapped = dcp.dcp_ipc_open(h)
+                    self._mapped.append(mapped)
+                    base_of[r] = mapped + off
+            # step parity i, owner r: chunk `rank` of owner r's buffer i
+            self.owner_ptrs = [[base_of[r] + ((i * self.D + self.rank) * self.chunk) * 4 for r in range(self.D)]
+                               for i in range(2)]
+            self.steps_done = 0
         self.O = torch.empty((self.batch, q_len, self.Hk, head_dim_v), dtype=torch.float32, device=self.device)
         self.LSE = torch.empty((self.batch, q_len, self.Hk), dtype=torch.float32, device=self.device)
 
@@ -121,12 +153,31 @@ class RankShardedDecode:
     def step(self, q: torch.Tensor, stream=None):
         """One decode step for the full query ``q`` (``[batch][q_len][Hq][d_qk]`` bf16 bits)."""
         d = self.desc
-        dcp.dcp_decode_partial_owner_major(d, q, self.pool, self.pool_pages, self.table, self.seq_lens_dev,
-                                           self.rank, self.D, self.D, self.send, self.workspace, stream=stream)
-        exchange(self.send, self.recv, self.group)
-        Os, Ls = split_chunks(self.recv, self.D, self.rows, d.head_dim_v)
+        if self.exchange_kind == "nccl":
+            dcp.dcp_decode_partial_owner_major(d, q, self.pool, self.pool_pages, self.table, self.seq_lens_dev,
+                                               self.rank, self.D, self.D, self.send, self.workspace, stream=stream)
+            exchange(self.send, self.recv, self.group)
+            recv = self.recv
+        else:
+            import torch.distributed as dist
+            i = self.steps_done & 1
+            self.steps_done += 1
+            dcp.dcp_decode_partial_to_owners(d, q, self.pool, self.pool_pages, self.table, self.seq_lens_dev,
+                                             self.rank, self.D, self.owner_ptrs[i], self.workspace, stream=stream)
+            # every rank's stores into this rank's chunks are complete before the merge reads them
+            (torch.cuda.current_stream(self.device) if stream is None else stream).synchronize()
+            dist.barrier(group=self.group)
+            recv = self.recv_pair[i * self.D * self.chunk:(i + 1) * self.D * self.chunk]
+        Os, Ls = split_chunks(recv, self.D, self.rows, d.head_dim_v)
         dcp.dcp_lse_merge(Os, Ls, self.D, self.rows, d.head_dim_v, self.O, self.LSE, stream=stream)
         return self.O, self.LSE
 
     def device_error(self) -> int:
         return dcp.dcp_read_device_error(self.workspace)
+
+    def close(self) -> None:
+        """Unmap the other ranks' receive buffers (p2p exchange); call on every rank before any of
+        them frees its own, e.g. followed by a barrier of the group."""
+        for base in self._mapped:
+            dcp.dcp_ipc_close(base)
+        self._mapped = []

@@ -75,6 +75,44 @@ def test_owner_major_partial_is_the_standard_partial_permuted(idx, n_owners):
     assert cache.device_error() == 0
 
 
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("n_owners", [2, 4])
+def test_partial_to_owners_writes_the_owner_major_chunks(idx, n_owners):
+    # each owner's chunk in its own allocation (on a multi-GPU run: another GPU's buffer); the rows
+    # must be the owner-major chunks, bit for bit, and nothing outside a chunk may be written
+    name, w, D, fp8 = _cases()[idx]
+    cache, q = _fp8_cache(w, D) if fp8 else build_cache(w, D)
+    d = cache.desc
+    chunk = dcp.dcp_owner_chunk_floats(d, n_owners)
+    for s in range(D):
+        send = torch.empty((n_owners * chunk,), dtype=torch.float32, device="cuda")
+        dcp.dcp_decode_partial_owner_major(d, q, cache.pools[s], int(cache.pool_pages[s]), cache.tables[s],
+                                           cache.seq_lens_dev, s, D, n_owners, send, cache.workspace)
+        # guard bands around every chunk
+        bufs = [torch.full((chunk + 128,), float("nan"), dtype=torch.float32, device="cuda") for _ in range(n_owners)]
+        dcp.dcp_decode_partial_to_owners(d, q, cache.pools[s], int(cache.pool_pages[s]), cache.tables[s],
+                                         cache.seq_lens_dev, s, D, [b[64:64 + chunk] for b in bufs], cache.workspace)
+        torch.cuda.synchronize()
+        rows = w.batch * w.q_len * (w.num_q_heads // n_owners)
+        used = rows * w.head_dim_v + rows  # O rows, then LSE rows (the padding is never written)
+        for k in range(n_owners):
+            got = bufs[k][64:64 + used]
+            assert torch.equal(got, send[k * chunk:k * chunk + used]), f"{name} shard {s} owner {k}"
+            assert torch.isnan(bufs[k][:64]).all() and torch.isnan(bufs[k][64 + used:]).all()
+    assert cache.device_error() == 0
+
+
+def test_partial_to_owners_rejects_misaligned_chunks():
+    w = synth.custom(synth.GQA, [100], 8, 2, 64, 64, 16, seed=71)
+    cache, q = build_cache(w, 1)
+    chunk = dcp.dcp_owner_chunk_floats(cache.desc, 2)
+    buf = torch.empty(2 * chunk + 8, dtype=torch.float32, device="cuda")
+    with pytest.raises(dcp.DcpError) as e:
+        dcp.dcp_decode_partial_to_owners(cache.desc, q, cache.pools[0], int(cache.pool_pages[0]), cache.tables[0],
+                                         cache.seq_lens_dev, 0, 1, [buf[1:], buf[chunk + 4:]], cache.workspace)
+    assert e.value.status == dcp.DCP_ERR_INVALID_ARG
+
+
 def test_owner_major_rejects_uneven_owners():
     w = synth.custom(synth.GQA, [100], 8, 2, 64, 64, 16, seed=65)
     cache, q = build_cache(w, 1)

@@ -151,7 +151,9 @@ using namespace dcp;
 
 extern "C" {
 
-int32_t dcp_version(void) { return 200; }  // 0.2.0: q_len, kv_dtype, scales and shard_rule in dcp_attn_desc
+// 0.2.0: q_len, kv_dtype, scales and shard_rule in dcp_attn_desc; 0.3.0: FP8 pools for every layout,
+// dcp_decode_partial_to_owners and the CUDA IPC helpers
+int32_t dcp_version(void) { return 300; }
 
 const char* dcp_status_string(dcp_status s) {
   switch (s) {

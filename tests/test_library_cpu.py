@@ -34,6 +34,17 @@ def test_library_exports_every_declared_symbol():
     assert dcp.dcp_version() >= 100
 
 
+def test_ipc_helpers_check_their_arguments_on_the_host():
+    # a CUDA IPC handle is 64 bytes; null arguments come back as status codes before any CUDA call
+    assert dcp.dcp_ipc_handle_bytes() == 64
+    lib = ctypes.CDLL(dcp.LIB_PATH)
+    off = ctypes.c_uint64(0)
+    buf = ctypes.create_string_buffer(64)
+    assert lib.dcp_ipc_export(None, buf, ctypes.byref(off)) == dcp.DCP_ERR_INVALID_ARG
+    assert lib.dcp_ipc_open(None, ctypes.byref(ctypes.c_void_p())) == dcp.DCP_ERR_INVALID_ARG
+    assert lib.dcp_ipc_close(None) == dcp.DCP_ERR_INVALID_ARG
+
+
 @pytest.mark.parametrize("D", [1, 2, 3, 4, 8, 16])
 @pytest.mark.parametrize("bs", [16, 64])
 @pytest.mark.parametrize("perm", [0, 99])

@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(mla_threads<KV8>(), 1) mla_decode_kernel(const
         const float mh = misc->mref[ts];
         misc->inv_l[ts] = lt > 0.f ? (KV8 ? p.v_scale / lt : 1.f / lt) : 0.f;
         misc->lse2[ts] = lt > 0.f ? mh + __log2f(lt) : -INFINITY;
-        // row offsets once per piece, so that the stores below need no owner arithmetic
+        // row pointers once per piece, so that the stores below need no owner arithmetic
         misc->rowptr[ts] = complete ? o_row(ts) : slot_base + (size_t)ts * kMlaDv;
       }
       named_bar_sync(2, kSoftmaxThreads);

@@ -111,6 +111,34 @@ def test_decode_parity_unit_scale_and_contiguous_rule():
         _check(w, 3, cache, 1.0, rule)
 
 
+def test_decode_parity_with_saturated_codes():
+    # scale 2^-9: values past 448 * 2^-9 = 0.875 saturate to the largest code, as the oracle's cache
+    # write does -- the decode must see exactly those values
+    w = synth.custom(synth.MLA, [700, 64, 2000], 64, 1, 576, 512, 64, seed=93)
+    scale = 2.0 ** -9
+    cache, q = _cache(w, 2, scale)
+    codes = np.concatenate([p.cpu().numpy().view(np.uint8) for p in cache.pools])
+    assert ((codes & 0x7F) == 0x7E).sum() > 1000  # many saturated codes
+    cache.step(q)
+    torch.cuda.synchronize()
+    _check(w, 2, cache, scale)
+
+
+def test_out_of_pool_page_is_flagged_and_skipped():
+    # one table entry of request 1 names a page past its pool: the page is never loaded or widened,
+    # status bit 0 is set, every output stays finite and the other requests are exact
+    w = synth.custom(synth.MLA, [900, 600, 1300], 64, 1, 576, 512, 64, seed=94)
+    D = 2
+    cache, q = _cache(w, D, 0.05)
+    t = cache.tables[1]
+    t[1, 2] = int(cache.pool_pages[1]) + 7
+    cache.step(q)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 1
+    assert torch.isfinite(cache.O).all() and torch.isfinite(cache.LSE).all()
+    _check(w, D, cache, 0.05, requests=[0, 2])
+
+
 def test_wide_score_range():
     # query amplitude 8: scores spread far, so reference raises and O^T rescales happen mid-piece
     w = synth.custom(synth.MLA, [3000, 900], 64, 1, 576, 512, 64, seed=91, q_amp=8.0)

@@ -30,7 +30,11 @@
  *     scaled scores; each partial O_i is normalised by its own sum;
  *   - an empty token set has O = 0 and LSE = -inf and carries merge weight 0;
  *   - MLA: a token's key is its whole latent row (d_qk wide), its value is
- *     the first d_v entries of the same row.
+ *     the first d_v entries of the same row;
+ *   - an FP8 (E4M3) cache holds code = e4m3(float32(x) * float32(1/scale)),
+ *     standing for scale * e4m3_value(code), with one scale for GQA keys,
+ *     one for GQA values, and one for the whole MLA latent row (the latent
+ *     is a single tensor read as key and value).
  */
 #include <math.h>
 #include <stdint.h>

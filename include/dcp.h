@@ -368,11 +368,14 @@ DCP_API dcp_status dcp_decode_partial_to_owners(const dcp_attn_desc *desc, const
  * Mapping a device buffer of another process (CUDA IPC), for owner chunks on
  * other GPUs.  [The multi-GPU form above; the pages name no mechanism.]
  *   dcp_ipc_handle_bytes  size of a handle (host bytes).
- *   dcp_ipc_export        device_ptr: device memory of this process.  Writes the
- *                         handle of the allocation that holds it to handle_out
- *                         (host, dcp_ipc_handle_bytes()) and device_ptr's byte
- *                         offset inside that allocation to *offset_out.
- *                         DCP_ERR_INVALID_ARG if device_ptr is not device memory.
+ *   dcp_ipc_export        device_ptr: device memory of this process from
+ *                         cudaMalloc (e.g. PyTorch's default caching allocator;
+ *                         not stream-ordered pool memory).  Writes the handle of
+ *                         the allocation that holds it to handle_out (host,
+ *                         dcp_ipc_handle_bytes()) and device_ptr's byte offset
+ *                         inside that allocation to *offset_out.
+ *                         DCP_ERR_INVALID_ARG if device_ptr is not device memory;
+ *                         DCP_ERR_CUDA if its allocation cannot be exported.
  *   dcp_ipc_open          maps the allocation a handle names (from another
  *                         process; peer access is enabled when needed) and
  *                         returns its base in *base_out; the buffer is at

@@ -71,6 +71,17 @@ def split_chunks(buf: torch.Tensor, D: int, rows: int, head_dim_v: int):
     return Os, Ls
 
 
+def owner_chunk_addresses(recv_bases, rank: int, chunk_floats: int, parity: int):
+    """Where rank ``rank``'s decode kernel stores each owner's rows in the folded exchange.
+
+    ``recv_bases[r]`` is the address (in this process) of rank r's pair of receive buffers, each
+    D chunks of ``chunk_floats`` fp32; step parity ``parity`` uses buffer 0 or 1.  Owner r takes
+    this shard's rows as chunk ``rank`` of its buffer, so after the step owner r's buffer holds
+    every shard's rows for its heads in shard order -- the layout ``split_chunks`` reads."""
+    D = len(recv_bases)
+    return [recv_bases[r] + ((parity * D + rank) * chunk_floats) * 4 for r in range(D)]
+
+
 class RankShardedDecode:
     """Shard ``rank`` of a D-rank DCP group (D = the group's size) on this process's GPU.
 
@@ -134,9 +145,8 @@ class RankShardedDecode:
                     mapped = dcp.dcp_ipc_open(h)
                     self._mapped.append(mapped)
                     base_of[r] = mapped + off
-            # step parity i, owner r: chunk `rank` of owner r's buffer i
-            self.owner_ptrs = [[base_of[r] + ((i * self.D + self.rank) * self.chunk) * 4 for r in range(self.D)]
-                               for i in range(2)]
+            bases = [base_of[r] for r in range(self.D)]
+            self.owner_ptrs = [owner_chunk_addresses(bases, self.rank, self.chunk, i) for i in range(2)]
             self.steps_done = 0
         self.O = torch.empty((self.batch, q_len, self.Hk, head_dim_v), dtype=torch.float32, device=self.device)
         self.LSE = torch.empty((self.batch, q_len, self.Hk), dtype=torch.float32, device=self.device)

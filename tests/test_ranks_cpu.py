@@ -155,3 +155,29 @@ def test_chunk_size_matches_the_library():
         assert dcp.dcp_owner_chunk_floats(desc, n) % 64 == 0 or (B * ql * Hq // n * d_v) % 4 == 0
     desc = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 2, 8, 2, 64, 64, 16, 4, 0.1)
     assert dcp.dcp_owner_chunk_floats(desc, 3) == 0  # 3 owners do not split 8 heads
+
+
+def test_folded_exchange_addresses_assemble_the_owner_layout():
+    # emulate D ranks' receive buffers as numpy arrays at fake base addresses: every rank "stores"
+    # its owner-major chunks at the addresses owner_chunk_addresses gives; each owner's buffer must
+    # then hold, chunk by chunk in shard order, the rows it merges -- for both step parities
+    from sequence_sharded_decode_paged_b200.ranks import owner_chunk_addresses, split_chunks
+    D, rows, dv = 3, 5, 4
+    chunk = rows * dv + 64  # O rows, then LSE rows padded to 64 floats
+    bases = [(1 << 40) * (r + 1) for r in range(D)]
+    bufs = [np.full(2 * D * chunk, np.nan, dtype=np.float32) for _ in range(D)]
+    for parity in (0, 1):
+        for shard in range(D):
+            for owner, addr in enumerate(owner_chunk_addresses(bases, shard, chunk, parity)):
+                r = next(k for k in range(D) if bases[k] <= addr < bases[k] + bufs[k].nbytes)
+                assert r == owner
+                off = (addr - bases[r]) // 4
+                vals = np.arange(chunk, dtype=np.float32) + 1000 * shard + 100 * owner + 10 * parity
+                bufs[r][off:off + chunk] = vals
+        for owner in range(D):
+            half = torch.from_numpy(bufs[owner][parity * D * chunk:(parity + 1) * D * chunk].copy())
+            Os, Ls = split_chunks(half, D, rows, dv)
+            for shard in range(D):
+                base = 1000 * shard + 100 * owner + 10 * parity
+                assert torch.equal(Os[shard].reshape(-1), torch.arange(rows * dv, dtype=torch.float32) + base)
+                assert torch.equal(Ls[shard], torch.arange(rows * dv, rows * dv + rows, dtype=torch.float32) + base)

@@ -46,7 +46,10 @@ dcp_status dcp_ipc_export(const void* device_ptr, void* handle_out, uint64_t* of
   if (fn(&base, CU_POINTER_ATTRIBUTE_RANGE_START_ADDR, reinterpret_cast<CUdeviceptr>(device_ptr)) != CUDA_SUCCESS)
     return DCP_ERR_INVALID_ARG;  // not device memory of this process
   cudaIpcMemHandle_t h;
-  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return DCP_ERR_CUDA;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) {
+    cudaGetLastError();  // do not leave the failure to be reported by the next launch check
+    return DCP_ERR_CUDA;
+  }
   memcpy(handle_out, &h, sizeof(h));
   *offset_out = (uint64_t)(reinterpret_cast<CUdeviceptr>(device_ptr) - base);
   return DCP_OK;
@@ -57,14 +60,21 @@ dcp_status dcp_ipc_open(const void* handle, void** base_out) {
   cudaIpcMemHandle_t h;
   memcpy(&h, handle, sizeof(h));
   void* p = nullptr;
-  if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return DCP_ERR_CUDA;
+  if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    return DCP_ERR_CUDA;
+  }
   *base_out = p;
   return DCP_OK;
 }
 
 dcp_status dcp_ipc_close(void* base) {
   if (base == nullptr) return DCP_ERR_INVALID_ARG;
-  return cudaIpcCloseMemHandle(base) == cudaSuccess ? DCP_OK : DCP_ERR_CUDA;
+  if (cudaIpcCloseMemHandle(base) != cudaSuccess) {
+    cudaGetLastError();
+    return DCP_ERR_CUDA;
+  }
+  return DCP_OK;
 }
 
 }  // extern "C"

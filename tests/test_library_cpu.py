@@ -34,6 +34,27 @@ def test_library_exports_every_declared_symbol():
     assert dcp.dcp_version() >= 100
 
 
+def test_owner_calls_check_their_arguments_on_the_host():
+    # refused before anything is launched (fake, aligned device addresses; no GPU needed): more than 16
+    # owners, a null or misaligned owner chunk
+    lib = ctypes.CDLL(dcp.LIB_PATH)
+    desc = dcp.make_desc(dcp.DCP_LAYOUT_GQA, 2, 32, 4, 64, 64, 16, 8, 0.125)
+    fake = [0x10000 * (i + 1) for i in range(8)]
+    args = lambda n_owners, chunks: (ctypes.byref(desc), fake[0], fake[1], 4, fake[2], fake[3], 0, 1, n_owners,
+                                     chunks, fake[4], 1 << 40, None)
+    to_owners = lib.dcp_decode_partial_to_owners
+    to_owners.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int32] + [ctypes.c_void_p] * 2 + [ctypes.c_int32] * 3 + \
+        [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    ptrs = lambda xs: (ctypes.c_void_p * len(xs))(*xs)
+    assert to_owners(*args(32, ptrs([fake[5]] * 32))) == dcp.DCP_ERR_INVALID_ARG   # 32 owners > 16
+    assert to_owners(*args(2, ptrs([fake[5], 0]))) == dcp.DCP_ERR_INVALID_ARG       # null chunk
+    assert to_owners(*args(2, ptrs([fake[5], fake[6] + 4]))) == dcp.DCP_ERR_INVALID_ARG  # misaligned chunk
+    assert to_owners(*args(3, ptrs([fake[5]] * 3))) == dcp.DCP_ERR_INVALID_ARG      # 3 does not divide 32 heads
+    major = lib.dcp_decode_partial_owner_major
+    major.argtypes = to_owners.argtypes
+    assert major(*args(32, fake[5])) == dcp.DCP_ERR_INVALID_ARG                      # 32 owners > 16
+
+
 def test_ipc_helpers_check_their_arguments_on_the_host():
     # a CUDA IPC handle is 64 bytes; null arguments come back as status codes before any CUDA call
     assert dcp.dcp_ipc_handle_bytes() == 64
